@@ -1,0 +1,151 @@
+/*
+ * ck.h -- C ABI of the ConvRot W4A4 quantized linear for NVIDIA B200 (sm_100a).
+ *
+ * The operation (comfy-kitchen PR #198 "Consolidate INT8, RotateQuant, RoPE and
+ * ConvRot W4A4 backends", section "W4A4 correctness and performance scope"; PR #201
+ * "Avoid activation pack/unpack in ConvRot W4A4", section "Summary"):
+ *
+ *   stage 1  y[m, j*g + c] = sum_i x[m, j*g + i] * R[i, c]     (rotation per K-group,
+ *                                                               result in x's dtype)
+ *            s[m] = max(fp32(max_k |y[m, k]|) / 7, FLT_MIN)    (per-row scale)
+ *            q[m, k] = clamp(round_half_even(y[m, k] / s[m]), -8, 7)   (INT8 storage)
+ *   stage 2  acc[m, n] = sum_k q[m, k] * w[n, k]               (exact INT32)
+ *            out[m, n] = cvt(((fp32(acc) * s[m]) * w_scale[n]) + bias[n])
+ *
+ * where w[n, k] are signed 4-bit weight codes packed two per byte, (N, K/2), the
+ * even k in the low nibble (comfy_kitchen/tensor/svdquant_w4a4.py module docstring
+ * for the (N, K // 2) layout).
+ *
+ * Conventions for every entry point:
+ *   - All data pointers are DEVICE pointers owned by the caller; the library
+ *     allocates no memory and keeps no state between calls (except cached kernel
+ *     attributes and a per-process table of driver entry points).
+ *   - Work is enqueued on `stream`; the call returns before the GPU finishes.
+ *   - Arguments are validated on the host before anything is launched; an invalid
+ *     call returns an error and touches no memory.
+ *   - Strides and leading dimensions are in ELEMENTS of the tensor they describe
+ *     (bytes for int8 tensors).
+ *   - M == 0 is a successful no-op ("empty rows").
+ *   - dev_status, when not NULL, is a device int that a kernel sets to
+ *     CK_ERR_TIMEOUT if one of its bounded internal waits expires (the kernel then
+ *     exits early and its outputs are undefined).  The caller clears it and reads
+ *     it after synchronising the stream.
+ */
+#ifndef CK_H
+#define CK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CK_OK = 0,
+    CK_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad dtype, bad group size        */
+    CK_ERR_UNSUPPORTED = 2,   /* a valid call this build does not implement               */
+    CK_ERR_OVERFLOW = 3,      /* 64 * K > INT32_MAX: the INT32 accumulator could overflow */
+    CK_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required               */
+    CK_ERR_CUDA = 5,          /* a CUDA runtime/driver call or a launch failed            */
+    CK_ERR_TIMEOUT = 6        /* written to *dev_status by a kernel whose wait expired    */
+} ck_status;
+
+typedef enum { CK_F32 = 0, CK_F16 = 1, CK_BF16 = 2, CK_I8 = 3 } ck_dtype;
+
+/*
+ * Stage 1: group-wise rotation, then row-wise signed-INT4 quantization with codes
+ * kept in INT8 storage (PR #198 "W4A4 correctness and performance scope": rotation
+ * keeps the FP32/FP16/BF16 input dtype, the reference signed-INT4 quantizer; PR #201
+ * "Summary": codes are never packed; PR #155 "Add fused RotateQuant backend": group
+ * sizes 16/64/256, batched / non-contiguous inputs, asymmetric rotations, zero-scale
+ * handling).
+ *
+ *   x        (M, K) activations of x_dtype (CK_F32, CK_F16 or CK_BF16), element
+ *            (m, k) at x[m*stride_m + k*stride_k]; any strides (row pitch, transposed
+ *            views).  A batched (..., K) tensor is passed as its flattened 2-D view.
+ *   R        (g, g) row-major rotation in x_dtype; y_group = x_group @ R.
+ *   g        16, 64 or 256; K must be a positive multiple of g (and so even).
+ *   scale_in NULL: dynamic per-row scales.  Otherwise a device pointer to ONE fp32
+ *            tensor-wise scale used for every row after the same lower clamp at
+ *            FLT_MIN (a zero scale becomes FLT_MIN, as the eager path does).
+ *   codes    (M, K) int8 output, row pitch ldq >= K bytes; values in [-8, 7].
+ *   scales   (M,) fp32 output, the scale each row was divided by (always written).
+ *
+ * Accumulation is fp32 and the rotated value is rounded to x_dtype before the
+ * absmax, so a code may differ by one from an exact-arithmetic evaluation where
+ * y / s lies within rounding of a half-integer.
+ * Errors: CK_ERR_INVALID_ARG (null x/R/codes/scales, M < 0, K <= 0, K % g != 0,
+ * bad g or dtype, ldq < K), CK_ERR_CUDA (launch failure).
+ */
+ck_status ck_rotate_quant(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                          int64_t stride_m, int64_t stride_k, const void* R, int g,
+                          const float* scale_in, int8_t* codes, int64_t ldq, float* scales,
+                          int* dev_status, cudaStream_t stream);
+
+/*
+ * The whole W4A4 linear (PR #198 "W4A4 correctness and performance scope": INT8
+ * codes contracted with npu_quant_matmul-style INT32 accumulation at unit scale,
+ * then cast, activation scale, weight scale and bias in eager's order, with an
+ * INT32 overflow guard).
+ *
+ *   x, x_dtype, M, K, stride_m, stride_k, R, g
+ *            as in ck_rotate_quant when x_dtype is CK_F32/CK_F16/CK_BF16: stage 1
+ *            runs into the workspace, then stage 2.
+ *            When x_dtype == CK_I8, x already holds (M, K) int8 codes with row pitch
+ *            stride_m (stride_k must be 1), a_scale holds their (M,) fp32 row scales,
+ *            and R/g are ignored: the GEMM-only path.
+ *   a_scale  (M,) fp32 row scales for CK_I8 input; ignored (may be NULL) otherwise.
+ *   w_packed (N, K/2) int8, row pitch w_ld >= K/2 bytes, two signed 4-bit codes per
+ *            byte, code of k = 2i in the low nibble of byte i.
+ *   w_scale  (N,) per-output-channel weight scale, scale_dtype (CK_F32/F16/BF16).
+ *   bias     (N,) of scale_dtype, or NULL.
+ *   out      (M, N) of out_dtype (CK_F32/F16/BF16), row pitch ldo >= N.
+ *   workspace, workspace_bytes
+ *            caller-owned device scratch of at least
+ *            ck_w4a4_linear_workspace_bytes(M, N, K, w_ld) bytes, 256-byte aligned.
+ *            After a floating-point-input call it holds the stage-1 result: int8
+ *            codes (M, K) with row pitch ck_workspace_codes_pitch(K) at offset 0,
+ *            then fp32 row scales (M,) at offset ck_workspace_scales_offset(M, K).
+ *
+ * Errors: CK_ERR_INVALID_ARG, CK_ERR_OVERFLOW (64*K > 2^31 - 1, the bound
+ * |acc| <= 8*8*K), CK_ERR_WORKSPACE, CK_ERR_CUDA.
+ */
+ck_status ck_w4a4_linear(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                         int64_t stride_m, int64_t stride_k, const void* R, int g,
+                         const float* a_scale, const int8_t* w_packed, int64_t N, int64_t w_ld,
+                         const void* w_scale, ck_dtype scale_dtype, const void* bias,
+                         void* out, ck_dtype out_dtype, int64_t ldo,
+                         void* workspace, size_t workspace_bytes, int* dev_status,
+                         cudaStream_t stream);
+
+/* Workspace ck_w4a4_linear needs for these sizes: the stage-1 codes and scales (also
+ * used to re-pitch CK_I8 codes whose rows are not 16-byte aligned) and, when w_ld is
+ * not a multiple of 16, a 16-byte-pitched copy of the packed weights.  Assumes a
+ * 16-byte aligned w_packed.  Returns 0 for invalid sizes. */
+size_t ck_w4a4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t w_ld);
+
+/* Layout of the stage-1 result inside the workspace (see ck_w4a4_linear). */
+int64_t ck_workspace_codes_pitch(int64_t K);
+size_t ck_workspace_scales_offset(int64_t M, int64_t K);
+
+/*
+ * Weight unpack (PR #198: the W4 codes are unpacked to INT8; PR #201: only weights
+ * are unpacked): packed (N, K/2) int8 with row pitch ld_packed bytes ->
+ * out (N, K) int8 sign-extended codes in [-8, 7], row pitch ld_out bytes.
+ * Bit-exact.  Errors: CK_ERR_INVALID_ARG (null pointers, N < 0, K <= 0 or odd,
+ * ld_packed < K/2, ld_out < K), CK_ERR_CUDA.
+ */
+ck_status ck_unpack_w4(const int8_t* packed, int64_t N, int64_t K, int64_t ld_packed,
+                       int8_t* out, int64_t ld_out, cudaStream_t stream);
+
+/* Static description of a status code (never NULL). */
+const char* ck_status_string(ck_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CK_H */

@@ -1,0 +1,163 @@
+"""Thin Python binding over libck.so (include/ck.h): argument marshalling only.
+
+Each function takes CUDA torch tensors, passes their device pointers, sizes and
+strides to the C entry point of the same name, and raises CkError on a non-OK
+status.  Every step of the computation runs in the library's CUDA kernels; there is
+no CPU path.  Loading fails loudly if libck.so has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libck.so")
+
+CK_OK, CK_ERR_INVALID_ARG, CK_ERR_UNSUPPORTED, CK_ERR_OVERFLOW = 0, 1, 2, 3
+CK_ERR_WORKSPACE, CK_ERR_CUDA, CK_ERR_TIMEOUT = 4, 5, 6
+CK_F32, CK_F16, CK_BF16, CK_I8 = 0, 1, 2, 3
+
+DTYPE_CODE = {torch.float32: CK_F32, torch.float16: CK_F16, torch.bfloat16: CK_BF16,
+              torch.int8: CK_I8}
+CODE_DTYPE = {v: k for k, v in DTYPE_CODE.items()}
+
+# every entry point include/ck.h declares, with its ctypes signature
+_P, _I64, _I, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = {
+    "ck_rotate_quant": ([_P, _I, _I64, _I64, _I64, _I64, _P, _I, _P, _P, _I64, _P, _P, _P], _I),
+    "ck_w4a4_linear": ([_P, _I, _I64, _I64, _I64, _I64, _P, _I, _P, _P, _I64, _I64, _P, _I, _P,
+                        _P, _I, _I64, _P, _SZ, _P, _P], _I),
+    "ck_w4a4_linear_workspace_bytes": ([_I64, _I64, _I64, _I64], _SZ),
+    "ck_workspace_codes_pitch": ([_I64], _I64),
+    "ck_workspace_scales_offset": ([_I64, _I64], _SZ),
+    "ck_unpack_w4": ([_P, _I64, _I64, _I64, _P, _I64, _P], _I),
+    "ck_status_string": ([_I], ctypes.c_char_p),
+}
+
+
+class CkError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libck.so (raises if it is missing: build it with the package's build module)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libck.so not found at {LIB_PATH}; run "
+                              "`python -m rotated_w4a4_quantized_group_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().ck_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != CK_OK:
+        raise CkError(status, where)
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def workspace_bytes(M: int, N: int, K: int, w_ld: int) -> int:
+    return int(lib().ck_w4a4_linear_workspace_bytes(M, N, K, w_ld))
+
+
+def workspace_codes_pitch(K: int) -> int:
+    return int(lib().ck_workspace_codes_pitch(K))
+
+
+def workspace_scales_offset(M: int, K: int) -> int:
+    return int(lib().ck_workspace_scales_offset(M, K))
+
+
+def _check_rotation(x: torch.Tensor, R: torch.Tensor, g: int):
+    # the C ABI reads R as g*g row-major elements of x's dtype
+    if tuple(R.shape) != (g, g) or R.dtype != x.dtype or not R.is_contiguous():
+        raise ValueError(f"R must be a contiguous ({g}, {g}) tensor of {x.dtype}; got "
+                         f"{tuple(R.shape)} {R.dtype} strides {R.stride()}")
+
+
+def ck_rotate_quant(x: torch.Tensor, R: torch.Tensor, g: int, scale_in: torch.Tensor | None = None,
+                    codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                    dev_status: torch.Tensor | None = None, stream=None):
+    """Stage 1 on a 2-D (M, K) CUDA view; returns (codes int8 (M, K), scales fp32 (M,))."""
+    M, K = x.shape
+    _check_rotation(x, R, g)
+    if codes is None:
+        codes = torch.empty(M, K, dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty(M, dtype=torch.float32, device=x.device)
+    st = lib().ck_rotate_quant(_ptr(x), DTYPE_CODE[x.dtype], M, K, x.stride(0), x.stride(1),
+                               _ptr(R), g, _ptr(scale_in), _ptr(codes), codes.stride(0),
+                               _ptr(scales), _ptr(dev_status), _stream(stream))
+    _check(st, "ck_rotate_quant")
+    return codes, scales
+
+
+def ck_w4a4_linear(x: torch.Tensor, R: torch.Tensor | None, g: int, w_packed: torch.Tensor,
+                   w_scale: torch.Tensor, bias: torch.Tensor | None = None, *,
+                   a_scale: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                   out_dtype: torch.dtype | None = None, workspace: torch.Tensor | None = None,
+                   dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The whole W4A4 linear.  x is (M, K) activations (fp32/fp16/bf16) or int8 codes (with
+    a_scale); w_packed is (N, K/2) int8.  Returns out (M, N)."""
+    M, K = x.shape
+    N = w_packed.shape[0]
+    if x.dtype != torch.int8:
+        _check_rotation(x, R, g)
+    if w_packed.stride(1) != 1 or tuple(w_packed.shape) != (N, K // 2):
+        raise ValueError("w_packed must be (N, K/2) with unit inner stride")
+    if out is None:
+        odt = out_dtype or (x.dtype if x.dtype != torch.int8 else w_scale.dtype)
+        out = torch.empty(M, N, dtype=odt, device=x.device)
+    if workspace is None:
+        nbytes = workspace_bytes(M, N, K, w_packed.stride(0))
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+    st = lib().ck_w4a4_linear(
+        _ptr(x), DTYPE_CODE[x.dtype], M, K, x.stride(0), x.stride(1), _ptr(R), int(g),
+        _ptr(a_scale), _ptr(w_packed), N, w_packed.stride(0), _ptr(w_scale),
+        DTYPE_CODE[w_scale.dtype], _ptr(bias), _ptr(out), DTYPE_CODE[out.dtype], out.stride(0),
+        _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream))
+    _check(st, "ck_w4a4_linear")
+    return out
+
+
+def ck_unpack_w4(packed: torch.Tensor, K: int, out: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """(N, K/2) packed int8 -> (N, K) int8 codes."""
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty(N, K, dtype=torch.int8, device=packed.device)
+    st = lib().ck_unpack_w4(_ptr(packed), N, K, packed.stride(0), _ptr(out), out.stride(0),
+                            _stream(stream))
+    _check(st, "ck_unpack_w4")
+    return out

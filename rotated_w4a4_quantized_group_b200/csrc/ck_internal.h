@@ -1,0 +1,42 @@
+// ck_internal.h -- host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime_api.h>
+#include <stdint.h>
+
+#include "ck.h"
+
+namespace ck {
+
+// Encode a tiled TMA descriptor through the driver entry point (no -lcuda link).
+// Returns CK_ERR_CUDA if the driver call fails.
+ck_status encode_tma(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                     const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                     CUtensorMapSwizzle swizzle);
+
+int num_sms();
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Stage 1 launch (arguments already validated).
+ck_status launch_rotate_quant(const void* x, ck_dtype dt, int64_t M, int64_t K, int64_t sm,
+                              int64_t sk, const void* R, int g, const float* scale_in,
+                              int8_t* codes, int64_t ldq, float* scales, int* dev_status,
+                              cudaStream_t stream);
+
+// Stage 2 launch: codes (M, K) int8 with 16-byte-aligned rows (ldq % 16 == 0), packed
+// weights with 16-byte-aligned rows (w_ld % 16 == 0).
+ck_status launch_w4a4_gemm(const int8_t* codes, int64_t ldq, const float* a_scale, int64_t M,
+                           int64_t K, const int8_t* w_packed, int64_t w_ld, int64_t N,
+                           const void* w_scale, ck_dtype scale_dt, const void* bias, void* out,
+                           ck_dtype out_dt, int64_t ldo, int* dev_status, cudaStream_t stream);
+
+ck_status launch_unpack_w4(const int8_t* packed, int64_t N, int64_t K, int64_t ld_packed,
+                           int8_t* out, int64_t ld_out, cudaStream_t stream);
+
+// Copy a (rows, cols) byte matrix between pitches (used to re-pitch misaligned inputs).
+ck_status launch_copy_rows(const int8_t* src, int64_t ld_src, int8_t* dst, int64_t ld_dst,
+                           int64_t rows, int64_t cols, cudaStream_t stream);
+
+}  // namespace ck

@@ -1,0 +1,494 @@
+// ck_rotate_quant.cu -- stage 1: group-wise rotation in the input dtype, then row-wise
+// signed-INT4 quantization with the codes kept in INT8 storage.
+//
+// Operation (comfy-kitchen PR #198 "Consolidate INT8, RotateQuant, RoPE and ConvRot W4A4
+// backends", "W4A4 correctness and performance scope"; PR #201 "Avoid activation
+// pack/unpack in ConvRot W4A4", "Summary"; PR #155 "Add fused RotateQuant backend"):
+//   y[m, j*g + c] = dtype( sum_i x[m, j*g + i] * R[i, c] )      (fp32 accumulation)
+//   s[m] = max(fp32(max_k |y[m, k]|) / 7, FLT_MIN)   or the caller's tensor-wise scale
+//   q[m, k] = clamp(round_half_even(y[m, k] / s[m]), -8, 7)
+//
+// Two kernels:
+//   rq_mma_kernel      bf16/fp16, g in {16, 64}, unit K stride, 16-byte aligned rows.
+//                      A block of rows arrives by one TMA tensor copy (swizzled, so the
+//                      warp-level MMA fragment loads are bank-conflict free), is rotated
+//                      in place by mma.sync with R held in registers, and then quantized
+//                      from shared memory with 16-byte coalesced code stores.
+//   rq_generic_kernel  every dtype, g and stride: one row per CTA step, fp32 FFMA with R
+//                      in shared memory (or read through L1 when it does not fit).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <float.h>
+#include <stdint.h>
+
+#include "ck_device.cuh"
+#include "ck_internal.h"
+
+namespace ck {
+
+// ===================================================================== generic kernel
+
+constexpr int kGenThreads = 256;
+constexpr int kGenMaxChunks = 16;  // 4-wide chunks kept in registers per thread: K <= 16384
+
+template <typename T>
+__device__ __forceinline__ float4 load4(const T* p);
+template <>
+__device__ __forceinline__ float4 load4<float>(const float* p) {
+    return *reinterpret_cast<const float4*>(p);
+}
+template <>
+__device__ __forceinline__ float4 load4<__half>(const __half* p) {
+    uint2 u = *reinterpret_cast<const uint2*>(p);
+    float2 a = __half22float2(*reinterpret_cast<__half2*>(&u.x));
+    float2 b = __half22float2(*reinterpret_cast<__half2*>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+template <>
+__device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p) {
+    uint2 u = *reinterpret_cast<const uint2*>(p);
+    float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.x));
+    float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+// One rotated 4-wide chunk: columns c0..c0+3 of group j, rounded to T.
+template <typename T>
+__device__ __forceinline__ float4 rotate_chunk(const float* xs, const T* Rp, int g, int64_t k0) {
+    const int64_t j0 = (k0 / g) * g;
+    const int c0 = (int)(k0 - j0);
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    for (int i = 0; i < g; ++i) {
+        const float xv = xs[j0 + i];
+        const float4 r = load4<T>(Rp + (int64_t)i * g + c0);
+        a0 = fmaf(xv, r.x, a0);
+        a1 = fmaf(xv, r.y, a1);
+        a2 = fmaf(xv, r.z, a2);
+        a3 = fmaf(xv, r.w, a3);
+    }
+    return make_float4(round_through<T>(a0), round_through<T>(a1), round_through<T>(a2),
+                       round_through<T>(a3));
+}
+
+__device__ __forceinline__ float amax4(float m, float4 v) {
+    m = fmax_nan(m, fabsf(v.x));
+    m = fmax_nan(m, fabsf(v.y));
+    m = fmax_nan(m, fabsf(v.z));
+    return fmax_nan(m, fabsf(v.w));
+}
+
+__device__ __forceinline__ void store_codes4(int8_t* dst, float4 v, float s, bool vec) {
+    const int q0 = quant_code(v.x, s), q1 = quant_code(v.y, s), q2 = quant_code(v.z, s),
+              q3 = quant_code(v.w, s);
+    if (vec) {
+        uint32_t p = (uint32_t)(q0 & 0xFF) | ((uint32_t)(q1 & 0xFF) << 8) |
+                     ((uint32_t)(q2 & 0xFF) << 16) | ((uint32_t)(q3 & 0xFF) << 24);
+        *reinterpret_cast<uint32_t*>(dst) = p;
+    } else {
+        dst[0] = (int8_t)q0;
+        dst[1] = (int8_t)q1;
+        dst[2] = (int8_t)q2;
+        dst[3] = (int8_t)q3;
+    }
+}
+
+__device__ __forceinline__ float row_scale(float amax, const float* scale_in) {
+    float s = scale_in ? *scale_in : __fdiv_rn(amax, 7.0f);
+    return (s < FLT_MIN) ? FLT_MIN : s;   // lower clamp; NaN stays NaN
+}
+
+template <typename T, bool kKeep>
+__global__ void __launch_bounds__(kGenThreads)
+    rq_generic_kernel(const T* __restrict__ x, int64_t M, int64_t K, int64_t sm, int64_t sk,
+                      const T* __restrict__ R, int g, int r_in_smem,
+                      const float* __restrict__ scale_in, int8_t* __restrict__ codes, int64_t ldq,
+                      float* __restrict__ scales, int vec_codes) {
+    extern __shared__ __align__(16) unsigned char gen_smem[];
+    float* xs = reinterpret_cast<float*>(gen_smem);
+    T* Rs = reinterpret_cast<T*>(xs + K);
+    __shared__ float warp_max[kGenThreads / 32];
+
+    const int tid = threadIdx.x;
+    if (r_in_smem)
+        for (int i = tid; i < g * g; i += kGenThreads) Rs[i] = R[i];
+    const T* Rp = r_in_smem ? Rs : R;
+    const int64_t nchunk = K / 4;
+
+    for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+        __syncthreads();
+        const T* xr = x + m * sm;
+        for (int64_t k = tid; k < K; k += kGenThreads) xs[k] = Elem<T>::to_f(xr[k * sk]);
+        __syncthreads();
+
+        float4 keep[kKeep ? kGenMaxChunks : 1];
+        float mx = 0.f;
+        if (kKeep) {
+#pragma unroll
+            for (int it = 0; it < kGenMaxChunks; ++it) {
+                const int64_t ci = tid + (int64_t)it * kGenThreads;
+                if (ci < nchunk) {
+                    keep[it] = rotate_chunk<T>(xs, Rp, g, ci * 4);
+                    mx = amax4(mx, keep[it]);
+                }
+            }
+        } else {
+            for (int64_t ci = tid; ci < nchunk; ci += kGenThreads)
+                mx = amax4(mx, rotate_chunk<T>(xs, Rp, g, ci * 4));
+        }
+        for (int o = 16; o > 0; o >>= 1) mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if ((tid & 31) == 0) warp_max[tid >> 5] = mx;
+        __syncthreads();
+        float amax = 0.f;
+        for (int w = 0; w < kGenThreads / 32; ++w) amax = fmax_nan(amax, warp_max[w]);
+        const float s = row_scale(amax, scale_in);
+        if (tid == 0) scales[m] = s;
+
+        int8_t* qr = codes + m * ldq;
+        if (kKeep) {
+#pragma unroll
+            for (int it = 0; it < kGenMaxChunks; ++it) {
+                const int64_t ci = tid + (int64_t)it * kGenThreads;
+                if (ci < nchunk) store_codes4(qr + ci * 4, keep[it], s, vec_codes != 0);
+            }
+        } else {
+            for (int64_t ci = tid; ci < nchunk; ci += kGenThreads)
+                store_codes4(qr + ci * 4, rotate_chunk<T>(xs, Rp, g, ci * 4), s, vec_codes != 0);
+        }
+    }
+}
+
+// ===================================================================== MMA kernel
+
+constexpr int kMmaThreads = 256;
+
+template <typename T> struct MmaOp;
+template <> struct MmaOp<__nv_bfloat16> {
+    __device__ static __forceinline__ void run(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, "
+            "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    __device__ static __forceinline__ uint32_t pack(float lo, float hi) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&v);
+    }
+    __device__ static __forceinline__ float2 unpack(uint32_t u) {
+        return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
+    }
+};
+template <> struct MmaOp<__half> {
+    __device__ static __forceinline__ void run(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
+            "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    __device__ static __forceinline__ uint32_t pack(float lo, float hi) {
+        __half2 v = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&v);
+    }
+    __device__ static __forceinline__ float2 unpack(uint32_t u) {
+        return __half22float2(*reinterpret_cast<__half2*>(&u));
+    }
+};
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t saddr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(saddr));
+}
+
+// Byte offset of 16-byte chunk `c` of group-row `rho` in the TMA-swizzled box buffer.
+// G = 64: 128-byte rows, 128-byte swizzle (chunk ^= rho % 8).
+// G = 16: 32-byte rows, 32-byte swizzle (chunk ^= (rho / 4) % 2).
+template <int G>
+__device__ __forceinline__ uint32_t swz_off(int rho, int c) {
+    if (G == 64) return (uint32_t)rho * 128u + (uint32_t)((c ^ (rho & 7)) << 4);
+    return (uint32_t)rho * 32u + (uint32_t)((c ^ ((rho >> 2) & 1)) << 4);
+}
+
+struct RqMmaParams {
+    int64_t M, K, ldq;
+    int Gn;          // groups per row (K / G)
+    int GB;          // groups per TMA box
+    int NB;          // boxes per row block
+    int RB;          // rows per block
+    uint32_t box_stride;  // bytes between box buffers in shared memory
+    uint32_t box_bytes;   // bytes one box copy delivers
+    int vec_codes;
+};
+
+template <typename T, int G>
+__global__ void __launch_bounds__(kMmaThreads, 2)
+    rq_mma_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ R,
+                  const float* __restrict__ scale_in, int8_t* __restrict__ codes,
+                  float* __restrict__ scales, RqMmaParams p, int* dev_status) {
+    constexpr int KT = G / 16;   // k-tiles of the m16n8k16 MMA
+    constexpr int NT = G / 8;    // n-tiles
+    extern __shared__ __align__(1024) unsigned char mma_smem[];
+    unsigned char* buf = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(mma_smem) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ unsigned int amax_bits[16];
+    __shared__ float row_s[16];
+    __shared__ int abort_flag;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    // R as the B operand (k = input channel i, n = output channel c), held in registers:
+    // b0 = {R[k0 + 2q][n], R[k0 + 2q + 1][n]}, b1 = the same 8 rows further, n = lane / 4.
+    uint32_t bfr[KT][NT][2];
+    {
+        const int q = lane & 3, n_in = lane >> 2;
+#pragma unroll
+        for (int kt = 0; kt < KT; ++kt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int k = kt * 16 + h * 8 + 2 * q, n = nt * 8 + n_in;
+                    const float lo = Elem<T>::to_f(R[k * G + n]);
+                    const float hi = Elem<T>::to_f(R[(k + 1) * G + n]);
+                    bfr[kt][nt][h] = MmaOp<T>::pack(lo, hi);
+                }
+    }
+
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&xmap);
+    }
+    __syncthreads();
+
+    const int rows_per_box = p.RB * p.GB;            // valid group-rows in one box
+    const int tiles_per_box = (rows_per_box + 15) / 16;
+    const int n_tiles = tiles_per_box * p.NB;
+    const int64_t n_blocks = (p.M + p.RB - 1) / p.RB;
+    const int chunks_per_row = (int)(p.K / 16);
+    uint32_t phase = 0;
+
+    for (int64_t blk = blockIdx.x; blk < n_blocks; blk += gridDim.x) {
+        const int64_t m0 = blk * p.RB;
+        if (tid == 0) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(&bar, p.box_bytes * (uint32_t)p.NB);
+            for (int b = 0; b < p.NB; ++b)
+                tma_load_3d(buf + (size_t)b * p.box_stride, &xmap, &bar, 0, b * p.GB, (int32_t)m0);
+        }
+        if (tid < 16) amax_bits[tid] = 0u;
+        mbar_wait(&bar, phase, &abort_flag, dev_status);
+        phase ^= 1u;
+        __syncthreads();
+        if (abort_flag) return;
+
+        // ---- rotation: 16 consecutive group-rows per MMA tile, y written back in place
+        for (int t = warp; t < n_tiles; t += kMmaThreads / 32) {
+            const int b = t / tiles_per_box;
+            const int rho0 = (t - b * tiles_per_box) * 16;
+            const uint32_t base = smem_u32(buf + (size_t)b * p.box_stride);
+            uint32_t afr[KT][4];
+            {
+                const int rho = rho0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int cadd = lane >> 4;   // 0: k 0-7, 1: k 8-15 of the k-tile
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt)
+                    ldmatrix_x4(afr[kt], base + swz_off<G>(rho, kt * 2 + cadd));
+            }
+            float acc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt)
+                    MmaOp<T>::run(acc[nt], afr[kt], bfr[kt][nt][0], bfr[kt][nt][1]);
+            }
+            // round to T, store in place, row absmax
+            const int rA = rho0 + (lane >> 2), rB = rA + 8;
+            float mA = 0.f, mB = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint32_t pA = MmaOp<T>::pack(acc[nt][0], acc[nt][1]);
+                const uint32_t pB = MmaOp<T>::pack(acc[nt][2], acc[nt][3]);
+                const float2 yA = MmaOp<T>::unpack(pA), yB = MmaOp<T>::unpack(pB);
+                mA = fmax_nan(mA, fmax_nan(fabsf(yA.x), fabsf(yA.y)));
+                mB = fmax_nan(mB, fmax_nan(fabsf(yB.x), fabsf(yB.y)));
+                const uint32_t within = (uint32_t)(lane & 3) * 4u;
+                if (rA < rows_per_box)
+                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(base + swz_off<G>(rA, nt) + within),
+                                 "r"(pA));
+                if (rB < rows_per_box)
+                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(base + swz_off<G>(rB, nt) + within),
+                                 "r"(pB));
+            }
+            mA = fmax_nan(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
+            mA = fmax_nan(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
+            mB = fmax_nan(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
+            mB = fmax_nan(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
+            if ((lane & 3) == 0) {
+                if (rA < rows_per_box) atomicMax(&amax_bits[rA / p.GB], __float_as_uint(mA));
+                if (rB < rows_per_box) atomicMax(&amax_bits[rB / p.GB], __float_as_uint(mB));
+            }
+        }
+        __syncthreads();
+        if (tid < p.RB) {
+            const float s = row_scale(__uint_as_float(amax_bits[tid]), scale_in);
+            row_s[tid] = s;
+            if (m0 + tid < p.M) scales[m0 + tid] = s;
+        }
+        __syncthreads();
+
+        // ---- quantize: 16 consecutive channels per thread step, 16-byte code stores
+        const int n_chunks = p.RB * chunks_per_row;
+        for (int ci = tid; ci < n_chunks; ci += kMmaThreads) {
+            const int r = ci / chunks_per_row;
+            if (m0 + r >= p.M) break;
+            const int k = (ci - r * chunks_per_row) * 16;
+            const int j = k / G, e = k - j * G;
+            const int b = j / p.GB, jj = j - b * p.GB;
+            const int rho = r * p.GB + jj;
+            const unsigned char* bb = buf + (size_t)b * p.box_stride;
+            const uint4 u0 = *reinterpret_cast<const uint4*>(bb + swz_off<G>(rho, e / 8));
+            const uint4 u1 = *reinterpret_cast<const uint4*>(bb + swz_off<G>(rho, e / 8 + 1));
+            const float s = row_s[r];
+            const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            uint32_t out[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 a = MmaOp<T>::unpack(w[2 * i]), c = MmaOp<T>::unpack(w[2 * i + 1]);
+                out[i] = (uint32_t)(quant_code(a.x, s) & 0xFF) |
+                         ((uint32_t)(quant_code(a.y, s) & 0xFF) << 8) |
+                         ((uint32_t)(quant_code(c.x, s) & 0xFF) << 16) |
+                         ((uint32_t)(quant_code(c.y, s) & 0xFF) << 24);
+            }
+            int8_t* dst = codes + (m0 + r) * p.ldq + k;
+            if (p.vec_codes) {
+                *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) dst[i] = (int8_t)((out[i / 4] >> (8 * (i % 4))) & 0xFF);
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ===================================================================== host launch
+
+template <typename T, int G>
+static ck_status launch_mma(const void* x, int64_t M, int64_t K, int64_t sm, const void* R,
+                            const float* scale_in, int8_t* codes, int64_t ldq, float* scales,
+                            int* dev_status, cudaStream_t stream, CUtensorMapDataType tdt) {
+    RqMmaParams p;
+    p.M = M;
+    p.K = K;
+    p.ldq = ldq;
+    p.Gn = (int)(K / G);
+    p.NB = (p.Gn + 255) / 256;
+    p.GB = (p.Gn + p.NB - 1) / p.NB;
+    const int row_bytes = p.GB * G * 2;                 // per row, per box
+    // rows per block: fill about 96 KB with at least 2 blocks per SM in flight
+    int RB = 16;
+    while (RB > 1 && (int64_t)RB * row_bytes * p.NB > 96 * 1024) RB >>= 1;
+    const int64_t want_blocks = 2LL * num_sms();
+    while (RB > 1 && (M + RB - 1) / RB < want_blocks) RB >>= 1;
+    p.RB = RB;
+    p.box_bytes = (uint32_t)(RB * row_bytes);
+    // room for a ragged last 16-row MMA tile, rounded to the 1024-byte swizzle atom
+    const uint32_t tile_rows = (uint32_t)(((RB * p.GB) + 15) / 16 * 16);
+    p.box_stride = (tile_rows * G * 2 + 1023u) & ~1023u;
+    p.vec_codes = (aligned(codes, 16) && ldq % 16 == 0) ? 1 : 0;
+
+    CUtensorMap map;
+    const uint64_t dims[3] = {(uint64_t)G, (uint64_t)p.Gn, (uint64_t)M};
+    const uint64_t strides[2] = {(uint64_t)G * 2, (uint64_t)sm * 2};
+    const uint32_t box[3] = {(uint32_t)G, (uint32_t)p.GB, (uint32_t)RB};
+    ck_status st = encode_tma(&map, tdt, 3, x, dims, strides, box,
+                              G == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B);
+    if (st != CK_OK) return st;
+
+    const size_t smem = (size_t)p.box_stride * p.NB + 1024;
+    auto kern = rq_mma_kernel<T, G>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return CK_ERR_CUDA;
+    const int64_t n_blocks = (M + RB - 1) / RB;
+    int grid = (int)(n_blocks < 2LL * num_sms() ? n_blocks : 2LL * num_sms());
+    kern<<<grid, kMmaThreads, smem, stream>>>(map, static_cast<const T*>(R), scale_in, codes,
+                                              scales, p, dev_status);
+    return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+}
+
+template <typename T>
+static ck_status launch_generic(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
+                                const void* R, int g, const float* scale_in, int8_t* codes,
+                                int64_t ldq, float* scales, cudaStream_t stream) {
+    const size_t r_bytes = (size_t)g * g * sizeof(T);
+    const size_t xs_bytes = (size_t)K * sizeof(float);
+    const int r_in_smem = (xs_bytes + r_bytes <= 200 * 1024) ? 1 : 0;
+    const size_t smem = xs_bytes + (r_in_smem ? r_bytes : 0);
+    if (smem > 220 * 1024) return CK_ERR_UNSUPPORTED;
+    const int vec = (aligned(codes, 4) && ldq % 4 == 0) ? 1 : 0;
+    const int grid = (int)(M < 4LL * num_sms() ? M : 4LL * num_sms());
+    const bool keep = K <= (int64_t)kGenThreads * 4 * kGenMaxChunks;
+    if (keep) {
+        auto kern = rq_generic_kernel<T, true>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return CK_ERR_CUDA;
+        kern<<<grid, kGenThreads, smem, stream>>>(static_cast<const T*>(x), M, K, sm, sk,
+                                                  static_cast<const T*>(R), g, r_in_smem,
+                                                  scale_in, codes, ldq, scales, vec);
+    } else {
+        auto kern = rq_generic_kernel<T, false>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return CK_ERR_CUDA;
+        kern<<<grid, kGenThreads, smem, stream>>>(static_cast<const T*>(x), M, K, sm, sk,
+                                                  static_cast<const T*>(R), g, r_in_smem,
+                                                  scale_in, codes, ldq, scales, vec);
+    }
+    return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+}
+
+ck_status launch_rotate_quant(const void* x, ck_dtype dt, int64_t M, int64_t K, int64_t sm,
+                              int64_t sk, const void* R, int g, const float* scale_in,
+                              int8_t* codes, int64_t ldq, float* scales, int* dev_status,
+                              cudaStream_t stream) {
+    if (M == 0) return CK_OK;
+    const bool mma_ok = (dt == CK_BF16 || dt == CK_F16) && (g == 16 || g == 64) && sk == 1 &&
+                        aligned(x, 16) && sm % 8 == 0 && sm > 0 && M < (1LL << 31) &&
+                        K / g <= (1LL << 31);
+    if (mma_ok) {
+        if (dt == CK_BF16)
+            return g == 64 ? launch_mma<__nv_bfloat16, 64>(x, M, K, sm, R, scale_in, codes, ldq,
+                                                           scales, dev_status, stream,
+                                                           CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
+                           : launch_mma<__nv_bfloat16, 16>(x, M, K, sm, R, scale_in, codes, ldq,
+                                                           scales, dev_status, stream,
+                                                           CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+        return g == 64 ? launch_mma<__half, 64>(x, M, K, sm, R, scale_in, codes, ldq, scales,
+                                                dev_status, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)
+                       : launch_mma<__half, 16>(x, M, K, sm, R, scale_in, codes, ldq, scales,
+                                                dev_status, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    }
+    switch (dt) {
+        case CK_F32:
+            return launch_generic<float>(x, M, K, sm, sk, R, g, scale_in, codes, ldq, scales, stream);
+        case CK_F16:
+            return launch_generic<__half>(x, M, K, sm, sk, R, g, scale_in, codes, ldq, scales, stream);
+        case CK_BF16:
+            return launch_generic<__nv_bfloat16>(x, M, K, sm, sk, R, g, scale_in, codes, ldq, scales,
+                                                 stream);
+        default:
+            return CK_ERR_INVALID_ARG;
+    }
+}
+
+}  // namespace ck

@@ -122,7 +122,7 @@ def haar_orthogonal(g: int, gen: torch.Generator) -> torch.Tensor:
     """Random orthogonal g x g matrix (float64): QR of a Gaussian, with the diagonal of R made positive."""
     a = torch.randn(g, g, generator=gen, dtype=torch.float64)
     q, r = torch.linalg.qr(a)
-    return q * torch.sign(torch.diagonal(r)).unsqueeze(0)
+    return (q * torch.sign(torch.diagonal(r)).unsqueeze(0)).contiguous()
 
 
 def _activations(M: int, K: int, dist: str, outlier_frac: float, outlier_scale: float,

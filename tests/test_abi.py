@@ -1,0 +1,142 @@
+"""The C-ABI library loads without a GPU, exports every entry point include/ck.h declares,
+and rejects invalid calls on the host before any CUDA work (no device needed)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from rotated_w4a4_quantized_group_b200 import build as ck_build
+from rotated_w4a4_quantized_group_b200 import ck
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ck.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    ck_build.build()
+    return ck.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ck_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("ck_rotate_quant", "ck_w4a4_linear", "ck_unpack_w4"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(ck.SIGNATURES), "binding signatures must cover the header exactly"
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert ck.status_string(s)
+    assert "overflow" in ck.status_string(ck.CK_ERR_OVERFLOW).lower()
+
+
+def test_workspace_sizes(L):
+    M, N, K = 8192, 3840, 3840
+    P = ck.workspace_codes_pitch(K)
+    assert P == 3840 and ck.workspace_codes_pitch(48) == 48 and ck.workspace_codes_pitch(40) == 48
+    off = ck.workspace_scales_offset(M, K)
+    assert off >= M * P and off % 256 == 0
+    assert ck.workspace_bytes(M, N, K, K // 2) >= off + 4 * M
+    # an unaligned weight pitch adds room for a 16-byte-pitched weight copy
+    assert ck.workspace_bytes(7, 5, 48, 24) >= ck.workspace_bytes(7, 5, 48, 32) + 5 * 32
+    assert ck.workspace_bytes(7, 5, 47, 24) == 0          # odd K is invalid
+
+
+NULL = None
+
+
+def rq(L, **kw):
+    a = dict(x=1 << 20, dt=ck.CK_BF16, M=4, K=64, sm=64, sk=1, R=1 << 20, g=16, scale_in=NULL,
+             codes=1 << 20, ldq=64, scales=1 << 20, dev_status=NULL, stream=NULL)
+    a.update(kw)
+    return L.ck_rotate_quant(a["x"], a["dt"], a["M"], a["K"], a["sm"], a["sk"], a["R"], a["g"],
+                             a["scale_in"], a["codes"], a["ldq"], a["scales"], a["dev_status"],
+                             a["stream"])
+
+
+@pytest.mark.parametrize("bad", [dict(g=32), dict(g=0), dict(K=48, g=64), dict(K=0), dict(M=-1),
+                                 dict(ldq=63), dict(dt=ck.CK_I8), dict(dt=9), dict(x=NULL),
+                                 dict(R=NULL), dict(codes=NULL), dict(scales=NULL),
+                                 dict(R=(1 << 20) + 2)])
+def test_rotate_quant_rejects_on_host(L, bad):
+    assert rq(L, **bad) == ck.CK_ERR_INVALID_ARG
+
+
+def test_rotate_quant_empty_rows_is_a_noop(L):
+    assert rq(L, M=0, x=NULL, codes=NULL, scales=NULL) == ck.CK_OK
+
+
+def lin(L, **kw):
+    a = dict(x=1 << 20, dt=ck.CK_BF16, M=4, K=64, sm=64, sk=1, R=1 << 20, g=16, a_scale=NULL,
+             w=1 << 20, N=8, w_ld=32, w_scale=1 << 20, sdt=ck.CK_BF16, bias=NULL, out=1 << 20,
+             odt=ck.CK_BF16, ldo=8, ws=1 << 20, ws_bytes=1 << 20, dev_status=NULL, stream=NULL)
+    a.update(kw)
+    return L.ck_w4a4_linear(a["x"], a["dt"], a["M"], a["K"], a["sm"], a["sk"], a["R"], a["g"],
+                            a["a_scale"], a["w"], a["N"], a["w_ld"], a["w_scale"], a["sdt"],
+                            a["bias"], a["out"], a["odt"], a["ldo"], a["ws"], a["ws_bytes"],
+                            a["dev_status"], a["stream"])
+
+
+@pytest.mark.parametrize("bad", [dict(K=63), dict(K=48, g=64), dict(g=8), dict(w_ld=31),
+                                 dict(ldo=7), dict(sdt=ck.CK_I8), dict(odt=ck.CK_I8), dict(dt=7),
+                                 dict(M=-2), dict(N=-1), dict(x=NULL), dict(w=NULL),
+                                 dict(w_scale=NULL), dict(out=NULL), dict(R=NULL),
+                                 dict(dt=ck.CK_I8, sk=2), dict(dt=ck.CK_I8, sm=32),
+                                 dict(dt=ck.CK_I8, a_scale=NULL)])
+def test_linear_rejects_on_host(L, bad):
+    assert lin(L, **bad) == ck.CK_ERR_INVALID_ARG
+
+
+def test_linear_overflow_guard(L):
+    K = (2 ** 31 - 1) // 64 + 1
+    K += K % 2
+    assert lin(L, dt=ck.CK_I8, K=K, sm=K, w_ld=K // 2, a_scale=1 << 20) == ck.CK_ERR_OVERFLOW
+    # the largest even K under the bound passes the guard (and then fails on the fake
+    # null workspace, still on the host)
+    Kfit = (2 ** 31 - 1) // 64 // 2 * 2
+    assert lin(L, K=Kfit, g=16, sm=Kfit, w_ld=Kfit // 2, ws=NULL, ws_bytes=0) in (
+        ck.CK_ERR_INVALID_ARG, ck.CK_ERR_WORKSPACE)
+
+
+def test_linear_missing_workspace(L):
+    assert lin(L, ws=NULL, ws_bytes=0) == ck.CK_ERR_WORKSPACE
+    assert lin(L, ws_bytes=10) == ck.CK_ERR_WORKSPACE
+    assert lin(L, ws=(1 << 20) + 16) == ck.CK_ERR_WORKSPACE     # not 256-byte aligned
+
+
+def test_linear_empty_is_a_noop(L):
+    assert lin(L, M=0, x=NULL, out=NULL, ws=NULL, ws_bytes=0) == ck.CK_OK
+    assert lin(L, N=0, ldo=0, x=NULL, out=NULL, ws=NULL, ws_bytes=0) == ck.CK_OK
+
+
+@pytest.mark.parametrize("bad", [dict(K=7), dict(K=0), dict(N=-1), dict(ldp=3), dict(ldo=15),
+                                 dict(p=NULL), dict(o=NULL)])
+def test_unpack_rejects_on_host(L, bad):
+    a = dict(p=1 << 20, N=4, K=16, ldp=8, o=1 << 20, ldo=16)
+    a.update(bad)
+    assert L.ck_unpack_w4(a["p"], a["N"], a["K"], a["ldp"], a["o"], a["ldo"], None) == \
+        ck.CK_ERR_INVALID_ARG
+
+
+def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(ck, "_lib", None)
+    monkeypatch.setattr(ck, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        ck.lib()
