@@ -55,15 +55,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait that may suspend the thread (up to about 20 us) until the phase completes, so a
+// waiting warp does not take issue slots from the working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false (after
-// recording a timeout) if it does not complete within kWaitLimitCycles, or at once
-// if *abort is already set by another role of the CTA.
+// recording a timeout) if it does not complete within kWaitLimitCycles, or as soon as
+// *abort is seen set by another role of the CTA.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* dev_status) {
     if (mbar_try_wait(bar, parity)) return true;
-    long long t0 = clock64();
+    const long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity)) return true;
         if (abort && *abort) return false;
         if (clock64() - t0 > kWaitLimitCycles) {
             if (abort) *abort = 1;
@@ -71,6 +85,60 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
             return false;
         }
     }
+}
+
+// ------------------------------------------------------------------ CTA pairs (clusters of 2)
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Shared::cluster address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void* local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+    return r;
+}
+
+// Arrive (release at cluster scope) on an mbarrier given by its shared::cluster address.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+                 : "memory");
+}
+
+// Wait (acquire at cluster scope) for a phase of a local mbarrier that receives arrivals
+// from the peer CTA.  Bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort, int* dev_status) {
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (abort && *abort) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            if (abort) *abort = 1;
+            record_timeout(dev_status);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+                 ::: "memory");
 }
 
 // ------------------------------------------------------------------ TMA
@@ -94,6 +162,17 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// Tile load into this CTA's shared memory whose completion is counted on an mbarrier that
+// may live in the peer CTA of the pair (given by its shared::cluster address).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map,
+                                                 uint32_t cluster_bar, int32_t c0, int32_t c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(cluster_bar), "r"(c0), "r"(c1)
         : "memory");
 }
 
@@ -139,6 +218,45 @@ __device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t a_desc, uint
         : "memory");
 }
 
+// Pair versions (cta_group::2): one warp of each CTA of the pair allocates / frees the same
+// columns in both CTAs' tensor memory.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// D (+)= A * B^T across the CTA pair: M = 256 rows, A rows 0-127 from this CTA's shared
+// memory and 128-255 from the peer's at the same offsets, B rows split the same way,
+// D rows 0-127 in this CTA's tensor memory and 128-255 in the peer's.
+__device__ __forceinline__ void tc_mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on the mbarrier at this offset in both CTAs of the pair once every tcgen05
+// operation this thread issued so far completes.
+__device__ __forceinline__ void tc_commit_pair_both(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"((uint16_t)0x3)
+        : "memory");
+}
+
 // Arrive on an mbarrier once every tcgen05 operation this thread issued so far completes.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -158,6 +276,17 @@ __device__ __forceinline__ void tc_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[3
           "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
           "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
           "=r"(r[31])
+        : "r"(taddr));
+}
+
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
 }
 
@@ -227,6 +356,68 @@ __device__ __forceinline__ int quant_code(float y, float s) {
     t = rintf(t);
     t = fminf(fmaxf(t, -8.0f), 7.0f);
     return (int)t;
+}
+
+// The divisor of one row: s and r = fl(1 / s).  `fast` is false when r is not a normal
+// number (or s is NaN), in which case every code of the row takes the IEEE division.
+struct RowDivisor {
+    float s, r;
+    bool fast;
+    __device__ __forceinline__ explicit RowDivisor(float s_) : s(s_) {
+        r = __frcp_rn(s_);
+        fast = (r >= 1.17549435e-38f) && (r <= 3.40282347e38f);
+    }
+};
+
+// The same code as quant_code(y, d.s), with a multiply instead of the division.  The
+// product t = fl(y * fl(1/s)) is within 9 * 1.5 * 2^-23 < 2^-19 of the IEEE quotient
+// fl(y / s) wherever |t| < 9, so both round to the same integer unless t lies within 2^-19
+// of a half-integer; those rare values (and rows without a normal reciprocal) are divided
+// exactly.  Beyond |t| = 9 both clamp alike.  NaN converts to 0 and +-inf saturates, as in
+// quant_code.
+__device__ __forceinline__ int quant_code_fast(float y, const RowDivisor& d) {
+    if (!d.fast) return quant_code(y, d.s);
+    const float t = __fmul_rn(y, d.r);
+    float f = rintf(t);
+    if (fabsf(t - f) >= 0.5f - 0x1p-19f) f = rintf(__fdiv_rn(y, d.s));
+    return min(max(__float2int_rn(f), -8), 7);
+}
+
+// Sixteen codes of one row (divisor d) packed four per word, first code lowest.  The fast
+// path has no per-element branch: it flags the near-tie values and divides only those, in
+// a second pass that almost never runs.
+__device__ __forceinline__ uint32_t pack4_codes(int q0, int q1, int q2, int q3);
+__device__ __forceinline__ void quant16(const float (&y)[16], const RowDivisor& d,
+                                        uint32_t (&out)[4]) {
+    int q[16];
+    if (d.fast) {
+        uint32_t fix = 0u;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float t = __fmul_rn(y[i], d.r);
+            fix |= (fabsf(t - rintf(t)) >= 0.5f - 0x1p-19f) ? (1u << i) : 0u;
+            q[i] = __float2int_rn(t);          // ties to even; NaN -> 0; saturates
+        }
+        if (fix) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if ((fix >> i) & 1u) q[i] = __float2int_rn(__fdiv_rn(y[i], d.s));
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) q[i] = __float2int_rn(__fdiv_rn(y[i], d.s));
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = min(max(q[i], -8), 7);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) out[w] = pack4_codes(q[4 * w], q[4 * w + 1], q[4 * w + 2], q[4 * w + 3]);
+}
+
+// Four codes in [-8, 7] packed into the bytes of one word, first code lowest.
+__device__ __forceinline__ uint32_t pack4_codes(int q0, int q1, int q2, int q3) {
+    const uint32_t lo = __byte_perm((uint32_t)q0, (uint32_t)q1, 0x0040);
+    const uint32_t hi = __byte_perm((uint32_t)q2, (uint32_t)q3, 0x0040);
+    return __byte_perm(lo, hi, 0x5410);
 }
 
 }  // namespace ck

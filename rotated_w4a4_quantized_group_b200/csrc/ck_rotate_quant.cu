@@ -78,13 +78,11 @@ __device__ __forceinline__ float amax4(float m, float4 v) {
     return fmax_nan(m, fabsf(v.w));
 }
 
-__device__ __forceinline__ void store_codes4(int8_t* dst, float4 v, float s, bool vec) {
-    const int q0 = quant_code(v.x, s), q1 = quant_code(v.y, s), q2 = quant_code(v.z, s),
-              q3 = quant_code(v.w, s);
+__device__ __forceinline__ void store_codes4(int8_t* dst, float4 v, const RowDivisor& d, bool vec) {
+    const int q0 = quant_code_fast(v.x, d), q1 = quant_code_fast(v.y, d),
+              q2 = quant_code_fast(v.z, d), q3 = quant_code_fast(v.w, d);
     if (vec) {
-        uint32_t p = (uint32_t)(q0 & 0xFF) | ((uint32_t)(q1 & 0xFF) << 8) |
-                     ((uint32_t)(q2 & 0xFF) << 16) | ((uint32_t)(q3 & 0xFF) << 24);
-        *reinterpret_cast<uint32_t*>(dst) = p;
+        *reinterpret_cast<uint32_t*>(dst) = pack4_codes(q0, q1, q2, q3);
     } else {
         dst[0] = (int8_t)q0;
         dst[1] = (int8_t)q1;
@@ -143,17 +141,18 @@ __global__ void __launch_bounds__(kGenThreads)
         for (int w = 0; w < kGenThreads / 32; ++w) amax = fmax_nan(amax, warp_max[w]);
         const float s = row_scale(amax, scale_in);
         if (tid == 0) scales[m] = s;
+        const RowDivisor dv(s);
 
         int8_t* qr = codes + m * ldq;
         if (kKeep) {
 #pragma unroll
             for (int it = 0; it < kGenMaxChunks; ++it) {
                 const int64_t ci = tid + (int64_t)it * kGenThreads;
-                if (ci < nchunk) store_codes4(qr + ci * 4, keep[it], s, vec_codes != 0);
+                if (ci < nchunk) store_codes4(qr + ci * 4, keep[it], dv, vec_codes != 0);
             }
         } else {
             for (int64_t ci = tid; ci < nchunk; ci += kGenThreads)
-                store_codes4(qr + ci * 4, rotate_chunk<T>(xs, Rp, g, ci * 4), s, vec_codes != 0);
+                store_codes4(qr + ci * 4, rotate_chunk<T>(xs, Rp, g, ci * 4), dv, vec_codes != 0);
         }
     }
 }
@@ -179,6 +178,13 @@ template <> struct MmaOp<__nv_bfloat16> {
     __device__ static __forceinline__ float2 unpack(uint32_t u) {
         return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
     }
+    // running max of |.| over packed pairs, NaN-propagating
+    __device__ static __forceinline__ uint32_t absmax2(uint32_t m, uint32_t v) {
+        uint32_t a = v & 0x7FFF7FFFu;
+        __nv_bfloat162 r = __hmax2_nan(*reinterpret_cast<__nv_bfloat162*>(&m),
+                                       *reinterpret_cast<__nv_bfloat162*>(&a));
+        return *reinterpret_cast<uint32_t*>(&r);
+    }
 };
 template <> struct MmaOp<__half> {
     __device__ static __forceinline__ void run(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
@@ -195,6 +201,11 @@ template <> struct MmaOp<__half> {
     }
     __device__ static __forceinline__ float2 unpack(uint32_t u) {
         return __half22float2(*reinterpret_cast<__half2*>(&u));
+    }
+    __device__ static __forceinline__ uint32_t absmax2(uint32_t m, uint32_t v) {
+        uint32_t a = v & 0x7FFF7FFFu;
+        __half2 r = __hmax2_nan(*reinterpret_cast<__half2*>(&m), *reinterpret_cast<__half2*>(&a));
+        return *reinterpret_cast<uint32_t*>(&r);
     }
 };
 
@@ -221,9 +232,12 @@ struct RqMmaParams {
     int RB;          // rows per block
     uint32_t box_stride;  // bytes between box buffers in shared memory
     uint32_t box_bytes;   // bytes one box copy delivers
+    uint32_t buf_bytes;   // bytes of one row-block buffer (NB boxes)
     int vec_codes;
 };
 
+// Two row-block buffers per CTA: while one block is rotated and quantized, the TMA copy of
+// the next one is in flight.
 template <typename T, int G>
 __global__ void __launch_bounds__(kMmaThreads, 2)
     rq_mma_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ R,
@@ -232,9 +246,9 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
     constexpr int KT = G / 16;   // k-tiles of the m16n8k16 MMA
     constexpr int NT = G / 8;    // n-tiles
     extern __shared__ __align__(1024) unsigned char mma_smem[];
-    unsigned char* buf = reinterpret_cast<unsigned char*>(
+    unsigned char* bufs = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(mma_smem) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t bar;
+    __shared__ __align__(8) uint64_t bar[2];
     __shared__ unsigned int amax_bits[16];
     __shared__ float row_s[16];
     __shared__ int abort_flag;
@@ -259,40 +273,49 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
                 }
     }
 
+    const int64_t n_blocks = (p.M + p.RB - 1) / p.RB;
+    auto issue = [&](int b, int64_t blk) {
+        unsigned char* buf = bufs + (size_t)b * p.buf_bytes;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&bar[b], p.box_bytes * (uint32_t)p.NB);
+        for (int bx = 0; bx < p.NB; ++bx)
+            tma_load_3d(buf + (size_t)bx * p.box_stride, &xmap, &bar[b], 0, bx * p.GB,
+                        (int32_t)(blk * p.RB));
+    };
     if (tid == 0) {
-        mbar_init(&bar, 1);
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
         abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&xmap);
+        for (int b = 0; b < 2; ++b) {
+            const int64_t blk = blockIdx.x + (int64_t)b * gridDim.x;
+            if (blk < n_blocks) issue(b, blk);
+        }
     }
     __syncthreads();
 
     const int rows_per_box = p.RB * p.GB;            // valid group-rows in one box
     const int tiles_per_box = (rows_per_box + 15) / 16;
     const int n_tiles = tiles_per_box * p.NB;
-    const int64_t n_blocks = (p.M + p.RB - 1) / p.RB;
     const int chunks_per_row = (int)(p.K / 16);
-    uint32_t phase = 0;
 
-    for (int64_t blk = blockIdx.x; blk < n_blocks; blk += gridDim.x) {
+    for (int64_t i = 0;; ++i) {
+        const int64_t blk = blockIdx.x + i * gridDim.x;
+        if (blk >= n_blocks) break;
+        const int b = (int)(i & 1);
+        unsigned char* buf = bufs + (size_t)b * p.buf_bytes;
         const int64_t m0 = blk * p.RB;
-        if (tid == 0) {
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&bar, p.box_bytes * (uint32_t)p.NB);
-            for (int b = 0; b < p.NB; ++b)
-                tma_load_3d(buf + (size_t)b * p.box_stride, &xmap, &bar, 0, b * p.GB, (int32_t)m0);
-        }
         if (tid < 16) amax_bits[tid] = 0u;
-        mbar_wait(&bar, phase, &abort_flag, dev_status);
-        phase ^= 1u;
+        mbar_wait(&bar[b], (uint32_t)(i >> 1) & 1u, &abort_flag, dev_status);
         __syncthreads();
         if (abort_flag) return;
 
         // ---- rotation: 16 consecutive group-rows per MMA tile, y written back in place
         for (int t = warp; t < n_tiles; t += kMmaThreads / 32) {
-            const int b = t / tiles_per_box;
-            const int rho0 = (t - b * tiles_per_box) * 16;
-            const uint32_t base = smem_u32(buf + (size_t)b * p.box_stride);
+            const int bx = t / tiles_per_box;
+            const int rho0 = (t - bx * tiles_per_box) * 16;
+            const uint32_t base = smem_u32(buf + (size_t)bx * p.box_stride);
             uint32_t afr[KT][4];
             {
                 const int rho = rho0 + (lane & 7) + ((lane >> 3) & 1) * 8;
@@ -311,14 +334,13 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
             }
             // round to T, store in place, row absmax
             const int rA = rho0 + (lane >> 2), rB = rA + 8;
-            float mA = 0.f, mB = 0.f;
+            uint32_t mA2 = 0u, mB2 = 0u;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const uint32_t pA = MmaOp<T>::pack(acc[nt][0], acc[nt][1]);
                 const uint32_t pB = MmaOp<T>::pack(acc[nt][2], acc[nt][3]);
-                const float2 yA = MmaOp<T>::unpack(pA), yB = MmaOp<T>::unpack(pB);
-                mA = fmax_nan(mA, fmax_nan(fabsf(yA.x), fabsf(yA.y)));
-                mB = fmax_nan(mB, fmax_nan(fabsf(yB.x), fabsf(yB.y)));
+                mA2 = MmaOp<T>::absmax2(mA2, pA);
+                mB2 = MmaOp<T>::absmax2(mB2, pB);
                 const uint32_t within = (uint32_t)(lane & 3) * 4u;
                 if (rA < rows_per_box)
                     asm volatile("st.shared.b32 [%0], %1;" ::"r"(base + swz_off<G>(rA, nt) + within),
@@ -327,6 +349,8 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
                     asm volatile("st.shared.b32 [%0], %1;" ::"r"(base + swz_off<G>(rB, nt) + within),
                                  "r"(pB));
             }
+            const float2 fA = MmaOp<T>::unpack(mA2), fB = MmaOp<T>::unpack(mB2);
+            float mA = fmax_nan(fA.x, fA.y), mB = fmax_nan(fB.x, fB.y);
             mA = fmax_nan(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
             mA = fmax_nan(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
             mB = fmax_nan(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
@@ -345,37 +369,48 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
         __syncthreads();
 
         // ---- quantize: 16 consecutive channels per thread step, 16-byte code stores
-        const int n_chunks = p.RB * chunks_per_row;
-        for (int ci = tid; ci < n_chunks; ci += kMmaThreads) {
-            const int r = ci / chunks_per_row;
+        for (int r = 0; r < p.RB; ++r) {
             if (m0 + r >= p.M) break;
-            const int k = (ci - r * chunks_per_row) * 16;
-            const int j = k / G, e = k - j * G;
-            const int b = j / p.GB, jj = j - b * p.GB;
-            const int rho = r * p.GB + jj;
-            const unsigned char* bb = buf + (size_t)b * p.box_stride;
-            const uint4 u0 = *reinterpret_cast<const uint4*>(bb + swz_off<G>(rho, e / 8));
-            const uint4 u1 = *reinterpret_cast<const uint4*>(bb + swz_off<G>(rho, e / 8 + 1));
-            const float s = row_s[r];
-            const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-            uint32_t out[4];
+            const RowDivisor dv(row_s[r]);
+            int8_t* dst_row = codes + (m0 + r) * p.ldq;
+            for (int c = tid; c < chunks_per_row; c += kMmaThreads) {
+                const int k = c * 16;
+                const int j = k / G, e = k - j * G;
+                int bx = 0, jj = j;
+                if (p.NB > 1) {
+                    bx = j / p.GB;
+                    jj = j - bx * p.GB;
+                }
+                const int rho = r * p.GB + jj;
+                const unsigned char* bb = buf + (size_t)bx * p.box_stride;
+                const uint4 u0 = *reinterpret_cast<const uint4*>(bb + swz_off<G>(rho, e / 8));
+                const uint4 u1 = *reinterpret_cast<const uint4*>(bb + swz_off<G>(rho, e / 8 + 1));
+                const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+                float y[16];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 a = MmaOp<T>::unpack(w[2 * i]), c = MmaOp<T>::unpack(w[2 * i + 1]);
-                out[i] = (uint32_t)(quant_code(a.x, s) & 0xFF) |
-                         ((uint32_t)(quant_code(a.y, s) & 0xFF) << 8) |
-                         ((uint32_t)(quant_code(c.x, s) & 0xFF) << 16) |
-                         ((uint32_t)(quant_code(c.y, s) & 0xFF) << 24);
-            }
-            int8_t* dst = codes + (m0 + r) * p.ldq + k;
-            if (p.vec_codes) {
-                *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
-            } else {
+                for (int h = 0; h < 8; ++h) {
+                    const float2 a = MmaOp<T>::unpack(w[h]);
+                    y[2 * h] = a.x;
+                    y[2 * h + 1] = a.y;
+                }
+                uint32_t out[4];
+                quant16(y, dv, out);
+                int8_t* dst = dst_row + k;
+                if (p.vec_codes) {
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+                } else {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) dst[i] = (int8_t)((out[i / 4] >> (8 * (i % 4))) & 0xFF);
+                    for (int q = 0; q < 16; ++q)
+                        dst[q] = (int8_t)((out[q / 4] >> (8 * (q % 4))) & 0xFF);
+                }
             }
         }
         __syncthreads();
+        // the buffer is free again: fetch the block two steps ahead into it
+        if (tid == 0) {
+            const int64_t nb = blk + 2LL * gridDim.x;
+            if (nb < n_blocks) issue(b, nb);
+        }
     }
 }
 
@@ -392,17 +427,20 @@ static ck_status launch_mma(const void* x, int64_t M, int64_t K, int64_t sm, con
     p.Gn = (int)(K / G);
     p.NB = (p.Gn + 255) / 256;
     p.GB = (p.Gn + p.NB - 1) / p.NB;
-    const int row_bytes = p.GB * G * 2;                 // per row, per box
-    // rows per block: fill about 96 KB with at least 2 blocks per SM in flight
+    // rows per block: two buffers per CTA within about 100 KB (two CTAs per SM), and
+    // enough blocks for every CTA
+    const int sms = num_sms();
+    auto stride_for = [&](int rb) {
+        const uint32_t tile_rows = (uint32_t)(((rb * p.GB) + 15) / 16 * 16);
+        return (tile_rows * G * 2 + 1023u) & ~1023u;
+    };
     int RB = 16;
-    while (RB > 1 && (int64_t)RB * row_bytes * p.NB > 96 * 1024) RB >>= 1;
-    const int64_t want_blocks = 2LL * num_sms();
-    while (RB > 1 && (M + RB - 1) / RB < want_blocks) RB >>= 1;
+    while (RB > 1 && 2ULL * stride_for(RB) * p.NB > 100 * 1024) RB >>= 1;
+    while (RB > 1 && (M + RB - 1) / RB < 2LL * sms) RB >>= 1;
     p.RB = RB;
-    p.box_bytes = (uint32_t)(RB * row_bytes);
-    // room for a ragged last 16-row MMA tile, rounded to the 1024-byte swizzle atom
-    const uint32_t tile_rows = (uint32_t)(((RB * p.GB) + 15) / 16 * 16);
-    p.box_stride = (tile_rows * G * 2 + 1023u) & ~1023u;
+    p.box_bytes = (uint32_t)(RB * p.GB * G * 2);
+    p.box_stride = stride_for(RB);
+    p.buf_bytes = p.box_stride * (uint32_t)p.NB;
     p.vec_codes = (aligned(codes, 16) && ldq % 16 == 0) ? 1 : 0;
 
     CUtensorMap map;
@@ -413,13 +451,13 @@ static ck_status launch_mma(const void* x, int64_t M, int64_t K, int64_t sm, con
                               G == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B);
     if (st != CK_OK) return st;
 
-    const size_t smem = (size_t)p.box_stride * p.NB + 1024;
+    const size_t smem = 2 * (size_t)p.buf_bytes + 1024;
     auto kern = rq_mma_kernel<T, G>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return CK_ERR_CUDA;
     const int64_t n_blocks = (M + RB - 1) / RB;
-    int grid = (int)(n_blocks < 2LL * num_sms() ? n_blocks : 2LL * num_sms());
+    int grid = (int)(n_blocks < 2LL * sms ? n_blocks : 2LL * sms);
     kern<<<grid, kMmaThreads, smem, stream>>>(map, static_cast<const T*>(R), scale_in, codes,
                                               scales, p, dev_status);
     return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;

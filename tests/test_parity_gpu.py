@@ -334,3 +334,41 @@ def test_binding_rejects_a_transposed_rotation():
         ck.ck_rotate_quant(x, R.t(), 64)
     with pytest.raises(ValueError):
         ck.ck_rotate_quant(x, R.float(), 64)
+
+
+def test_gemm_at_the_overflow_guard():
+    """K just under the 64*K <= INT32_MAX guard with extreme codes: the true accumulator
+    (-56 K and 49 K) fits in int32 even where intermediate sums are larger."""
+    K = (2 ** 31 - 1) // 64 // 128 * 128
+    M, N = 2, 16
+    q = torch.full((M, K), -8, dtype=torch.int8)
+    q[1] = 7
+    wp = torch.full((N, K // 2), 0x77, dtype=torch.int8)     # every code 7
+    out = ck.ck_w4a4_linear(q.cuda(), None, 0, wp.cuda(), torch.ones(N, device="cuda"),
+                            a_scale=torch.ones(M, device="cuda"), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    acc = np.array([-56 * K, 49 * K], dtype=np.int64)
+    assert np.abs(acc).max() <= 2 ** 31 - 1
+    ref = acc.astype(np.float32)[:, None].repeat(N, 1)
+    np.testing.assert_array_equal(out.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("g", [16, 64])
+def test_quantizer_exact_ties_with_inexact_reciprocal(dt, g):
+    """Row absmax 21 gives s = 3 exactly, whose reciprocal is inexact: y / s is an exact
+    half-integer for y = 3 (k + 1/2), and only the IEEE quotient rounds those half-to-even.
+    Expected codes worked by hand: 1.5/3 = 0.5 -> 0, 4.5/3 = 1.5 -> 2, 7.5/3 = 2.5 -> 2,
+    10.5/3 = 3.5 -> 4, 13.5/3 = 4.5 -> 4, 16.5/3 = 5.5 -> 6, 19.5/3 = 6.5 -> 6."""
+    vals = [21, 1.5, 4.5, 7.5, 10.5, 13.5, 16.5, 19.5, -1.5, -4.5, -7.5, -10.5, -13.5, -16.5,
+            -19.5, -21]
+    want = [7, 0, 2, 2, 4, 4, 6, 6, 0, -2, -2, -4, -4, -6, -6, -7]
+    x = torch.tensor(vals * (g // 16) * 2, dtype=torch.float64).reshape(1, -1).repeat(40, 1)
+    x = x.to(DT[dt])
+    R = torch.eye(g, dtype=torch.float64).to(DT[dt])
+    codes, scales = ck.ck_rotate_quant(x.cuda(), R.cuda(), g)
+    torch.cuda.synchronize()
+    assert (scales.cpu() == 3.0).all()
+    np.testing.assert_array_equal(codes.cpu().numpy(), np.array(want * (g // 16) * 2)[None].repeat(40, 0))
+    oc, os_ = oracle.rotate_quant(x, R, g)
+    np.testing.assert_array_equal(codes.cpu().numpy(), oc)
