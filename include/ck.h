@@ -141,6 +141,33 @@ size_t ck_workspace_scales_offset(int64_t M, int64_t K);
 ck_status ck_unpack_w4(const int8_t* packed, int64_t N, int64_t K, int64_t ld_packed,
                        int8_t* out, int64_t ld_out, cudaStream_t stream);
 
+/*
+ * The whole linear without a caller-provided workspace, for callers that cannot allocate
+ * device memory (a plugin inside a host framework that owns all device memory and offers no
+ * allocation hook, or a latency-critical loop that must not call cudaMalloc, which may
+ * synchronise the device).  This entry point has no counterpart on the pages: it is a
+ * deployment convenience around ck_w4a4_linear, with the same arguments, results and errors
+ * except workspace / workspace_bytes.
+ *
+ * Scratch memory comes from an array compiled into the library: 32 MiB of device memory
+ * that every GPU which loads the library holds until the process exits.  The call allocates
+ * nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *   - Limit: calls whose scratch need (ck_w4a4_linear_workspace_bytes for the same sizes,
+ *     or 0 for 16-byte-aligned int8 codes with 16-byte-pitched weights) exceeds 32 MiB
+ *     return CK_ERR_WORKSPACE and launch nothing (e.g. 8192 x 3840 activations fit,
+ *     8192 x 10240 do not).
+ *   - The first call on each device looks up the array's device address (with that device
+ *     current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array and nothing in it needs clearing between
+ *     calls; calls whose GPU work overlaps in time (different streams) race on it.
+ */
+ck_status ck_w4a4_linear_noalloc(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                                 int64_t stride_m, int64_t stride_k, const void* R, int g,
+                                 const float* a_scale, const int8_t* w_packed, int64_t N,
+                                 int64_t w_ld, const void* w_scale, ck_dtype scale_dtype,
+                                 const void* bias, void* out, ck_dtype out_dtype, int64_t ldo,
+                                 int* dev_status, cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 const char* ck_status_string(ck_status status);
 

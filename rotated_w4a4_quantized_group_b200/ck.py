@@ -32,6 +32,8 @@ SIGNATURES = {
     "ck_w4a4_linear_workspace_bytes": ([_I64, _I64, _I64, _I64], _SZ),
     "ck_workspace_codes_pitch": ([_I64], _I64),
     "ck_workspace_scales_offset": ([_I64, _I64], _SZ),
+    "ck_w4a4_linear_noalloc": ([_P, _I, _I64, _I64, _I64, _I64, _P, _I, _P, _P, _I64, _I64, _P,
+                                _I, _P, _P, _I, _I64, _P, _P], _I),
     "ck_unpack_w4": ([_P, _I64, _I64, _I64, _P, _I64, _P], _I),
     "ck_status_string": ([_I], ctypes.c_char_p),
 }
@@ -148,6 +150,26 @@ def ck_w4a4_linear(x: torch.Tensor, R: torch.Tensor | None, g: int, w_packed: to
         DTYPE_CODE[w_scale.dtype], _ptr(bias), _ptr(out), DTYPE_CODE[out.dtype], out.stride(0),
         _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream))
     _check(st, "ck_w4a4_linear")
+    return out
+
+
+def ck_w4a4_linear_noalloc(x: torch.Tensor, R: torch.Tensor | None, g: int,
+                           w_packed: torch.Tensor, w_scale: torch.Tensor,
+                           bias: torch.Tensor | None = None, *, out: torch.Tensor,
+                           a_scale: torch.Tensor | None = None,
+                           dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """ck_w4a4_linear with the library's built-in 32 MiB scratch instead of a workspace, for
+    callers that cannot allocate device memory; `out` must be given (nothing is allocated)."""
+    M, K = x.shape
+    N = w_packed.shape[0]
+    if x.dtype != torch.int8:
+        _check_rotation(x, R, g)
+    st = lib().ck_w4a4_linear_noalloc(
+        _ptr(x), DTYPE_CODE[x.dtype], M, K, x.stride(0), x.stride(1), _ptr(R), int(g),
+        _ptr(a_scale), _ptr(w_packed), N, w_packed.stride(0), _ptr(w_scale),
+        DTYPE_CODE[w_scale.dtype], _ptr(bias), _ptr(out), DTYPE_CODE[out.dtype], out.stride(0),
+        _ptr(dev_status), _stream(stream))
+    _check(st, "ck_w4a4_linear_noalloc")
     return out
 
 
