@@ -58,16 +58,22 @@ def source_sha(path: str) -> str:
 
 
 def recorded_traffic(kernel_file: str, workload: str):
-    """DRAM bytes per launch recorded from an ncu capture of this exact kernel source."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch recorded (profiles/traffic.md) from an ncu capture of this exact
+    kernel source; None when no row matches the current source."""
+    p = os.path.join(ROOT, "profiles", "traffic.md")
     if not os.path.exists(p):
         return None
+    sha = source_sha(kernel_file)
+    name = os.path.basename(kernel_file)
     with open(p) as f:
-        d = json.load(f)
-    e = d.get(os.path.basename(kernel_file), {}).get(workload)
-    if not e or e.get("source_sha") != source_sha(kernel_file):
-        return None
-    return e.get("dram_bytes_per_launch")
+        for line in f:
+            cells = [c.strip() for c in line.strip().strip("|").split("|")]
+            if len(cells) >= 4 and cells[0] == name and cells[1] == workload and cells[2] == sha:
+                try:
+                    return int(cells[3])
+                except ValueError:
+                    return None
+    return None
 
 
 class ClockSampler:

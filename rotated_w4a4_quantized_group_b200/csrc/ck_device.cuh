@@ -383,27 +383,39 @@ __device__ __forceinline__ int quant_code_fast(float y, const RowDivisor& d) {
     return min(max(__float2int_rn(f), -8), 7);
 }
 
+// Two fp32 products at once (sm_100 packed fp32 multiply), each rounded to nearest even.
+__device__ __forceinline__ float2 mul2_rn(float a0, float a1, float b) {
+    unsigned long long x, y, z;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a0), "f"(a1));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(y) : "f"(b));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(z));
+    return r;
+}
+
 // Sixteen codes of one row (divisor d) packed four per word, first code lowest.  The fast
-// path has no per-element branch: it flags the near-tie values and divides only those, in
-// a second pass that almost never runs.
+// path has no per-element branch: it notes whether any product lies within 2^-19 of a
+// half-integer, and only then (rarely) recomputes the sixteen codes with the IEEE divide.
 __device__ __forceinline__ uint32_t pack4_codes(int q0, int q1, int q2, int q3);
 __device__ __forceinline__ void quant16(const float (&y)[16], const RowDivisor& d,
                                         uint32_t (&out)[4]) {
     int q[16];
+    bool exact = !d.fast;
     if (d.fast) {
-        uint32_t fix = 0u;
+        bool near_tie = false;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float t = __fmul_rn(y[i], d.r);
-            fix |= (fabsf(t - rintf(t)) >= 0.5f - 0x1p-19f) ? (1u << i) : 0u;
-            q[i] = __float2int_rn(t);          // ties to even; NaN -> 0; saturates
+        for (int i = 0; i < 16; i += 2) {
+            const float2 t = mul2_rn(y[i], y[i + 1], d.r);
+            const float f0 = rintf(t.x), f1 = rintf(t.y);
+            near_tie |= fabsf(t.x - f0) >= 0.5f - 0x1p-19f;
+            near_tie |= fabsf(t.y - f1) >= 0.5f - 0x1p-19f;
+            q[i] = __float2int_rn(f0);          // NaN -> 0; +-inf saturates
+            q[i + 1] = __float2int_rn(f1);
         }
-        if (fix) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if ((fix >> i) & 1u) q[i] = __float2int_rn(__fdiv_rn(y[i], d.s));
-        }
-    } else {
+        exact = near_tie;
+    }
+    if (exact) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) q[i] = __float2int_rn(__fdiv_rn(y[i], d.s));
     }

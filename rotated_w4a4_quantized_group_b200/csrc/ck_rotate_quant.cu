@@ -159,7 +159,6 @@ __global__ void __launch_bounds__(kGenThreads)
 
 // ===================================================================== MMA kernel
 
-constexpr int kMmaThreads = 256;
 
 template <typename T> struct MmaOp;
 template <> struct MmaOp<__nv_bfloat16> {
@@ -209,6 +208,13 @@ template <> struct MmaOp<__half> {
     }
 };
 
+__device__ __forceinline__ void stmatrix_x4(uint32_t saddr, uint32_t r0, uint32_t r1, uint32_t r2,
+                                            uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(saddr),
+                 "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+}
+
 __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t saddr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -230,188 +236,236 @@ struct RqMmaParams {
     int GB;          // groups per TMA box
     int NB;          // boxes per row block
     int RB;          // rows per block
+    int S;           // ring stages (row blocks in flight)
     uint32_t box_stride;  // bytes between box buffers in shared memory
     uint32_t box_bytes;   // bytes one box copy delivers
-    uint32_t buf_bytes;   // bytes of one row-block buffer (NB boxes)
+    uint32_t stage_bytes; // bytes of one ring stage (NB boxes)
     int vec_codes;
 };
 
-// Two row-block buffers per CTA: while one block is rotated and quantized, the TMA copy of
-// the next one is in flight.
+constexpr int kRqMaxStages = 8;
+constexpr int kRqGroupWarps = 8;                            // warps of one compute group
+constexpr int kRqGroups = 2;                                // groups take alternate blocks
+constexpr int kRqComputeWarps = kRqGroupWarps * kRqGroups;
+constexpr int kRqThreads = (kRqComputeWarps + 1) * 32;      // + one TMA producer warp
+
+// R transposed (RT[n][k] = R[k][n]) in shared memory: rows of G bf16/fp16 values with the
+// 16-byte chunks of row n XOR-swizzled by n % 8 (rows of 32 bytes for G = 16 use n / 4 % 2),
+// so that ldmatrix of 8 consecutive rows is bank-conflict free.
+template <int G>
+__device__ __forceinline__ uint32_t rt_off(int n, int chunk) {
+    if (G == 16) return (uint32_t)n * 32u + (uint32_t)((chunk ^ ((n >> 2) & 1)) << 4);
+    return (uint32_t)n * (uint32_t)(G * 2) + (uint32_t)(((chunk & ~7) | ((chunk & 7) ^ (n & 7))) << 4);
+}
+
+// One persistent CTA per SM.  Warp 16 streams row blocks into a ring of shared-memory stages
+// with TMA (several blocks in flight per SM); two groups of eight compute warps take
+// alternate blocks: rotate in place (B fragments of R from shared memory), reduce the row
+// absmax, compute the row scales, quantize, store the codes, and release the stage.  The
+// phases of one block are separated by mbarriers (bounded waits), so one group's scale
+// step overlaps the other group's work.
 template <typename T, int G>
-__global__ void __launch_bounds__(kMmaThreads, 2)
+__global__ void __launch_bounds__(kRqThreads, 1)
     rq_mma_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ R,
                   const float* __restrict__ scale_in, int8_t* __restrict__ codes,
                   float* __restrict__ scales, RqMmaParams p, int* dev_status) {
     constexpr int KT = G / 16;   // k-tiles of the m16n8k16 MMA
     constexpr int NT = G / 8;    // n-tiles
     extern __shared__ __align__(1024) unsigned char mma_smem[];
-    unsigned char* bufs = reinterpret_cast<unsigned char*>(
+    unsigned char* ring = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(mma_smem) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t bar[2];
-    __shared__ unsigned int amax_bits[16];
-    __shared__ float row_s[16];
+    __shared__ __align__(8) uint64_t full_bar[kRqMaxStages], empty_bar[kRqMaxStages];
+    __shared__ __align__(8) uint64_t rot_done[kRqMaxStages], scale_ready[kRqMaxStages];
+    __shared__ unsigned int amax_bits[kRqMaxStages][16];
+    __shared__ float row_s[kRqMaxStages][16], row_r[kRqMaxStages][16];
     __shared__ int abort_flag;
+    __shared__ __align__(128) unsigned char rt_sh[G * G * 2];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-    // R as the B operand (k = input channel i, n = output channel c), held in registers:
-    // b0 = {R[k0 + 2q][n], R[k0 + 2q + 1][n]}, b1 = the same 8 rows further, n = lane / 4.
-    uint32_t bfr[KT][NT][2];
-    {
-        const int q = lane & 3, n_in = lane >> 2;
-#pragma unroll
-        for (int kt = 0; kt < KT; ++kt)
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int k = kt * 16 + h * 8 + 2 * q, n = nt * 8 + n_in;
-                    const float lo = Elem<T>::to_f(R[k * G + n]);
-                    const float hi = Elem<T>::to_f(R[(k + 1) * G + n]);
-                    bfr[kt][nt][h] = MmaOp<T>::pack(lo, hi);
-                }
-    }
-
     const int64_t n_blocks = (p.M + p.RB - 1) / p.RB;
-    auto issue = [&](int b, int64_t blk) {
-        unsigned char* buf = bufs + (size_t)b * p.buf_bytes;
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&bar[b], p.box_bytes * (uint32_t)p.NB);
-        for (int bx = 0; bx < p.NB; ++bx)
-            tma_load_3d(buf + (size_t)bx * p.box_stride, &xmap, &bar[b], 0, bx * p.GB,
-                        (int32_t)(blk * p.RB));
-    };
+    const int my_blocks =
+        blockIdx.x < n_blocks ? (int)((n_blocks - 1 - blockIdx.x) / gridDim.x) + 1 : 0;
+
     if (tid == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
+        for (int s = 0; s < p.S; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], kRqGroupWarps);
+            mbar_init(&rot_done[s], kRqGroupWarps);
+            mbar_init(&scale_ready[s], 1);
+        }
         abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&xmap);
-        for (int b = 0; b < 2; ++b) {
-            const int64_t blk = blockIdx.x + (int64_t)b * gridDim.x;
-            if (blk < n_blocks) issue(b, blk);
-        }
+    }
+    if (tid < kRqMaxStages * 16) amax_bits[tid >> 4][tid & 15] = 0u;
+    // R transposed into shared memory (the B operand: n = output channel, k = input channel)
+    for (int i = tid; i < G * G; i += kRqThreads) {
+        const int n = i / G, k = i % G;
+        const T v = R[k * G + n];
+        *reinterpret_cast<T*>(rt_sh + rt_off<G>(n, k / 8) + (k % 8) * 2) = v;
     }
     __syncthreads();
 
-    const int rows_per_box = p.RB * p.GB;            // valid group-rows in one box
-    const int tiles_per_box = (rows_per_box + 15) / 16;
-    const int n_tiles = tiles_per_box * p.NB;
-    const int chunks_per_row = (int)(p.K / 16);
-
-    for (int64_t i = 0;; ++i) {
-        const int64_t blk = blockIdx.x + i * gridDim.x;
-        if (blk >= n_blocks) break;
-        const int b = (int)(i & 1);
-        unsigned char* buf = bufs + (size_t)b * p.buf_bytes;
-        const int64_t m0 = blk * p.RB;
-        if (tid < 16) amax_bits[tid] = 0u;
-        mbar_wait(&bar[b], (uint32_t)(i >> 1) & 1u, &abort_flag, dev_status);
-        __syncthreads();
-        if (abort_flag) return;
-
-        // ---- rotation: 16 consecutive group-rows per MMA tile, y written back in place
-        for (int t = warp; t < n_tiles; t += kMmaThreads / 32) {
-            const int bx = t / tiles_per_box;
-            const int rho0 = (t - bx * tiles_per_box) * 16;
-            const uint32_t base = smem_u32(buf + (size_t)bx * p.box_stride);
-            uint32_t afr[KT][4];
-            {
-                const int rho = rho0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-                const int cadd = lane >> 4;   // 0: k 0-7, 1: k 8-15 of the k-tile
-#pragma unroll
-                for (int kt = 0; kt < KT; ++kt)
-                    ldmatrix_x4(afr[kt], base + swz_off<G>(rho, kt * 2 + cadd));
+    if (warp == kRqComputeWarps) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int i = 0; i < my_blocks; ++i) {
+                const int s = i % p.S;
+                if (i >= p.S &&
+                    !mbar_wait(&empty_bar[s], (uint32_t)((i / p.S) - 1) & 1u, &abort_flag, dev_status))
+                    break;
+                const int64_t blk = blockIdx.x + (int64_t)i * gridDim.x;
+                unsigned char* stage = ring + (size_t)s * p.stage_bytes;
+                mbar_arrive_expect_tx(&full_bar[s], p.box_bytes * (uint32_t)p.NB);
+                for (int bx = 0; bx < p.NB; ++bx)
+                    tma_load_3d(stage + (size_t)bx * p.box_stride, &xmap, &full_bar[s], 0, bx * p.GB,
+                                (int32_t)(blk * p.RB));
+                ++issued;
             }
-            float acc[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-#pragma unroll
-                for (int kt = 0; kt < KT; ++kt)
-                    MmaOp<T>::run(acc[nt], afr[kt], bfr[kt][nt][0], bfr[kt][nt][1]);
-            }
-            // round to T, store in place, row absmax
-            const int rA = rho0 + (lane >> 2), rB = rA + 8;
-            uint32_t mA2 = 0u, mB2 = 0u;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const uint32_t pA = MmaOp<T>::pack(acc[nt][0], acc[nt][1]);
-                const uint32_t pB = MmaOp<T>::pack(acc[nt][2], acc[nt][3]);
-                mA2 = MmaOp<T>::absmax2(mA2, pA);
-                mB2 = MmaOp<T>::absmax2(mB2, pB);
-                const uint32_t within = (uint32_t)(lane & 3) * 4u;
-                if (rA < rows_per_box)
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(base + swz_off<G>(rA, nt) + within),
-                                 "r"(pA));
-                if (rB < rows_per_box)
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(base + swz_off<G>(rB, nt) + within),
-                                 "r"(pB));
-            }
-            const float2 fA = MmaOp<T>::unpack(mA2), fB = MmaOp<T>::unpack(mB2);
-            float mA = fmax_nan(fA.x, fA.y), mB = fmax_nan(fB.x, fB.y);
-            mA = fmax_nan(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
-            mA = fmax_nan(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
-            mB = fmax_nan(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
-            mB = fmax_nan(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
-            if ((lane & 3) == 0) {
-                if (rA < rows_per_box) atomicMax(&amax_bits[rA / p.GB], __float_as_uint(mA));
-                if (rB < rows_per_box) atomicMax(&amax_bits[rB / p.GB], __float_as_uint(mB));
-            }
+            if (abort_flag)   // copies still in flight land before the CTA leaves
+                for (int j = issued > p.S ? issued - p.S : 0; j < issued; ++j)
+                    mbar_wait(&full_bar[j % p.S], (uint32_t)(j / p.S) & 1u, nullptr, nullptr);
         }
-        __syncthreads();
-        if (tid < p.RB) {
-            const float s = row_scale(__uint_as_float(amax_bits[tid]), scale_in);
-            row_s[tid] = s;
-            if (m0 + tid < p.M) scales[m0 + tid] = s;
-        }
-        __syncthreads();
+    } else {
+        // ---------------------------------------------------------------- compute warps
+        const int group = warp / kRqGroupWarps, gw = warp % kRqGroupWarps;
+        const int gtid = tid % (kRqGroupWarps * 32);
+        const uint32_t rt_base = smem_u32(rt_sh);
+        const int rows_per_box = p.RB * p.GB;            // valid group-rows in one box
+        const int tiles_per_box = (rows_per_box + 15) / 16;
+        const int n_tiles = tiles_per_box * p.NB;
+        const int chunks_per_row = (int)(p.K / 16);
 
-        // ---- quantize: 16 consecutive channels per thread step, 16-byte code stores
-        for (int r = 0; r < p.RB; ++r) {
-            if (m0 + r >= p.M) break;
-            const RowDivisor dv(row_s[r]);
-            int8_t* dst_row = codes + (m0 + r) * p.ldq;
-            for (int c = tid; c < chunks_per_row; c += kMmaThreads) {
-                const int k = c * 16;
-                const int j = k / G, e = k - j * G;
-                int bx = 0, jj = j;
-                if (p.NB > 1) {
-                    bx = j / p.GB;
-                    jj = j - bx * p.GB;
-                }
-                const int rho = r * p.GB + jj;
-                const unsigned char* bb = buf + (size_t)bx * p.box_stride;
-                const uint4 u0 = *reinterpret_cast<const uint4*>(bb + swz_off<G>(rho, e / 8));
-                const uint4 u1 = *reinterpret_cast<const uint4*>(bb + swz_off<G>(rho, e / 8 + 1));
-                const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-                float y[16];
+        for (int i = group; i < my_blocks; i += kRqGroups) {
+            const int s = i % p.S;
+            const uint32_t par = (uint32_t)(i / p.S) & 1u;
+            const int64_t m0 = (blockIdx.x + (int64_t)i * gridDim.x) * p.RB;
+            unsigned char* buf = ring + (size_t)s * p.stage_bytes;
+            if (!mbar_wait(&full_bar[s], par, &abort_flag, dev_status)) break;
+
+            // ---- rotation: 16 consecutive group-rows per MMA tile, y written back in place
+            for (int t = gw; t < n_tiles; t += kRqGroupWarps) {
+                const int bx = t / tiles_per_box;
+                const int rho0 = (t - bx * tiles_per_box) * 16;
+                const uint32_t base = smem_u32(buf + (size_t)bx * p.box_stride);
+                uint32_t afr[KT][4];
+                {
+                    const int rho = rho0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                    const int cadd = lane >> 4;   // 0: k 0-7, 1: k 8-15 of the k-tile
 #pragma unroll
-                for (int h = 0; h < 8; ++h) {
-                    const float2 a = MmaOp<T>::unpack(w[h]);
-                    y[2 * h] = a.x;
-                    y[2 * h + 1] = a.y;
+                    for (int kt = 0; kt < KT; ++kt)
+                        ldmatrix_x4(afr[kt], base + swz_off<G>(rho, kt * 2 + cadd));
                 }
-                uint32_t out[4];
-                quant16(y, dv, out);
-                int8_t* dst = dst_row + k;
-                if (p.vec_codes) {
-                    *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
-                } else {
+                float acc[NT][4];
 #pragma unroll
-                    for (int q = 0; q < 16; ++q)
-                        dst[q] = (int8_t)((out[q / 4] >> (8 * (q % 4))) & 0xFF);
+                for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt) {
+                    // B fragments of two n-tiles per ldmatrix.x4: matrices (nt, k 0-7),
+                    // (nt, k 8-15), (nt + 1, k 0-7), (nt + 1, k 8-15) of this k-tile
+#pragma unroll
+                    for (int nt = 0; nt < NT; nt += 2) {
+                        uint32_t b4[4];
+                        const int n = nt * 8 + ((lane >> 4) << 3) + (lane & 7);
+                        ldmatrix_x4(b4, rt_base + rt_off<G>(n, kt * 2 + ((lane >> 3) & 1)));
+                        MmaOp<T>::run(acc[nt], afr[kt], b4[0], b4[1]);
+                        MmaOp<T>::run(acc[nt + 1], afr[kt], b4[2], b4[3]);
+                    }
+                }
+                // round to T, store in place with stmatrix (8x8 blocks: rows rho0..+7 and
+                // rho0+8..+15 of n-tiles nt and nt + 1; rows past the box land in its padding),
+                // row absmax
+                const int rA = rho0 + (lane >> 2), rB = rA + 8;
+                uint32_t mA2 = 0u, mB2 = 0u;
+                {
+                    const int srow = rho0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                    const int sn = (lane >> 4) & 1;
+#pragma unroll
+                    for (int nt = 0; nt < NT; nt += 2) {
+                        const uint32_t pA0 = MmaOp<T>::pack(acc[nt][0], acc[nt][1]);
+                        const uint32_t pB0 = MmaOp<T>::pack(acc[nt][2], acc[nt][3]);
+                        const uint32_t pA1 = MmaOp<T>::pack(acc[nt + 1][0], acc[nt + 1][1]);
+                        const uint32_t pB1 = MmaOp<T>::pack(acc[nt + 1][2], acc[nt + 1][3]);
+                        mA2 = MmaOp<T>::absmax2(MmaOp<T>::absmax2(mA2, pA0), pA1);
+                        mB2 = MmaOp<T>::absmax2(MmaOp<T>::absmax2(mB2, pB0), pB1);
+                        stmatrix_x4(base + swz_off<G>(srow, nt + sn), pA0, pB0, pA1, pB1);
+                    }
+                }
+                const float2 fA = MmaOp<T>::unpack(mA2), fB = MmaOp<T>::unpack(mB2);
+                float mA = fmax_nan(fA.x, fA.y), mB = fmax_nan(fB.x, fB.y);
+                mA = fmax_nan(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
+                mA = fmax_nan(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
+                mB = fmax_nan(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
+                mB = fmax_nan(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
+                if ((lane & 3) == 0) {
+                    if (rA < rows_per_box) atomicMax(&amax_bits[s][rA / p.GB], __float_as_uint(mA));
+                    if (rB < rows_per_box) atomicMax(&amax_bits[s][rB / p.GB], __float_as_uint(mB));
                 }
             }
-        }
-        __syncthreads();
-        // the buffer is free again: fetch the block two steps ahead into it
-        if (tid == 0) {
-            const int64_t nb = blk + 2LL * gridDim.x;
-            if (nb < n_blocks) issue(b, nb);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&rot_done[s]);
+            if (!mbar_wait(&rot_done[s], par, &abort_flag, dev_status)) break;
+
+            // ---- row scales (the group's first warp), published through scale_ready
+            if (gw == 0) {
+                if (lane < p.RB) {
+                    const float sc = row_scale(__uint_as_float(amax_bits[s][lane]), scale_in);
+                    const RowDivisor dv(sc);
+                    row_s[s][lane] = sc;
+                    row_r[s][lane] = dv.r;
+                    amax_bits[s][lane] = 0u;     // ready for the stage's next block
+                    if (m0 + lane < p.M) scales[m0 + lane] = sc;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&scale_ready[s]);
+            }
+            if (!mbar_wait(&scale_ready[s], par, &abort_flag, dev_status)) break;
+
+            // ---- quantize: 16 consecutive channels per thread step, 16-byte code stores
+            for (int r = 0; r < p.RB; ++r) {
+                if (m0 + r >= p.M) break;
+                RowDivisor dv(row_s[s][r]);
+                dv.r = row_r[s][r];
+                int8_t* dst_row = codes + (m0 + r) * p.ldq;
+                for (int c = gtid; c < chunks_per_row; c += kRqGroupWarps * 32) {
+                    const int k = c * 16;
+                    const int j = k / G, e = k - j * G;
+                    int bx = 0, jj = j;
+                    if (p.NB > 1) {
+                        bx = j / p.GB;
+                        jj = j - bx * p.GB;
+                    }
+                    const int rho = r * p.GB + jj;
+                    const unsigned char* bb = buf + (size_t)bx * p.box_stride;
+                    const uint4 u0 = *reinterpret_cast<const uint4*>(bb + swz_off<G>(rho, e / 8));
+                    const uint4 u1 = *reinterpret_cast<const uint4*>(bb + swz_off<G>(rho, e / 8 + 1));
+                    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+                    float y[16];
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) {
+                        const float2 a = MmaOp<T>::unpack(w[h]);
+                        y[2 * h] = a.x;
+                        y[2 * h + 1] = a.y;
+                    }
+                    uint32_t out[4];
+                    quant16(y, dv, out);
+                    int8_t* dst = dst_row + k;
+                    if (p.vec_codes) {
+                        *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 16; ++q)
+                            dst[q] = (int8_t)((out[q / 4] >> (8 * (q % 4))) & 0xFF);
+                    }
+                }
+            }
+            // the stage's shared memory is no longer read by this warp
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_bar[s]);
         }
     }
+    __syncthreads();
 }
 
 // ===================================================================== host launch
@@ -427,20 +481,23 @@ static ck_status launch_mma(const void* x, int64_t M, int64_t K, int64_t sm, con
     p.Gn = (int)(K / G);
     p.NB = (p.Gn + 255) / 256;
     p.GB = (p.Gn + p.NB - 1) / p.NB;
-    // rows per block: two buffers per CTA within about 100 KB (two CTAs per SM), and
-    // enough blocks for every CTA
     const int sms = num_sms();
     auto stride_for = [&](int rb) {
         const uint32_t tile_rows = (uint32_t)(((rb * p.GB) + 15) / 16 * 16);
         return (tile_rows * G * 2 + 1023u) & ~1023u;
     };
+    // rows per block: a stage of about 32 KB, and at least 4 blocks per CTA
     int RB = 16;
-    while (RB > 1 && 2ULL * stride_for(RB) * p.NB > 100 * 1024) RB >>= 1;
-    while (RB > 1 && (M + RB - 1) / RB < 2LL * sms) RB >>= 1;
+    while (RB > 1 && (size_t)stride_for(RB) * p.NB > 36 * 1024) RB >>= 1;
+    while (RB > 1 && (M + RB - 1) / RB < 4LL * sms) RB >>= 1;
     p.RB = RB;
     p.box_bytes = (uint32_t)(RB * p.GB * G * 2);
     p.box_stride = stride_for(RB);
-    p.buf_bytes = p.box_stride * (uint32_t)p.NB;
+    p.stage_bytes = p.box_stride * (uint32_t)p.NB;
+    // ring depth: as many stages as fit in about 190 KB
+    p.S = (int)((190u * 1024u) / p.stage_bytes);
+    if (p.S > kRqMaxStages) p.S = kRqMaxStages;
+    if (p.S < 2) return CK_ERR_UNSUPPORTED;
     p.vec_codes = (aligned(codes, 16) && ldq % 16 == 0) ? 1 : 0;
 
     CUtensorMap map;
@@ -451,15 +508,15 @@ static ck_status launch_mma(const void* x, int64_t M, int64_t K, int64_t sm, con
                               G == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B);
     if (st != CK_OK) return st;
 
-    const size_t smem = 2 * (size_t)p.buf_bytes + 1024;
+    const size_t smem = (size_t)p.S * p.stage_bytes + 1024;
     auto kern = rq_mma_kernel<T, G>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return CK_ERR_CUDA;
     const int64_t n_blocks = (M + RB - 1) / RB;
-    int grid = (int)(n_blocks < 2LL * sms ? n_blocks : 2LL * sms);
-    kern<<<grid, kMmaThreads, smem, stream>>>(map, static_cast<const T*>(R), scale_in, codes,
-                                              scales, p, dev_status);
+    const int grid = (int)(n_blocks < sms ? n_blocks : sms);
+    kern<<<grid, kRqThreads, smem, stream>>>(map, static_cast<const T*>(R), scale_in, codes,
+                                             scales, p, dev_status);
     return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 
