@@ -9,26 +9,36 @@
 //   acc[m, n] = sum_k q[m, k] * w[n, k]
 //   out[m, n] = cvt(((fp32(acc) * a_scale[m]) * w_scale[n]) + bias[n])
 //
-// Persistent, warp-specialised, one CTA per SM, 128 x BN output tiles (BN <= 240):
-//   warp 0      TMA producer of the A codes (128 rows x 128 bytes, 128-byte swizzle), 4-stage ring
-//   warp 2      TMA producer of the packed weights (BN rows x 64 bytes), 3-stage ring
-//   warps 8-17  unpack each packed stage into the unpacked-weight ring (3 stages) in the
-//               128-byte-swizzled K-major layout the tensor core reads
-//   warp 1      TMEM allocation and the single MMA-issuing thread:
-//               tcgen05.mma.cta_group::1.kind::i8, 128 x (BN + 16) x 32 per instruction,
-//               into one of two TMEM accumulators (2 x 256 columns)
-//   warps 4-7   epilogue: tcgen05.ld of the finished accumulator, fp32 scale/bias, store,
-//               overlapped with the MMAs of the next tile
+// Persistent, warp-specialised, one CTA per SM.  The unpacked weights are the MMA's A
+// operand and live in tensor memory; the activation codes are its B operand, staged in
+// shared memory by TMA.  A tile is 128 output channels x BNA activation rows (BNA <= 192)
+// and is accumulated transposed, D[n, m] (TMEM lane = channel n, column = row m):
+//   warp 0      TMA producer of the codes: BNA rows x 128 bytes per stage, 128-byte swizzle
+//   warp 2      TMA producer of the packed weights: 128 rows x 64 bytes, 64-byte swizzle
+//   warps 8-23  unpack, in two sets of eight that take alternate super-stages: each thread
+//               owns one weight row (a TMEM lane) and one half of each k-block's K; it expands
+//               64 four-bit codes per k-block to bytes and writes them into the set's TMEM
+//               weight buffer with tcgen05.st
+//   warp 1      TMEM allocation and the single MMA-issuing thread: tcgen05.mma kind::i8 with
+//               A from TMEM, 128 x BNA x 32 per instruction.  Its waits, fences and commits
+//               cost far more than an MMA issue, so the ring is organised in super-stages of
+//               G k-blocks (G = 2-4): one wait for the codes, one for the weights and one
+//               commit per 4G MMAs
+//   warps 4-7, 24-27  epilogue, two warps per TMEM lane quarter taking alternate 16-row
+//               chunks: tcgen05.ld of the finished accumulator, fp32 scale/bias, and per output
+//               row one store of 32 consecutive channels per warp, overlapped with the MMAs of
+//               the next tile (two accumulators); the tile's row scales are loaded before its
+//               accumulator is ready
+// TMEM columns: accumulators [0, BNA) and [BNA, 2 BNA), then nb (2-4) weight buffers of G
+// k-blocks (32 columns each).  Every role walks its ring indices incrementally.
 //
-// Unsigned weight operand.  Each 4-bit code v in [-8, 7] is expanded to u = v + 8 in
-// [0, 15] (one LOP3 per 8 nibbles: (w & 0x0F) ^ 0x08 per byte) and the MMA runs signed A x
-// unsigned B, giving sum_k q*u = acc + 8 * sum_k q.  Sixteen extra B rows of constant 1 sit
-// after the BN weight rows of every stage (written once), so accumulator column BN holds
-// sum_k q[m, k] and the epilogue recovers acc = sum q*u - 8 * sum q exactly (mod 2^32, and
-// the true acc fits in int32 under the 64*K guard).
+// Weight bytes.  For K < 2^21 each code w is written as the byte 16 w (its nibble moved to
+// the byte's high half: two logic operations per four codes instead of a sign extension);
+// the exact accumulator 16 acc then fits in int32 (|16 acc| <= 16 * 64 * K < 2^31) and the
+// epilogue recovers acc with an arithmetic shift.  Larger K uses sign-extended bytes.
 //
-// Every wait is bounded (ck_device.cuh); out-of-range rows/columns arrive as zeros from TMA
-// and are masked at the store.
+// Every wait is bounded (ck_device.cuh); out-of-range rows, channels and K arrive as zeros
+// from TMA and are masked at the store.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -40,41 +50,43 @@
 namespace ck {
 
 namespace gemm {
-constexpr int BM = 128;                  // activation rows per tile (MMA M)
-constexpr int BK = 128;                  // K elements (bytes of A) per stage
-constexpr int BN_MAX = 240;              // weight rows per tile; MMA N = BN + 16 <= 256
-constexpr int ONES = 16;                 // constant-one B rows that produce the row sums
-constexpr int A_ST = 4, WP_ST = 3, B_ST = 3;
-constexpr int A_BYTES = BM * BK;         // 16 KB
-constexpr int WARP_TMA_A = 0, WARP_MMA = 1, WARP_TMA_W = 2;
-constexpr int EPI_WARP0 = 4;             // warps 4..7 own TMEM lanes 0..127
-constexpr int UNP_WARP0 = 8, UNP_WARPS = 10;
-constexpr int UNP_THREADS = UNP_WARPS * 32;
-constexpr int THREADS = UNP_WARP0 * 32 + UNP_THREADS;
-// unpack task = (row, quarter): 16 packed bytes -> 32 codes.  Thread ut takes tasks
-// ut + UNP_THREADS * j, i.e. rows (ut / 4) + UNP_ROW_STEP * j with the same quarter.
-constexpr int UNP_ROW_STEP = UNP_THREADS / 4;
-constexpr int UNP_MAX_J = (BN_MAX * 4 + UNP_THREADS - 1) / UNP_THREADS;
-static_assert(UNP_ROW_STEP % 8 == 0, "row step must keep the swizzle phase");
-constexpr uint32_t TMEM_COLS = 512;      // two accumulators of 256 columns
-constexpr uint32_t ACC_COLS = 256;
-
-__host__ __device__ constexpr uint32_t wp_stage_bytes(int bn) { return (uint32_t)bn * (BK / 2); }
-__host__ __device__ constexpr uint32_t b_stage_bytes(int bn) { return (uint32_t)(bn + ONES) * BK; }
-__host__ __device__ constexpr size_t smem_bytes(int bn) {
-    return (size_t)A_ST * A_BYTES + (size_t)WP_ST * wp_stage_bytes(bn) +
-           (size_t)B_ST * b_stage_bytes(bn) + 1024;
-}
+constexpr int BW = 128;                  // weight rows (output channels) per tile: MMA M
+constexpr int BK = 128;                  // K elements per stage (bytes of codes)
+constexpr int BNA_MAX = 192;             // activation rows per tile: MMA N
+constexpr int XS_MAX = 8;                // code super-stages in shared memory
+constexpr int G_MAX = 4;                 // k-blocks per super-stage
+constexpr int NB_MAX = 4;                // TMEM weight buffers (one super-stage each)
+constexpr int W_ST_MAX = 2 * G_MAX;      // packed-weight stages (one k-block each): 2G
+constexpr int ND = 16;                   // super-stage completion barriers (> XS_MAX + 1)
+constexpr uint32_t W_BYTES = BW * BK / 2;    // 8 KB
+constexpr uint32_t A_STAGE_COLS = BK / 4;    // 32 TMEM columns of 4 bytes per stage
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int WARP_TMA_X = 0, WARP_MMA = 1, WARP_TMA_W = 2;
+// epilogue: warps 4..7 and 24..27, two per TMEM lane quarter, taking alternate 16-row chunks
+constexpr int EPI_WARP0 = 4, EPI_WARP1 = 24, EPI_WARPS = 8;
+constexpr int UNP_WARP0 = 8, UNP_SET_WARPS = 8, UNP_SETS = 2;   // warps 8..23
+constexpr int UNP_WARPS = UNP_SET_WARPS * UNP_SETS;
+constexpr int THREADS = (EPI_WARP1 + 4) * 32;
+constexpr int64_t SCALED16_MAX_K = (1LL << 21) - 1;   // 16 * 64 * K < 2^31
+constexpr size_t SMEM_BUDGET = 220 * 1024;
+static_assert(UNP_WARP0 % 4 == 0 && EPI_WARP0 % 4 == 0 && EPI_WARP1 % 4 == 0,
+              "TMEM lane quarters follow warp % 4");
+static_assert(UNP_WARP0 + UNP_WARPS == EPI_WARP1, "warp roles tile the CTA");
+static_assert(BNA_MAX % 32 == 0, "the epilogue preloads row scales 32 rows at a time");
+static_assert(UNP_SETS == 2, "the packed-weight stages are split between two unpack sets");
+static_assert(ND == 16 && ND > XS_MAX + 1, "completion barrier index and parity use 4 bits");
 }  // namespace gemm
 
 struct GemmParams {
     int64_t M, N, ldo;
     int num_kb;        // K blocks of BK
-    int BN;            // weight rows per tile (multiple of 16, <= BN_MAX)
-    int tiles_n;       // tiles along N
+    int BNA;           // activation rows per tile (multiple of 16, <= BNA_MAX)
+    int tiles_n;       // tiles along N (channels)
     int tiles;         // total tiles
-    uint32_t idesc;    // MMA instruction descriptor for 128 x (BN + 16)
-    int vec_out;
+    int G;             // k-blocks per super-stage
+    int nb;            // TMEM weight buffers, 2 <= nb <= NB_MAX
+    int xs;            // code super-stages in shared memory
+    uint32_t idesc;    // MMA instruction descriptor for 128 x BNA
     const float* a_scale;
     const void* w_scale;
     const void* bias;
@@ -82,14 +94,36 @@ struct GemmParams {
     int* dev_status;
 };
 
-// Eight 4-bit codes of one packed word -> eight unsigned u = v + 8 bytes in k order
-// (the low nibble of byte i is k = 2i).
-__device__ __forceinline__ void unpack_word_u(uint32_t w, uint32_t& o0, uint32_t& o1) {
-    const uint32_t lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;          // k = 0, 2, 4, 6
-    const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;   // k = 1, 3, 5, 7
-    o0 = __byte_perm(lo, hi, 0x5140);                             // k0 k1 k2 k3
-    o1 = __byte_perm(lo, hi, 0x7362);                             // k4 k5 k6 k7
+// Eight signed 4-bit codes of one packed word -> eight sign-extended bytes in k order (the
+// low nibble of byte i is k = 2i).  Per byte, a nibble x in [0, 15] becomes
+// ((x + 0x78) ^ 0x78): x for x < 8 and x + 240 (x - 16 as a signed byte) for x >= 8; the sum
+// stays below 0x100, so no carry crosses a byte.
+__device__ __forceinline__ void unpack_word_s(uint32_t w, uint32_t& o0, uint32_t& o1) {
+    const uint32_t lo = ((w & 0x0F0F0F0Fu) + 0x78787878u) ^ 0x78787878u;          // k even
+    const uint32_t hi = (((w >> 4) & 0x0F0F0F0Fu) + 0x78787878u) ^ 0x78787878u;   // k odd
+    o0 = __byte_perm(lo, hi, 0x5140);                                             // k0 k1 k2 k3
+    o1 = __byte_perm(lo, hi, 0x7362);                                             // k4 k5 k6 k7
 }
+
+// The same eight codes as the bytes 16 w: a signed nibble placed in the high half of a byte
+// reads as 16 times its value.
+__device__ __forceinline__ void unpack_word_x16(uint32_t w, uint32_t& o0, uint32_t& o1) {
+    const uint32_t lo = (w << 4) & 0xF0F0F0F0u;   // k even
+    const uint32_t hi = w & 0xF0F0F0F0u;          // k odd
+    o0 = __byte_perm(lo, hi, 0x5140);
+    o1 = __byte_perm(lo, hi, 0x7362);
+}
+
+// A ring position: slot index and the parity of the slot's current fill.
+struct RingPos {
+    uint32_t idx = 0, phase = 0;
+    __device__ __forceinline__ void step(uint32_t n) {
+        if (++idx == n) {
+            idx = 0;
+            phase ^= 1u;
+        }
+    }
+};
 
 template <typename T> __device__ __forceinline__ float load_scale(const void* p, int64_t i);
 template <> __device__ __forceinline__ float load_scale<float>(const void* p, int64_t i) {
@@ -144,270 +178,277 @@ template <> struct OutStore<__half> {
     __device__ static __forceinline__ void one(__half* dst, float v) { *dst = __float2half_rn(v); }
 };
 
-template <typename OutT, typename ScaleT>
+template <typename OutT, typename ScaleT, bool X16>
 __global__ void __launch_bounds__(gemm::THREADS, 1)
-    w4a4_gemm_kernel(const __grid_constant__ CUtensorMap amap,
+    w4a4_gemm_kernel(const __grid_constant__ CUtensorMap xmap,
                      const __grid_constant__ CUtensorMap wmap, GemmParams p) {
     using namespace gemm;
     extern __shared__ __align__(1024) unsigned char gemm_smem[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(gemm_smem) + 1023) & ~uintptr_t(1023));
-    const uint32_t wp_bytes = wp_stage_bytes(p.BN);
-    const uint32_t b_bytes = b_stage_bytes(p.BN);
-    unsigned char* a_ring = smem;
-    unsigned char* wp_ring = a_ring + (size_t)A_ST * A_BYTES;
-    unsigned char* b_ring = wp_ring + (size_t)WP_ST * wp_bytes;
+    // packed-weight stage of k-block it: it % 2G, so each unpack set has its own G stages and
+    // waits for their fills in order
+    const uint32_t G = (uint32_t)p.G, XS = (uint32_t)p.xs, W_ST = 2u * G, NB = (uint32_t)p.nb;
+    const uint32_t x_bytes = (uint32_t)p.BNA * BK;          // one k-block of codes
+    const uint32_t xss_bytes = G * x_bytes;                  // one super-stage
+    unsigned char* x_ring = smem;
+    unsigned char* w_ring = x_ring + (size_t)XS * xss_bytes;
 
-    __shared__ __align__(8) uint64_t a_full[A_ST], a_empty[A_ST];
-    __shared__ __align__(8) uint64_t wp_full[WP_ST], wp_empty[WP_ST];
-    __shared__ __align__(8) uint64_t b_full[B_ST], b_empty[B_ST];
-    __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], drain_bar, vec_ready[2];
+    __shared__ __align__(8) uint64_t x_full[XS_MAX], w_full[W_ST_MAX], w_empty[W_ST_MAX];
+    __shared__ __align__(8) uint64_t a_full[NB_MAX], done[ND];
+    __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
-    __shared__ __align__(16) float ws_sh[2][BN_MAX], bias_sh[2][BN_MAX];   // per-tile epilogue vectors
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // k-blocks this CTA runs (its tiles blockIdx.x, + gridDim.x, ... times num_kb), numbered
+    // 0.. across tiles; super-stage s holds k-blocks [s G, s G + G)
+    const uint32_t my_tiles =
+        (uint32_t)((p.tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x);
+    const uint32_t my_kb = my_tiles * (uint32_t)p.num_kb;
+    const uint32_t my_ss = (my_kb + G - 1) / G;
 
     if (tid == 0) {
-        for (int s = 0; s < A_ST; ++s) { mbar_init(&a_full[s], 1); mbar_init(&a_empty[s], 1); }
-        for (int s = 0; s < WP_ST; ++s) {
-            mbar_init(&wp_full[s], 1);
-            mbar_init(&wp_empty[s], UNP_WARPS);
+        for (int s = 0; s < XS_MAX; ++s) mbar_init(&x_full[s], 1);
+        for (int s = 0; s < W_ST_MAX; ++s) {
+            mbar_init(&w_full[s], 1);
+            mbar_init(&w_empty[s], UNP_SET_WARPS);
         }
-        for (int s = 0; s < B_ST; ++s) {
-            mbar_init(&b_full[s], UNP_WARPS);
-            mbar_init(&b_empty[s], 1);
-        }
+        for (int s = 0; s < NB_MAX; ++s) mbar_init(&a_full[s], UNP_SET_WARPS);
+        for (int s = 0; s < ND; ++s) mbar_init(&done[s], 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&acc_full[s], 1);
-            mbar_init(&acc_empty[s], 4);
-            mbar_init(&vec_ready[s], 4);
+            mbar_init(&acc_empty[s], EPI_WARPS);
         }
         mbar_init(&drain_bar, 1);
         abort_flag = 0;
         fence_mbar_init();
-        tma_prefetch_desc(&amap);
+        tma_prefetch_desc(&xmap);
         tma_prefetch_desc(&wmap);
     }
     if (warp == WARP_MMA) {
         tmem_alloc(&tmem_base_sh, TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp >= UNP_WARP0) {
-        // the constant-one rows after the weight rows of every unpacked stage
-        const int ut = tid - UNP_WARP0 * 32;
-        for (int s = 0; s < B_ST; ++s) {
-            unsigned char* ones = b_ring + (size_t)s * b_bytes + (size_t)p.BN * BK;
-            for (int i = ut; i < ONES * BK / 16; i += UNP_THREADS)
-                reinterpret_cast<uint4*>(ones)[i] = make_uint4(0x01010101u, 0x01010101u,
-                                                              0x01010101u, 0x01010101u);
-        }
-        fence_proxy_async_smem();
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_sh;
+    const uint32_t a_col0 = 2u * (uint32_t)p.BNA;
 
-    if (warp == WARP_TMA_A) {
-        // ---------------------------------------------------------------- A codes producer
+    // super-stage s completes (all its MMAs done) on done[s % 16] with parity (s / 16) & 1
+    auto wait_done = [&](uint32_t s) -> bool {
+        return mbar_wait(&done[s & (ND - 1)], (s >> 4) & 1u, &abort_flag, p.dev_status);
+    };
+
+    if (warp == WARP_TMA_X) {
+        // ---------------------------------------------------------------- codes producer
         if (lane == 0) {
-            uint32_t it = 0, issued = 0;
+            uint32_t issued = 0;
+            uint32_t slot = 0, kb = 0;
+            int t = blockIdx.x;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x) {
-                const int32_t m0 = (t / p.tiles_n) * BM;
-                for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-                    const uint32_t s = it % A_ST, r = it / A_ST;
-                    if (it >= (uint32_t)A_ST &&
-                        !mbar_wait(&a_empty[s], (r - 1) & 1u, &abort_flag, p.dev_status)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&a_full[s], A_BYTES);
-                    tma_load_2d(a_ring + (size_t)s * A_BYTES, &amap, &a_full[s], kb * BK, m0);
-                    ++issued;
+            for (uint32_t ss = 0; ok && ss < my_ss; ++ss) {
+                if (ss >= XS && !wait_done(ss - XS)) {
+                    ok = false;
+                    break;
                 }
+                const uint32_t n_k = (my_kb - ss * G) < G ? (my_kb - ss * G) : G;
+                unsigned char* dst = x_ring + (size_t)slot * xss_bytes;
+                mbar_arrive_expect_tx(&x_full[slot], n_k * x_bytes);
+                for (uint32_t j = 0; j < n_k; ++j) {
+                    const int32_t m0 = (t / p.tiles_n) * p.BNA;
+                    tma_load_2d(dst + (size_t)j * x_bytes, &xmap, &x_full[slot], (int)kb * BK, m0);
+                    if (++kb == (uint32_t)p.num_kb) {
+                        kb = 0;
+                        t += gridDim.x;
+                    }
+                }
+                ++issued;
+                if (++slot == XS) slot = 0;
             }
-            if (!ok)
-                for (uint32_t j = issued > A_ST ? issued - A_ST : 0; j < issued; ++j)
-                    mbar_wait(&a_full[j % A_ST], (j / A_ST) & 1u, nullptr, nullptr);
+            if (!ok)   // copies still in flight land before the CTA leaves
+                for (uint32_t j = issued > XS ? issued - XS : 0; j < issued; ++j)
+                    mbar_wait(&x_full[j % XS], (j / XS) & 1u, nullptr, nullptr);
         }
     } else if (warp == WARP_TMA_W) {
         // ---------------------------------------------------------------- packed W producer
         if (lane == 0) {
             uint32_t it = 0, issued = 0;
+            RingPos rw;
             bool ok = true;
             for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x) {
-                const int32_t n0 = (t % p.tiles_n) * p.BN;
-                for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-                    const uint32_t s = it % WP_ST, r = it / WP_ST;
-                    if (it >= (uint32_t)WP_ST &&
-                        !mbar_wait(&wp_empty[s], (r - 1) & 1u, &abort_flag, p.dev_status)) {
+                const int32_t n0 = (t % p.tiles_n) * BW;
+                for (int kb = 0; kb < p.num_kb; ++kb, ++it, rw.step(W_ST)) {
+                    if (it >= W_ST && !mbar_wait(&w_empty[rw.idx], rw.phase ^ 1u, &abort_flag,
+                                                 p.dev_status)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&wp_full[s], wp_bytes);
-                    tma_load_2d(wp_ring + (size_t)s * wp_bytes, &wmap, &wp_full[s], kb * (BK / 2),
-                                n0);
+                    mbar_arrive_expect_tx(&w_full[rw.idx], W_BYTES);
+                    tma_load_2d(w_ring + (size_t)rw.idx * W_BYTES, &wmap, &w_full[rw.idx],
+                                kb * (BK / 2), n0);
                     ++issued;
                 }
             }
             if (!ok)
-                for (uint32_t j = issued > WP_ST ? issued - WP_ST : 0; j < issued; ++j)
-                    mbar_wait(&wp_full[j % WP_ST], (j / WP_ST) & 1u, nullptr, nullptr);
+                for (uint32_t j = issued > W_ST ? issued - W_ST : 0; j < issued; ++j)
+                    mbar_wait(&w_full[j % W_ST], (j / W_ST) & 1u, nullptr, nullptr);
         }
     } else if (warp == WARP_MMA) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            uint32_t it = 0, lt = 0;
+            // descriptor of code k-block 0 of slot 0; k-block j of slot s starts
+            // (s G + j) x_bytes later (start-address field counts 16-byte units)
+            const uint64_t bdesc0 = smem_desc_k_sw128(smem_u32(x_ring));
+            const uint32_t kstep = x_bytes >> 4;
+            uint32_t slot = 0, xphase = 0, kb = 0, lt = 0;
+            RingPos rb;   // TMEM weight buffer of the super-stage
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++lt) {
-                const uint32_t acc = lt & 1u;
-                if (lt >= 2 && !mbar_wait(&acc_empty[acc], ((lt >> 1) - 1) & 1u, &abort_flag,
-                                          p.dev_status)) {
+            uint32_t d_tmem = tmem_base;
+            for (uint32_t ss = 0; ok && ss < my_ss; ++ss, rb.step(NB)) {
+                if (!mbar_wait(&x_full[slot], xphase, &abort_flag, p.dev_status) ||
+                    !mbar_wait(&a_full[rb.idx], rb.phase, &abort_flag, p.dev_status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
-                for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-                    const uint32_t sa = it % A_ST, sb = it % B_ST;
-                    if (!mbar_wait(&a_full[sa], (it / A_ST) & 1u, &abort_flag, p.dev_status) ||
-                        !mbar_wait(&b_full[sb], (it / B_ST) & 1u, &abort_flag, p.dev_status)) {
-                        ok = false;
-                        break;
+                const uint32_t n_k = (my_kb - ss * G) < G ? (my_kb - ss * G) : G;
+                const uint32_t a_ss = tmem_base + a_col0 + rb.idx * G * A_STAGE_COLS;
+                for (uint32_t j = 0; j < n_k; ++j) {
+                    if (kb == 0) {
+                        // a new tile: its accumulator must have been drained by the epilogue
+                        const uint32_t acc = lt & 1u;
+                        if (lt >= 2 && !mbar_wait(&acc_empty[acc], ((lt >> 1) - 1) & 1u, &abort_flag,
+                                                  p.dev_status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        d_tmem = tmem_base + acc * (uint32_t)p.BNA;
                     }
-                    tc_fence_after();
-                    const uint64_t adesc = smem_desc_k_sw128(smem_u32(a_ring + (size_t)sa * A_BYTES));
-                    const uint64_t bdesc = smem_desc_k_sw128(smem_u32(b_ring + (size_t)sb * b_bytes));
+                    const uint64_t bdesc = bdesc0 + (uint64_t)((slot * G + j) * kstep);
+                    const uint32_t a_tmem = a_ss + j * A_STAGE_COLS;
 #pragma unroll
                     for (int kk = 0; kk < BK / 32; ++kk) {
-                        // advance 32 bytes (one MMA K step) inside the 128-byte swizzled row
-                        tc_mma_i8(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2),
-                                  p.idesc, (kb | kk) != 0 ? 1u : 0u);
+                        // one MMA K step: 32 bytes = 8 TMEM columns of A, 32 bytes of the
+                        // 128-byte swizzled B row
+                        tc_mma_i8_ts(d_tmem, a_tmem + (uint32_t)(kk * 8), bdesc + (uint64_t)(kk * 2),
+                                     p.idesc, (kb | (uint32_t)kk) != 0 ? 1u : 0u);
                     }
-                    tc_commit(&a_empty[sa]);
-                    tc_commit(&b_empty[sb]);
+                    if (++kb == (uint32_t)p.num_kb) {
+                        tc_commit(&acc_full[lt & 1u]);
+                        kb = 0;
+                        ++lt;
+                    }
                 }
-                if (ok) tc_commit(&acc_full[acc]);
+                if (!ok) break;
+                tc_commit(&done[ss & (ND - 1)]);
+                if (++slot == XS) {
+                    slot = 0;
+                    xphase ^= 1u;
+                }
             }
             // every MMA issued above has completed once drain_bar flips
             tc_commit(&drain_bar);
             mbar_wait(&drain_bar, 0, nullptr, p.dev_status);
         }
-    } else if (warp >= UNP_WARP0) {
-        // ---------------------------------------------------------------- unpack
-        constexpr int ROW_STEP = UNP_ROW_STEP;
-        const int ut = tid - UNP_WARP0 * 32;
-        const int row0 = ut >> 2, q = ut & 3;
-        const int n_j = (p.BN * 4 - ut + UNP_THREADS - 1) / UNP_THREADS;   // 0..UNP_MAX_J
-        const uint32_t ld_off = (uint32_t)(row0 * 64 + q * 16);
-        const uint32_t st_base = (uint32_t)((row0 >> 3) * 1024 + (row0 & 7) * 128);
-        const uint32_t st_off0 = st_base + (uint32_t)(((2 * q) ^ (row0 & 7)) << 4);
-        const uint32_t st_off1 = st_base + (uint32_t)(((2 * q + 1) ^ (row0 & 7)) << 4);
-        uint32_t it = 0;
+    } else if (warp >= UNP_WARP0 && warp < UNP_WARP0 + UNP_WARPS) {
+        // ---------------------------------------------------------------- unpack into TMEM
+        const int u = warp - UNP_WARP0;
+        const int q = warp & 3;                        // TMEM lanes 32q .. 32q + 31
+        const int h = (u >> 2) & 1;                    // K half of each k-block
+        const uint32_t set = (uint32_t)(u / UNP_SET_WARPS);   // super-stages ss == set (mod 2)
+        const int r = q * 32 + lane;                   // weight row of the tile
+        // 16-byte chunks 2h and 2h + 1 of the row under the 64-byte swizzle (chunk index
+        // XOR address bits 7-8, i.e. (r >> 1) & 3 for 64-byte rows)
+        const uint32_t phase = (uint32_t)((r >> 1) & 3);
+        const uint32_t off0 = (uint32_t)r * 64u + (((uint32_t)(2 * h) ^ phase) << 4);
+        const uint32_t off1 = (uint32_t)r * 64u + (((uint32_t)(2 * h + 1) ^ phase) << 4);
+        const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + a_col0 + (uint32_t)(h * 16);
         bool ok = true;
-        for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x) {
-            for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-                const uint32_t sw = it % WP_ST, sb = it % B_ST;
-                if (!mbar_wait(&wp_full[sw], (it / WP_ST) & 1u, &abort_flag, p.dev_status) ||
-                    (it >= (uint32_t)B_ST &&
-                     !mbar_wait(&b_empty[sb], ((it / B_ST) - 1) & 1u, &abort_flag, p.dev_status))) {
+        uint32_t buf = set;   // TMEM weight buffer of super-stage ss: ss % NB
+        for (uint32_t ss = set; ok && ss < my_ss; ss += UNP_SETS) {
+            // the buffer is free once the MMAs of its previous super-stage (ss - NB) completed
+            if (ss >= NB && !__all_sync(0xffffffffu, wait_done(ss - NB))) break;
+            tc_fence_after();
+            const uint32_t t_buf = t_row + buf * G * A_STAGE_COLS;
+            const uint32_t it0 = ss * G;
+            const uint32_t n_k = (my_kb - it0) < G ? (my_kb - it0) : G;
+            for (uint32_t j = 0; j < n_k; ++j) {
+                // k-block it0 + j: W stage (it0 + j) % 2G = set G + j, fill (it0 + j) / 2G = ss / 2
+                const uint32_t sw = set * G + j;
+                // every lane waits; the warp leaves together (tcgen05.st below is .aligned)
+                if (!__all_sync(0xffffffffu, mbar_wait(&w_full[sw], (ss >> 1) & 1u, &abort_flag,
+                                                       p.dev_status))) {
                     ok = false;
                     break;
                 }
-                const unsigned char* wp = wp_ring + (size_t)sw * wp_bytes + ld_off;
-                unsigned char* bdst = b_ring + (size_t)sb * b_bytes;
-                // all loads first (row step j: ROW_STEP * 64 packed bytes further, and
-                // ROW_STEP / 8 swizzle atoms of ROW_STEP * 128 bytes in the unpacked tile)
-                uint4 v[UNP_MAX_J];
-#pragma unroll
-                for (int j = 0; j < UNP_MAX_J; ++j)
-                    v[j] = *reinterpret_cast<const uint4*>(wp + (j < n_j ? j : 0) * ROW_STEP * 64);
-#pragma unroll
-                for (int j = 0; j < UNP_MAX_J; ++j) {
-                    uint4 o0, o1;
-                    unpack_word_u(v[j].x, o0.x, o0.y);
-                    unpack_word_u(v[j].y, o0.z, o0.w);
-                    unpack_word_u(v[j].z, o1.x, o1.y);
-                    unpack_word_u(v[j].w, o1.z, o1.w);
-                    if (j < n_j) {
-                        *reinterpret_cast<uint4*>(bdst + st_off0 + j * (ROW_STEP * BK)) = o0;
-                        *reinterpret_cast<uint4*>(bdst + st_off1 + j * (ROW_STEP * BK)) = o1;
-                    }
-                }
-                fence_proxy_async_smem();
+                const unsigned char* wst = w_ring + (size_t)sw * W_BYTES;
+                const uint4 c0 = *reinterpret_cast<const uint4*>(wst + off0);
+                const uint4 c1 = *reinterpret_cast<const uint4*>(wst + off1);
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&wp_empty[sw]);
-                    mbar_arrive(&b_full[sb]);
+                if (lane == 0) mbar_arrive(&w_empty[sw]);
+                uint32_t v[16];
+                const uint32_t c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (X16) unpack_word_x16(c[i], v[2 * i], v[2 * i + 1]);
+                    else unpack_word_s(c[i], v[2 * i], v[2 * i + 1]);
                 }
+                tc_st_32x32b_x16(t_buf + j * A_STAGE_COLS, v);
             }
+            if (!ok) break;
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[buf]);
+            buf += UNP_SETS;
+            if (buf >= NB) buf -= NB;
         }
-    } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
+    } else if ((warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) || warp >= EPI_WARP1) {
         // ---------------------------------------------------------------- epilogue
-        const int qd = warp & 3;   // TMEM lanes 32*qd .. 32*qd + 31
-        const int et = tid - EPI_WARP0 * 32;
+        const int q = warp & 3;                        // TMEM lanes 32q .. 32q + 31
+        const int eh = warp >= EPI_WARP1 ? 1 : 0;      // rows 32k + 16 eh .. + 15 of each 32
         uint32_t lt = 0;
         for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++lt) {
             const uint32_t acc = lt & 1u;
-            const int64_t m0 = (int64_t)(t / p.tiles_n) * BM;
-            const int64_t n0 = (int64_t)(t % p.tiles_n) * p.BN;
-            // this tile's weight scales and bias, once, into the buffer of its parity; each
-            // epilogue warp arrives on vec_ready after its share.  A warp rewrites a buffer
-            // only after the previous tile's vec_ready phase, for which every warp arrived
-            // after finishing the tile that last read it.
-            float* ws_t = ws_sh[acc];
-            float* bs_t = bias_sh[acc];
-            for (int i = et; i < p.BN; i += 128) {
-                const int64_t n = n0 + i;
-                ws_t[i] = n < p.N ? load_scale<ScaleT>(p.w_scale, n) : 0.f;
-                bs_t[i] = (p.bias && n < p.N) ? load_scale<ScaleT>(p.bias, n) : 0.f;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&vec_ready[acc]);
-            if (!mbar_wait(&vec_ready[acc], (lt >> 1) & 1u, &abort_flag, p.dev_status)) break;
-            if (!mbar_wait(&acc_full[acc], (lt >> 1) & 1u, &abort_flag, p.dev_status)) break;
+            const int64_t m0 = (int64_t)(t / p.tiles_n) * p.BNA;
+            const int64_t n = (int64_t)(t % p.tiles_n) * BW + q * 32 + lane;   // channel
+            const bool n_ok = n < p.N;
+            const float ws = n_ok ? load_scale<ScaleT>(p.w_scale, n) : 0.f;
+            const float bs = (p.bias && n_ok) ? load_scale<ScaleT>(p.bias, n) : 0.f;
+            const int rows = (int)((p.M - m0) < p.BNA ? (p.M - m0) : p.BNA);
+            // the tile's row scales, loaded before the accumulator is ready: lane l of
+            // as_r[k] holds a_scale[m0 + 32k + l]
+            float as_r[BNA_MAX / 32];
+#pragma unroll
+            for (int k = 0; k < BNA_MAX / 32; ++k)
+                as_r[k] = (32 * k + lane < rows) ? __ldg(p.a_scale + m0 + 32 * k + lane) : 0.f;
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(&acc_full[acc], (lt >> 1) & 1u, &abort_flag, p.dev_status)))
+                break;
             tc_fence_after();
-            const int64_t row = m0 + qd * 32 + lane;
-            const bool row_ok = row < p.M;
-            const float a_s = row_ok ? __ldg(p.a_scale + row) : 0.f;
-            const uint32_t tbase = tmem_base + acc * ACC_COLS + ((uint32_t)(qd * 32) << 16);
-            uint32_t rs[16];
-            tc_ld_32x32b_x16(tbase + (uint32_t)p.BN, rs);   // sum_k q[row, k] (16 copies)
-            tc_wait_ld();
-            const uint32_t corr = rs[0] * 8u;
-            OutT* orow = static_cast<OutT*>(p.out) + (row_ok ? row : 0) * p.ldo;
-            for (int c0 = 0; c0 < p.BN; c0 += 16) {
-                uint32_t r[16];
-                tc_ld_32x32b_x16(tbase + (uint32_t)c0, r);
-                tc_wait_ld();
-                const int64_t nb = n0 + c0;
-                float v[16], wsv[16];
+            const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + acc * (uint32_t)p.BNA;
+            OutT* ocol = static_cast<OutT*>(p.out) + (n_ok ? n : 0);
 #pragma unroll
-                for (int i = 0; i < 16; i += 4)
-                    *reinterpret_cast<float4*>(&wsv[i]) = *reinterpret_cast<const float4*>(ws_t + c0 + i);
+            for (int k = 0; k < BNA_MAX / 32; ++k) {
+                const int c0 = 32 * k + 16 * eh;       // first row of this warp's chunk
+                if (c0 < rows) {
+                    uint32_t r[16];
+                    tc_ld_32x32b_x16(tacc + (uint32_t)c0, r);
+                    tc_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float o = __int2float_rn((int)(r[i] - corr));
-                    o = __fmul_rn(o, a_s);
-                    v[i] = __fmul_rn(o, wsv[i]);
-                }
-                if (p.bias) {
-                    float bv[16];
-#pragma unroll
-                    for (int i = 0; i < 16; i += 4)
-                        *reinterpret_cast<float4*>(&bv[i]) =
-                            *reinterpret_cast<const float4*>(bs_t + c0 + i);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = __fadd_rn(v[i], bv[i]);
-                }
-                if (row_ok && nb < p.N) {
-                    if (p.vec_out && nb + 16 <= p.N) {
-                        OutStore<OutT>::vec16(orow + nb, v);
-                    } else {
-                        for (int i = 0; i < 16; ++i)
-                            if (nb + i < p.N) OutStore<OutT>::one(orow + nb + i, v[i]);
+                    for (int j = 0; j < 16; ++j) {
+                        const float a_s = __shfl_sync(0xffffffffu, as_r[k], 16 * eh + j);
+                        if (c0 + j < rows) {
+                            const int accv = X16 ? ((int)r[j] >> 4) : (int)r[j];   // exact: 16 | acc
+                            float o = __int2float_rn(accv);
+                            o = __fmul_rn(o, a_s);
+                            o = __fmul_rn(o, ws);
+                            if (p.bias) o = __fadd_rn(o, bs);
+                            if (n_ok) OutStore<OutT>::one(ocol + (m0 + c0 + j) * p.ldo, o);
+                        }
                     }
                 }
             }
@@ -426,41 +467,44 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
 }
 
 template <typename OutT, typename ScaleT>
-static ck_status launch_typed(const CUtensorMap& amap, const CUtensorMap& wmap,
-                              const GemmParams& p, int grid, cudaStream_t stream) {
-    auto kern = w4a4_gemm_kernel<OutT, ScaleT>;
-    const size_t smem = gemm::smem_bytes(p.BN);
+static ck_status launch_typed(const CUtensorMap& xmap, const CUtensorMap& wmap,
+                              const GemmParams& p, size_t smem, int grid, bool x16,
+                              cudaStream_t stream) {
+    auto kern = x16 ? w4a4_gemm_kernel<OutT, ScaleT, true> : w4a4_gemm_kernel<OutT, ScaleT, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return CK_ERR_CUDA;
-    kern<<<grid, gemm::THREADS, smem, stream>>>(amap, wmap, p);
+    kern<<<grid, gemm::THREADS, smem, stream>>>(xmap, wmap, p);
     return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 
 template <typename OutT>
-static ck_status launch_out(const CUtensorMap& amap, const CUtensorMap& wmap, const GemmParams& p,
-                            int grid, ck_dtype scale_dt, cudaStream_t stream) {
+static ck_status launch_out(const CUtensorMap& xmap, const CUtensorMap& wmap, const GemmParams& p,
+                            size_t smem, int grid, bool x16, ck_dtype scale_dt,
+                            cudaStream_t stream) {
     switch (scale_dt) {
-        case CK_F32: return launch_typed<OutT, float>(amap, wmap, p, grid, stream);
-        case CK_F16: return launch_typed<OutT, __half>(amap, wmap, p, grid, stream);
-        case CK_BF16: return launch_typed<OutT, __nv_bfloat16>(amap, wmap, p, grid, stream);
+        case CK_F32: return launch_typed<OutT, float>(xmap, wmap, p, smem, grid, x16, stream);
+        case CK_F16: return launch_typed<OutT, __half>(xmap, wmap, p, smem, grid, x16, stream);
+        case CK_BF16:
+            return launch_typed<OutT, __nv_bfloat16>(xmap, wmap, p, smem, grid, x16, stream);
         default: return CK_ERR_INVALID_ARG;
     }
 }
 
-// Tile width along N: the multiple of 16 (<= 240) that minimises the persistent schedule's
-// length, (waves of 128 x BN tiles over the SMs) x BN, preferring wider tiles on ties.
-static int choose_bn(int64_t M, int64_t N, int sms) {
-    const int64_t tiles_m = (M + gemm::BM - 1) / gemm::BM;
-    int best = gemm::BN_MAX;
+// Activation rows per tile: the multiple of 16 (<= 192) that minimises the persistent
+// schedule's length, (tiles of the busiest CTA) x (BNA + a small per-tile overhead),
+// preferring wider tiles on ties.
+static int choose_bna(int64_t M, int64_t N, int sms) {
+    const int64_t tiles_n = (N + gemm::BW - 1) / gemm::BW;
+    int best = gemm::BNA_MAX;
     int64_t best_cost = -1;
-    for (int bn = gemm::BN_MAX; bn >= 64; bn -= 16) {
-        const int64_t tiles = tiles_m * ((N + bn - 1) / bn);
-        const int64_t waves = (tiles + sms - 1) / sms;
-        const int64_t cost = waves * (bn + gemm::ONES);
+    for (int bna = gemm::BNA_MAX; bna >= 16; bna -= 16) {
+        const int64_t tiles = tiles_n * ((M + bna - 1) / bna);
+        const int64_t per_cta = (tiles + sms - 1) / sms;
+        const int64_t cost = per_cta * (bna + 32);
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
-            best = bn;
+            best = bna;
         }
     }
     return best;
@@ -473,49 +517,62 @@ ck_status launch_w4a4_gemm(const int8_t* codes, int64_t ldq, const float* a_scal
     using namespace gemm;
     if (M == 0 || N == 0) return CK_OK;
     const int sms = num_sms();
-    const int BN = choose_bn(M, N, sms);
-    CUtensorMap amap, wmap;
+    GemmParams p;
+    p.BNA = choose_bna(M, N, sms);
+    CUtensorMap xmap, wmap;
     {
         const uint64_t dims[2] = {(uint64_t)K, (uint64_t)M};
         const uint64_t strides[1] = {(uint64_t)ldq};
-        const uint32_t box[2] = {BK, BM};
-        ck_status st = encode_tma(&amap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, dims, strides,
+        const uint32_t box[2] = {BK, (uint32_t)p.BNA};
+        ck_status st = encode_tma(&xmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, dims, strides,
                                   box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (st != CK_OK) return st;
     }
     {
         const uint64_t dims[2] = {(uint64_t)(K / 2), (uint64_t)N};
         const uint64_t strides[1] = {(uint64_t)w_ld};
-        const uint32_t box[2] = {BK / 2, (uint32_t)BN};
+        const uint32_t box[2] = {BK / 2, BW};
         ck_status st = encode_tma(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w_packed, dims, strides,
-                                  box, CU_TENSOR_MAP_SWIZZLE_NONE);
+                                  box, CU_TENSOR_MAP_SWIZZLE_64B);
         if (st != CK_OK) return st;
     }
-    GemmParams p;
     p.M = M;
     p.N = N;
     p.ldo = ldo;
     p.num_kb = (int)((K + BK - 1) / BK);
-    p.BN = BN;
-    p.tiles_n = (int)((N + BN - 1) / BN);
-    const int64_t tiles = (int64_t)p.tiles_n * ((M + BM - 1) / BM);
+    p.tiles_n = (int)((N + BW - 1) / BW);
+    const int64_t tiles = (int64_t)p.tiles_n * ((M + p.BNA - 1) / p.BNA);
     if (tiles >= (1LL << 31)) return CK_ERR_UNSUPPORTED;
     p.tiles = (int)tiles;
-    // signed 8-bit A, unsigned 8-bit B, s32 accumulator, 128 x (BN + 16)
-    p.idesc = (2u << 4) | (1u << 7) | (0u << 10) | ((uint32_t)((BN + ONES) >> 3) << 17) |
-              ((uint32_t)(BM >> 4) << 24);
-    const size_t osz = out_dt == CK_F32 ? 4 : 2;
-    p.vec_out = (aligned(out, 16) && (ldo * (int64_t)osz) % 16 == 0) ? 1 : 0;
+    // TMEM: two accumulators of BNA columns; the rest holds the two weight buffers of G
+    // k-blocks (32 columns each)
+    // two k-blocks per super-stage and as many weight buffers as fit (2..4): the unpack of a
+    // super-stage may start once the MMAs of the super-stage nb before it completed
+    p.G = 2;
+    p.nb = (int)((TMEM_COLS - 2u * (uint32_t)p.BNA) / ((uint32_t)p.G * A_STAGE_COLS));
+    if (p.nb > NB_MAX) p.nb = NB_MAX;
+    if (p.nb < 2) return CK_ERR_UNSUPPORTED;
+    const size_t xss_bytes = (size_t)p.G * p.BNA * BK;
+    const size_t w_ring_bytes = (size_t)2 * p.G * W_BYTES;
+    p.xs = (int)((SMEM_BUDGET - w_ring_bytes) / xss_bytes);
+    if (p.xs > XS_MAX) p.xs = XS_MAX;
+    if (p.G < 1 || p.xs < 2) return CK_ERR_UNSUPPORTED;
+    const size_t smem = (size_t)p.xs * xss_bytes + w_ring_bytes + 1024;
+    // signed 8-bit A and B, s32 accumulator, 128 x BNA
+    p.idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(p.BNA >> 3) << 17) |
+              ((uint32_t)(BW >> 4) << 24);
     p.a_scale = a_scale;
     p.w_scale = w_scale;
     p.bias = bias;
     p.out = out;
     p.dev_status = dev_status;
     const int grid = (int)(p.tiles < sms ? p.tiles : sms);
+    const bool x16 = K <= SCALED16_MAX_K;
     switch (out_dt) {
-        case CK_F32: return launch_out<float>(amap, wmap, p, grid, scale_dt, stream);
-        case CK_F16: return launch_out<__half>(amap, wmap, p, grid, scale_dt, stream);
-        case CK_BF16: return launch_out<__nv_bfloat16>(amap, wmap, p, grid, scale_dt, stream);
+        case CK_F32: return launch_out<float>(xmap, wmap, p, smem, grid, x16, scale_dt, stream);
+        case CK_F16: return launch_out<__half>(xmap, wmap, p, smem, grid, x16, scale_dt, stream);
+        case CK_BF16:
+            return launch_out<__nv_bfloat16>(xmap, wmap, p, smem, grid, x16, scale_dt, stream);
         default: return CK_ERR_INVALID_ARG;
     }
 }
