@@ -77,33 +77,56 @@ def recorded_traffic(kernel_file: str, workload: str):
 
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while the timed region runs."""
+    """Samples SM clocks and throttle reasons while the timed region runs: through NVML every
+    10 ms when nvidia_ml_py is importable, else through nvidia-smi every 200 ms."""
 
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
     FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
         self.idx = device_index
-        self.samples = []
+        self.samples = []     # (sm_mhz, max_mhz, [reason flags in NAMES order])
         self._stop = threading.Event()
         self._t = None
+        self._nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._bits = [pynvml.nvmlClocksThrottleReasonHwSlowdown,
+                          pynvml.nvmlClocksThrottleReasonHwThermalSlowdown,
+                          pynvml.nvmlClocksThrottleReasonSwThermalSlowdown,
+                          pynvml.nvmlClocksThrottleReasonSwPowerCap]
+        except Exception:
+            self._nvml = None
 
     def _one(self):
         try:
+            if self._nvml is not None:
+                n = self._nvml
+                sm = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
+                mx = n.nvmlDeviceGetMaxClockInfo(self._h, n.NVML_CLOCK_SM)
+                r = n.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                self.samples.append((float(sm), float(mx), [bool(r & b) for b in self._bits]))
+                return
             r = subprocess.run(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
                                 "--format=csv,noheader,nounits"], capture_output=True, text=True,
                                timeout=5)
             vals = [v.strip() for v in r.stdout.strip().split(",")]
-            if len(vals) == 6:
-                self.samples.append(vals)
+            if len(vals) == 6 and vals[0].replace(".", "").isdigit():
+                self.samples.append((float(vals[0]), float(vals[1]),
+                                     [v.lower().startswith("active") for v in vals[2:]]))
         except Exception:
             pass
 
     def _loop(self):
+        period = 0.01 if self._nvml is not None else 0.2
         while not self._stop.is_set():
             self._one()
-            self._stop.wait(0.2)
+            self._stop.wait(period)
 
     def __enter__(self):
         self._t = threading.Thread(target=self._loop, daemon=True)
@@ -118,13 +141,11 @@ class ClockSampler:
     def summary(self):
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
-        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for s in self.samples for i in range(4)
-                          if s[2 + i].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(sm)}
+        sm = [s[0] for s in self.samples]
+        reasons = sorted({self.NAMES[i] for s in self.samples for i in range(4) if s[2][i]})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(s[1] for s in self.samples),
+                "sm_mhz_min": min(sm), "reasons": reasons, "samples": len(sm),
+                "source": "nvml" if self._nvml is not None else "nvidia-smi"}
 
 
 def dist_setup():
