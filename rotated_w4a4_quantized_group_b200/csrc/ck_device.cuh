@@ -319,27 +319,29 @@ __device__ __forceinline__ float2 mul2_rn(float a0, float a1, float b) {
 }
 
 // Sixteen codes of one row (divisor d) packed four per word, first code lowest.  The fast
-// path has no per-element branch: it notes whether any product lies within 2^-19 of a
-// half-integer, and only then (rarely) recomputes the sixteen codes with the IEEE divide.
+// path multiplies by the reciprocal and notes which products lie within 2^-19 of a
+// half-integer; only those (rarely any) are recomputed with the IEEE divide.
 __device__ __forceinline__ uint32_t pack4_codes(int q0, int q1, int q2, int q3);
 __device__ __forceinline__ void quant16(const float (&y)[16], const RowDivisor& d,
                                         uint32_t (&out)[4]) {
     int q[16];
-    bool exact = !d.fast;
     if (d.fast) {
-        bool near_tie = false;
+        uint32_t ties = 0;
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
             const float2 t = mul2_rn(y[i], y[i + 1], d.r);
             const float f0 = rintf(t.x), f1 = rintf(t.y);
-            near_tie |= fabsf(t.x - f0) >= 0.5f - 0x1p-19f;
-            near_tie |= fabsf(t.y - f1) >= 0.5f - 0x1p-19f;
+            ties |= (fabsf(t.x - f0) >= 0.5f - 0x1p-19f ? 1u : 0u) << i;
+            ties |= (fabsf(t.y - f1) >= 0.5f - 0x1p-19f ? 1u : 0u) << (i + 1);
             q[i] = __float2int_rn(f0);          // NaN -> 0; +-inf saturates
             q[i + 1] = __float2int_rn(f1);
         }
-        exact = near_tie;
-    }
-    if (exact) {
+        if (ties) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (ties & (1u << i)) q[i] = __float2int_rn(__fdiv_rn(y[i], d.s));
+        }
+    } else {
 #pragma unroll
         for (int i = 0; i < 16; ++i) q[i] = __float2int_rn(__fdiv_rn(y[i], d.s));
     }
@@ -354,6 +356,72 @@ __device__ __forceinline__ uint32_t pack4_codes(int q0, int q1, int q2, int q3) 
     const uint32_t lo = __byte_perm((uint32_t)q0, (uint32_t)q1, 0x0040);
     const uint32_t hi = __byte_perm((uint32_t)q2, (uint32_t)q3, 0x0040);
     return __byte_perm(lo, hi, 0x5410);
+}
+
+// Packed fp32 pairs as 64-bit registers for the sm_100 f32x2 instructions.
+__device__ __forceinline__ unsigned long long f2_pack(float a0, float a1) {
+    unsigned long long x;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a0), "f"(a1));
+    return x;
+}
+__device__ __forceinline__ float2 f2_unpack(unsigned long long x) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(x));
+    return r;
+}
+__device__ __forceinline__ unsigned long long add2_rn(unsigned long long a, unsigned long long b) {
+    unsigned long long z;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(a), "l"(b));
+    return z;
+}
+__device__ __forceinline__ unsigned long long sub2_rn(unsigned long long a, unsigned long long b) {
+    unsigned long long z;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(a), "l"(b));
+    return z;
+}
+__device__ __forceinline__ unsigned long long mul2s_rn(unsigned long long a, float b) {
+    unsigned long long y = f2_pack(b, b), z;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(a), "l"(y));
+    return z;
+}
+
+// quant16 for a row whose scale came from its own absmax (s = max(amax / 7, FLT_MIN)).
+// There every fast-path product satisfies |t| <= 7 (1 + 3 * 2^-24) < 7.5, so no code needs
+// the clamp, and adding 1.5 * 2^23 rounds t to an integer (half to even) that sits in the
+// low byte of the sum's bit pattern as a two's-complement code.  Elements whose product lies
+// within 2^-19 of a half-integer (the tie test of quant16) are redone one by one with the
+// IEEE division, so a rare tie costs one division rather than sixteen.
+__device__ __forceinline__ void quant16_dyn(const float (&y)[16], const RowDivisor& d,
+                                            uint32_t (&out)[4]) {
+    if (!d.fast) {
+        quant16(y, d, out);
+        return;
+    }
+    const unsigned long long magic = f2_pack(0x1.8p23f, 0x1.8p23f);
+    uint32_t u[16];
+    uint32_t ties = 0;
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        const unsigned long long t = mul2s_rn(f2_pack(y[i], y[i + 1]), d.r);
+        const unsigned long long r = add2_rn(t, magic);                 // 1.5 * 2^23 + rint(t)
+        const float2 dev = f2_unpack(sub2_rn(t, sub2_rn(r, magic)));    // t - rint(t), exact
+        ties |= (fabsf(dev.x) >= 0.5f - 0x1p-19f ? 1u : 0u) << i;
+        ties |= (fabsf(dev.y) >= 0.5f - 0x1p-19f ? 1u : 0u) << (i + 1);
+        const float2 rr = f2_unpack(r);
+        u[i] = __float_as_uint(rr.x);
+        u[i + 1] = __float_as_uint(rr.y);
+    }
+    if (ties) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (ties & (1u << i)) u[i] = (uint32_t)quant_code(y[i], d.s);
+    }
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const uint32_t lo = __byte_perm(u[4 * w], u[4 * w + 1], 0x0040);
+        const uint32_t hi = __byte_perm(u[4 * w + 2], u[4 * w + 3], 0x0040);
+        out[w] = __byte_perm(lo, hi, 0x5410);
+    }
 }
 
 }  // namespace ck

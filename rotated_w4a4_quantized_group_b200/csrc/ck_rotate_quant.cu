@@ -16,6 +16,8 @@
 //                      from shared memory with 16-byte coalesced code stores.
 //   rq_generic_kernel  every dtype, g and stride: one row per CTA step, fp32 FFMA with R
 //                      in shared memory (or read through L1 when it does not fit).
+#include <algorithm>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -468,6 +470,243 @@ __global__ void __launch_bounds__(kRqThreads, 1)
     __syncthreads();
 }
 
+// ===================================================================== row kernel
+
+// One persistent CTA per SM whose compute warps own whole rows.  The last warp streams rows
+// into per-warp double buffers with TMA (3-D boxes of group-rows, swizzled like the ring
+// kernel's); each compute warp rotates its row in place (mma.sync m16n8k16, R^T in shared
+// memory, results rounded to T and written back with stmatrix), reduces the row absmax with
+// warp shuffles, writes the row scale, quantizes from shared memory and stores the codes
+// 16 bytes per lane.  No barrier is shared between compute warps: each buffer has its own
+// full / empty mbarrier pair with the producer.
+constexpr int kRowMaxWarps = 12;   // compute warps
+constexpr int kRowBufs = 2;        // row buffers per compute warp
+
+struct RqRowParams {
+    int64_t M, K, ldq;
+    int GR;               // group-rows per row (K / G)
+    int GB;               // group-rows per TMA box (a multiple of 8 when a row takes >1 box)
+    int NB;               // boxes per row
+    int W;                // compute warps
+    uint32_t buf_bytes;   // one row buffer (a multiple of 1024 bytes)
+    uint32_t box_bytes;   // bytes one box delivers
+    int vec_codes;
+};
+
+template <typename T, int G, bool DYN>
+__global__ void __launch_bounds__((kRowMaxWarps + 1) * 32, 1)
+    rq_row_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ R,
+                  const float* __restrict__ scale_in, int8_t* __restrict__ codes,
+                  float* __restrict__ scales, RqRowParams p, int* dev_status) {
+    constexpr int KT = G / 16;   // k-tiles of the m16n8k16 MMA
+    constexpr int NT = G / 8;    // n-tiles
+    extern __shared__ __align__(1024) unsigned char row_smem[];
+    unsigned char* bufs = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(row_smem) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t full_bar[kRowMaxWarps * kRowBufs];
+    __shared__ __align__(8) uint64_t empty_bar[kRowMaxWarps * kRowBufs];
+    __shared__ int abort_flag;
+    __shared__ __align__(128) unsigned char rt_sh[G * G * 2];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int W = p.W;
+    // this CTA's rows: blockIdx.x + gridDim.x * j; row j goes to warp j % W, buffer (j / W) % 2
+    const int64_t my_rows =
+        (int64_t)blockIdx.x < p.M ? (p.M - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+    if (tid == 0) {
+        for (int b = 0; b < W * kRowBufs; ++b) {
+            mbar_init(&full_bar[b], 1);
+            mbar_init(&empty_bar[b], 1);
+        }
+        abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&xmap);
+    }
+    for (int i = tid; i < G * G; i += blockDim.x) {
+        const int n = i / G, k = i % G;
+        *reinterpret_cast<T*>(rt_sh + rt_off<G>(n, k / 8) + (k % 8) * 2) = R[k * G + n];
+    }
+    __syncthreads();
+
+    if (warp == W) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int64_t issued = 0;
+            for (int64_t j = 0; j < my_rows; ++j) {
+                const int64_t i = j / W;
+                const int bi = (int)(j % W) * kRowBufs + (int)(i % kRowBufs);
+                const int64_t f = i / kRowBufs;   // fill number of this buffer
+                if (f >= 1 &&
+                    !mbar_wait(&empty_bar[bi], (uint32_t)(f - 1) & 1u, &abort_flag, dev_status))
+                    break;
+                unsigned char* dst = bufs + (size_t)bi * p.buf_bytes;
+                mbar_arrive_expect_tx(&full_bar[bi], p.box_bytes * (uint32_t)p.NB);
+                const int32_t row = (int32_t)(blockIdx.x + j * gridDim.x);
+                for (int bx = 0; bx < p.NB; ++bx)
+                    tma_load_3d(dst + (size_t)bx * p.GB * G * 2, &xmap, &full_bar[bi], 0,
+                                bx * p.GB, row);
+                ++issued;
+            }
+            // copies still in flight land before the CTA leaves
+            const int64_t first = issued > (int64_t)W * kRowBufs ? issued - (int64_t)W * kRowBufs : 0;
+            if (abort_flag)
+                for (int64_t j = first; j < issued; ++j) {
+                    const int64_t i = j / W;
+                    const int bi = (int)(j % W) * kRowBufs + (int)(i % kRowBufs);
+                    mbar_wait(&full_bar[bi], (uint32_t)(i / kRowBufs) & 1u, nullptr, nullptr);
+                }
+        }
+    } else if (warp < W) {
+        // ---------------------------------------------------------------- compute warps
+        const uint32_t rt_base = smem_u32(rt_sh);
+        const int tiles = (p.GR + 15) / 16;
+        const int units = (int)(p.K / 16);             // 16-element quantize units per row
+        for (int64_t i = 0;; ++i) {
+            const int64_t j = warp + i * W;
+            if (j >= my_rows) break;
+            const int bi = warp * kRowBufs + (int)(i % kRowBufs);
+            if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[bi], (uint32_t)(i / kRowBufs) & 1u,
+                                                   &abort_flag, dev_status)))
+                break;
+            const int64_t row = blockIdx.x + j * gridDim.x;
+            unsigned char* buf = bufs + (size_t)bi * p.buf_bytes;
+            const uint32_t base = smem_u32(buf);
+
+            // ---- rotation, 16 group-rows per MMA tile, y written back in place; row absmax
+            uint32_t m2 = 0u;
+            for (int t = 0; t < tiles; ++t) {
+                const int rho0 = t * 16;
+                uint32_t afr[KT][4];
+                {
+                    const int rho = rho0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                    const int cadd = lane >> 4;
+#pragma unroll
+                    for (int kt = 0; kt < KT; ++kt)
+                        ldmatrix_x4(afr[kt], base + swz_off<G>(rho, kt * 2 + cadd));
+                }
+                float acc[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt) {
+#pragma unroll
+                    for (int nt = 0; nt < NT; nt += 2) {
+                        uint32_t b4[4];
+                        const int n = nt * 8 + ((lane >> 4) << 3) + (lane & 7);
+                        ldmatrix_x4(b4, rt_base + rt_off<G>(n, kt * 2 + ((lane >> 3) & 1)));
+                        MmaOp<T>::run(acc[nt], afr[kt], b4[0], b4[1]);
+                        MmaOp<T>::run(acc[nt + 1], afr[kt], b4[2], b4[3]);
+                    }
+                }
+                const bool okA = rho0 + (lane >> 2) < p.GR, okB = rho0 + 8 + (lane >> 2) < p.GR;
+                const int srow = rho0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int sn = (lane >> 4) & 1;
+#pragma unroll
+                for (int nt = 0; nt < NT; nt += 2) {
+                    const uint32_t pA0 = MmaOp<T>::pack(acc[nt][0], acc[nt][1]);
+                    const uint32_t pB0 = MmaOp<T>::pack(acc[nt][2], acc[nt][3]);
+                    const uint32_t pA1 = MmaOp<T>::pack(acc[nt + 1][0], acc[nt + 1][1]);
+                    const uint32_t pB1 = MmaOp<T>::pack(acc[nt + 1][2], acc[nt + 1][3]);
+                    if (okA) m2 = MmaOp<T>::absmax2(MmaOp<T>::absmax2(m2, pA0), pA1);
+                    if (okB) m2 = MmaOp<T>::absmax2(MmaOp<T>::absmax2(m2, pB0), pB1);
+                    stmatrix_x4(base + swz_off<G>(srow, nt + sn), pA0, pB0, pA1, pB1);
+                }
+            }
+            // ---- row scale (every lane of the warp holds the row's absmax)
+            const float2 mf = MmaOp<T>::unpack(m2);
+            float mx = fmax_nan(mf.x, mf.y);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const float sc = row_scale(mx, DYN ? nullptr : scale_in);
+            if (lane == 0) scales[row] = sc;
+            const RowDivisor dv(sc);
+            __syncwarp();   // the warp's stmatrix results are visible to all its lanes
+
+            // ---- quantize: 16 consecutive channels per lane step, 16-byte code stores
+            int8_t* dst_row = codes + row * p.ldq;
+            for (int u = lane; u < units; u += 32) {
+                const int k = u * 16;
+                const int rho = k / G, e = k - rho * G;
+                const uint4 u0 = *reinterpret_cast<const uint4*>(buf + swz_off<G>(rho, e / 8));
+                const uint4 u1 = *reinterpret_cast<const uint4*>(buf + swz_off<G>(rho, e / 8 + 1));
+                const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+                float y[16];
+#pragma unroll
+                for (int h = 0; h < 8; ++h) {
+                    const float2 a = MmaOp<T>::unpack(w[h]);
+                    y[2 * h] = a.x;
+                    y[2 * h + 1] = a.y;
+                }
+                uint32_t out[4];
+                if (DYN) quant16_dyn(y, dv, out);
+                else quant16(y, dv, out);
+                int8_t* dst = dst_row + k;
+                if (p.vec_codes) {
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) dst[q] = (int8_t)((out[q / 4] >> (8 * (q % 4))) & 0xFF);
+                }
+            }
+            // the buffer is no longer read by this warp
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_bar[bi]);
+        }
+    }
+    __syncthreads();
+}
+
+// Row kernel for bf16/fp16, g in {16, 64}: every row fits one buffer and at least four compute
+// warps with two buffers each fit in shared memory.  Returns CK_ERR_UNSUPPORTED otherwise.
+template <typename T, int G>
+static ck_status launch_row(const void* x, int64_t M, int64_t K, int64_t sm, const void* R,
+                            const float* scale_in, int8_t* codes, int64_t ldq, float* scales,
+                            int* dev_status, cudaStream_t stream, CUtensorMapDataType tdt) {
+    RqRowParams p;
+    p.M = M;
+    p.K = K;
+    p.ldq = ldq;
+    p.GR = (int)(K / G);
+    if (p.GR <= 256) {
+        p.GB = p.GR;
+        p.NB = 1;
+    } else {
+        p.GB = 256;
+        p.NB = (p.GR + 255) / 256;
+    }
+    const int64_t rows_alloc = std::max<int64_t>(((int64_t)p.GR + 15) / 16 * 16, (int64_t)p.GB * p.NB);
+    const int64_t buf = (rows_alloc * G * 2 + 1023) / 1024 * 1024;
+    const int64_t budget = 200 * 1024;
+    const int64_t warps = budget / (buf * kRowBufs);
+    if (warps < 4) return CK_ERR_UNSUPPORTED;
+    p.W = (int)std::min<int64_t>(warps, kRowMaxWarps);
+    p.buf_bytes = (uint32_t)buf;
+    p.box_bytes = (uint32_t)(G * 2 * p.GB);
+    p.vec_codes = (aligned(codes, 16) && ldq % 16 == 0) ? 1 : 0;
+
+    CUtensorMap map;
+    const uint64_t dims[3] = {(uint64_t)G, (uint64_t)p.GR, (uint64_t)M};
+    const uint64_t strides[2] = {(uint64_t)G * 2, (uint64_t)sm * 2};
+    const uint32_t box[3] = {(uint32_t)G, (uint32_t)p.GB, 1u};
+    ck_status st = encode_tma(&map, tdt, 3, x, dims, strides, box,
+                              G == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B);
+    if (st != CK_OK) return st;
+
+    const size_t smem = (size_t)p.W * kRowBufs * p.buf_bytes + 1024;
+    const int grid = (int)(M < num_sms() ? M : num_sms());
+    const int threads = (p.W + 1) * 32;
+    auto run = [&](auto kern) -> ck_status {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return CK_ERR_CUDA;
+        kern<<<grid, threads, smem, stream>>>(map, static_cast<const T*>(R), scale_in, codes,
+                                              scales, p, dev_status);
+        return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+    };
+    return scale_in ? run(rq_row_kernel<T, G, false>) : run(rq_row_kernel<T, G, true>);
+}
+
 // ===================================================================== host launch
 
 template <typename T, int G>
@@ -561,6 +800,20 @@ ck_status launch_rotate_quant(const void* x, ck_dtype dt, int64_t M, int64_t K, 
                         aligned(x, 16) && sm % 8 == 0 && sm > 0 && M < (1LL << 31) &&
                         K / g <= (1LL << 31);
     if (mma_ok) {
+        ck_status st = CK_ERR_UNSUPPORTED;
+        if (dt == CK_BF16)
+            st = g == 64 ? launch_row<__nv_bfloat16, 64>(x, M, K, sm, R, scale_in, codes, ldq, scales,
+                                                          dev_status, stream,
+                                                          CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
+                         : launch_row<__nv_bfloat16, 16>(x, M, K, sm, R, scale_in, codes, ldq, scales,
+                                                          dev_status, stream,
+                                                          CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+        else
+            st = g == 64 ? launch_row<__half, 64>(x, M, K, sm, R, scale_in, codes, ldq, scales,
+                                                   dev_status, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)
+                         : launch_row<__half, 16>(x, M, K, sm, R, scale_in, codes, ldq, scales,
+                                                   dev_status, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+        if (st != CK_ERR_UNSUPPORTED) return st;
         if (dt == CK_BF16)
             return g == 64 ? launch_mma<__nv_bfloat16, 64>(x, M, K, sm, R, scale_in, codes, ldq,
                                                            scales, dev_status, stream,
