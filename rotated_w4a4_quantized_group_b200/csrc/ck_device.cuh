@@ -282,64 +282,61 @@ __device__ __forceinline__ int quant_code(float y, float s) {
     return (int)t;
 }
 
-// The divisor of one row: s and r = fl(1 / s).  `fast` is false when r is not a normal
-// number (or s is NaN), in which case every code of the row takes the IEEE division.
+// The divisor of one row: s and r = fl(1 / s), the correctly rounded reciprocal.
+//
+// Division by s uses Markstein's correction step (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990):
+//   t = fl(y r);  e = fl(y - t s) (one FMA, exact);  q = fl(t + e r) (one FMA).
+// With r correctly rounded and t within a few ulps of y / s, q is the correctly rounded
+// quotient fl(y / s) as long as the remainder e is not subnormal.  The quotients needed
+// here are below 2^23 and y is at least 2^-24 |q| s, so s >= 2^-64 keeps e far above the
+// subnormal range.  `fast` is false when s is below that bound, not finite, or NaN, or when
+// r is not a normal number; every code of such a row takes the IEEE division.
 struct RowDivisor {
     float s, r;
     bool fast;
     __device__ __forceinline__ explicit RowDivisor(float s_) : s(s_) {
         r = __frcp_rn(s_);
-        fast = (r >= 1.17549435e-38f) && (r <= 3.40282347e38f);
+        fast = (s_ >= 0x1p-64f) && (r >= 1.17549435e-38f) && (r <= 3.40282347e38f);
     }
 };
 
-// The same code as quant_code(y, d.s), with a multiply instead of the division.  The
-// product t = fl(y * fl(1/s)) is within 9 * 1.5 * 2^-23 < 2^-19 of the IEEE quotient
-// fl(y / s) wherever |t| < 9, so both round to the same integer unless t lies within 2^-19
-// of a half-integer; those rare values (and rows without a normal reciprocal) are divided
-// exactly.  Beyond |t| = 9 both clamp alike.  NaN converts to 0 and +-inf saturates, as in
-// quant_code.
+// fl(y / s) for a fast RowDivisor (Markstein's correction, see RowDivisor).
+__device__ __forceinline__ float quotient_fast(float y, float s, float r) {
+    const float t = __fmul_rn(y, r);
+    const float e = __fmaf_rn(-t, s, y);
+    return __fmaf_rn(e, r, t);
+}
+
+// The same code as quant_code(y, d.s): the IEEE quotient from a reciprocal multiply and
+// Markstein's correction (RowDivisor), rounded half to even by the conversion.  NaN
+// converts to 0 and +-inf saturates, as in quant_code.
 __device__ __forceinline__ int quant_code_fast(float y, const RowDivisor& d) {
     if (!d.fast) return quant_code(y, d.s);
-    const float t = __fmul_rn(y, d.r);
-    float f = rintf(t);
-    if (fabsf(t - f) >= 0.5f - 0x1p-19f) f = rintf(__fdiv_rn(y, d.s));
-    return min(max(__float2int_rn(f), -8), 7);
+    return min(max(__float2int_rn(quotient_fast(y, d.s, d.r)), -8), 7);
 }
 
-// Two fp32 products at once (sm_100 packed fp32 multiply), each rounded to nearest even.
-__device__ __forceinline__ float2 mul2_rn(float a0, float a1, float b) {
-    unsigned long long x, y, z;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a0), "f"(a1));
-    asm("mov.b64 %0, {%1, %1};" : "=l"(y) : "f"(b));
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
-    float2 r;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(z));
-    return r;
-}
-
-// Sixteen codes of one row (divisor d) packed four per word, first code lowest.  The fast
-// path multiplies by the reciprocal and notes which products lie within 2^-19 of a
-// half-integer; only those (rarely any) are recomputed with the IEEE divide.
+// Sixteen codes of one row (divisor d) packed four per word, first code lowest: the
+// quotients of quant_code_fast computed two at a time with packed fp32 arithmetic.
 __device__ __forceinline__ uint32_t pack4_codes(int q0, int q1, int q2, int q3);
+__device__ __forceinline__ unsigned long long f2_pack(float a0, float a1);
+__device__ __forceinline__ float2 f2_unpack(unsigned long long x);
+__device__ __forceinline__ unsigned long long mul2s_rn(unsigned long long a, float b);
+__device__ __forceinline__ unsigned long long fma2_rn(unsigned long long a, unsigned long long b,
+                                                      unsigned long long c);
 __device__ __forceinline__ void quant16(const float (&y)[16], const RowDivisor& d,
                                         uint32_t (&out)[4]) {
     int q[16];
     if (d.fast) {
-        uint32_t ties = 0;
+        const unsigned long long ns = f2_pack(-d.s, -d.s), r2 = f2_pack(d.r, d.r);
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
-            const float2 t = mul2_rn(y[i], y[i + 1], d.r);
-            const float f0 = rintf(t.x), f1 = rintf(t.y);
-            ties |= (fabsf(t.x - f0) >= 0.5f - 0x1p-19f ? 1u : 0u) << i;
-            ties |= (fabsf(t.y - f1) >= 0.5f - 0x1p-19f ? 1u : 0u) << (i + 1);
-            q[i] = __float2int_rn(f0);          // NaN -> 0; +-inf saturates
-            q[i + 1] = __float2int_rn(f1);
-        }
-        if (ties) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (ties & (1u << i)) q[i] = __float2int_rn(__fdiv_rn(y[i], d.s));
+            const unsigned long long y2 = f2_pack(y[i], y[i + 1]);
+            const unsigned long long t = mul2s_rn(y2, d.r);
+            const unsigned long long e = fma2_rn(t, ns, y2);
+            const float2 qq = f2_unpack(fma2_rn(e, r2, t));
+            q[i] = __float2int_rn(qq.x);          // NaN -> 0; +-inf saturates
+            q[i + 1] = __float2int_rn(qq.y);
         }
     } else {
 #pragma unroll
@@ -385,36 +382,40 @@ __device__ __forceinline__ unsigned long long mul2s_rn(unsigned long long a, flo
     return z;
 }
 
-// quant16 for a row whose scale came from its own absmax (s = max(amax / 7, FLT_MIN)).
-// There every fast-path product satisfies |t| <= 7 (1 + 3 * 2^-24) < 7.5, so no code needs
-// the clamp, and adding 1.5 * 2^23 rounds t to an integer (half to even) that sits in the
-// low byte of the sum's bit pattern as a two's-complement code.  Elements whose product lies
-// within 2^-19 of a half-integer (the tie test of quant16) are redone one by one with the
-// IEEE division, so a rare tie costs one division rather than sixteen.
-__device__ __forceinline__ void quant16_dyn(const float (&y)[16], const RowDivisor& d,
-                                            uint32_t (&out)[4]) {
-    if (!d.fast) {
-        quant16(y, d, out);
-        return;
-    }
-    const unsigned long long magic = f2_pack(0x1.8p23f, 0x1.8p23f);
+__device__ __forceinline__ unsigned long long fma2_rn(unsigned long long a, unsigned long long b,
+                                                      unsigned long long c) {
+    unsigned long long z;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(z) : "l"(a), "l"(b), "l"(c));
+    return z;
+}
+
+// quant16 for a row whose scale came from its own absmax (s = max(amax / 7, FLT_MIN)), with
+// the input as eight fp32 pairs.  There every quotient satisfies |y / s| <= 7, so no code
+// needs the clamp, and adding 1.5 * 2^23 to the quotient rounds it to an integer (half to
+// even) that sits in the low byte of the sum's bit pattern as a two's-complement code.
+// A row that is not `fast` (NaN, inf, tiny or huge scale) takes quant_code per element.
+__device__ __forceinline__ void quant16_dyn2(const unsigned long long (&y2)[8], const RowDivisor& d,
+                                             uint32_t (&out)[4]) {
     uint32_t u[16];
-    uint32_t ties = 0;
+    if (d.fast) {
+        const unsigned long long magic = f2_pack(0x1.8p23f, 0x1.8p23f);
+        const unsigned long long ns = f2_pack(-d.s, -d.s), r2 = f2_pack(d.r, d.r);
 #pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-        const unsigned long long t = mul2s_rn(f2_pack(y[i], y[i + 1]), d.r);
-        const unsigned long long r = add2_rn(t, magic);                 // 1.5 * 2^23 + rint(t)
-        const float2 dev = f2_unpack(sub2_rn(t, sub2_rn(r, magic)));    // t - rint(t), exact
-        ties |= (fabsf(dev.x) >= 0.5f - 0x1p-19f ? 1u : 0u) << i;
-        ties |= (fabsf(dev.y) >= 0.5f - 0x1p-19f ? 1u : 0u) << (i + 1);
-        const float2 rr = f2_unpack(r);
-        u[i] = __float_as_uint(rr.x);
-        u[i + 1] = __float_as_uint(rr.y);
-    }
-    if (ties) {
+        for (int i = 0; i < 8; ++i) {
+            const unsigned long long t = mul2s_rn(y2[i], d.r);
+            const unsigned long long e = fma2_rn(t, ns, y2[i]);
+            const unsigned long long q = fma2_rn(e, r2, t);               // fl(y / s)
+            const float2 rr = f2_unpack(add2_rn(q, magic));               // 1.5 * 2^23 + rint
+            u[2 * i] = __float_as_uint(rr.x);
+            u[2 * i + 1] = __float_as_uint(rr.y);
+        }
+    } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-            if (ties & (1u << i)) u[i] = (uint32_t)quant_code(y[i], d.s);
+        for (int i = 0; i < 8; ++i) {
+            const float2 y = f2_unpack(y2[i]);
+            u[2 * i] = (uint32_t)quant_code(y.x, d.s);
+            u[2 * i + 1] = (uint32_t)quant_code(y.y, d.s);
+        }
     }
 #pragma unroll
     for (int w = 0; w < 4; ++w) {

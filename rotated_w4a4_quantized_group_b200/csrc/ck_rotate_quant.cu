@@ -179,6 +179,10 @@ template <> struct MmaOp<__nv_bfloat16> {
     __device__ static __forceinline__ float2 unpack(uint32_t u) {
         return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
     }
+    // the pair as an f32x2 register: a bf16 is the high half of its fp32
+    __device__ static __forceinline__ unsigned long long unpack2(uint32_t u) {
+        return f2_pack(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+    }
     // running max of |.| over packed pairs, NaN-propagating
     __device__ static __forceinline__ uint32_t absmax2(uint32_t m, uint32_t v) {
         uint32_t a = v & 0x7FFF7FFFu;
@@ -203,6 +207,10 @@ template <> struct MmaOp<__half> {
     __device__ static __forceinline__ float2 unpack(uint32_t u) {
         return __half22float2(*reinterpret_cast<__half2*>(&u));
     }
+    __device__ static __forceinline__ unsigned long long unpack2(uint32_t u) {
+        const float2 f = unpack(u);
+        return f2_pack(f.x, f.y);
+    }
     __device__ static __forceinline__ uint32_t absmax2(uint32_t m, uint32_t v) {
         uint32_t a = v & 0x7FFF7FFFu;
         __half2 r = __hmax2_nan(*reinterpret_cast<__half2*>(&m), *reinterpret_cast<__half2*>(&a));
@@ -216,6 +224,18 @@ __device__ __forceinline__ void stmatrix_x4(uint32_t saddr, uint32_t r0, uint32_
                  "r"(r0), "r"(r1), "r"(r2), "r"(r3)
                  : "memory");
 }
+
+// Four 8x8 b16 matrices stored transposed: lane i of matrix j gives the address of shared-
+// memory row i, which receives column i of the fragment matrix.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t r0, uint32_t r1,
+                                                  uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(saddr),
+                 "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+}
+
+// group-rows of x per step of the row kernel's rotation
+template <int G> constexpr int kRowStep = G == 64 ? 8 : 16;
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t saddr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -498,8 +518,8 @@ __global__ void __launch_bounds__((kRowMaxWarps + 1) * 32, 1)
     rq_row_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ R,
                   const float* __restrict__ scale_in, int8_t* __restrict__ codes,
                   float* __restrict__ scales, RqRowParams p, int* dev_status) {
-    constexpr int KT = G / 16;   // k-tiles of the m16n8k16 MMA
-    constexpr int NT = G / 8;    // n-tiles
+    constexpr int KT = G / 16;   // k-tiles of the m16n8k16 MMA (input channels)
+    constexpr int MT = G / 16;   // m-tiles (output channels)
     extern __shared__ __align__(1024) unsigned char row_smem[];
     unsigned char* bufs = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(row_smem) + 1023) & ~uintptr_t(1023));
@@ -560,7 +580,6 @@ __global__ void __launch_bounds__((kRowMaxWarps + 1) * 32, 1)
     } else if (warp < W) {
         // ---------------------------------------------------------------- compute warps
         const uint32_t rt_base = smem_u32(rt_sh);
-        const int tiles = (p.GR + 15) / 16;
         const int units = (int)(p.K / 16);             // 16-element quantize units per row
         for (int64_t i = 0;; ++i) {
             const int64_t j = warp + i * W;
@@ -573,44 +592,79 @@ __global__ void __launch_bounds__((kRowMaxWarps + 1) * 32, 1)
             unsigned char* buf = bufs + (size_t)bi * p.buf_bytes;
             const uint32_t base = smem_u32(buf);
 
-            // ---- rotation, 16 group-rows per MMA tile, y written back in place; row absmax
+            // ---- rotation y^T = R^T x^T: R^T is the A operand (fragments in registers), eight
+            // (G = 64) or sixteen (G = 16) group-rows of x the B operand; the fp32 results are
+            // rounded to T and stored transposed (stmatrix.trans) over x in place
+            // A fragments of R^T (rows c = output channel, columns i = input channel), reloaded
+            // per row so that they are not live across the quantize pass
+            uint32_t ra[MT][KT][4];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt)
+                    ldmatrix_x4(ra[mt][kt], rt_base + rt_off<G>(16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8,
+                                                                2 * kt + (lane >> 4)));
             uint32_t m2 = 0u;
-            for (int t = 0; t < tiles; ++t) {
-                const int rho0 = t * 16;
-                uint32_t afr[KT][4];
-                {
-                    const int rho = rho0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-                    const int cadd = lane >> 4;
+            for (int rho0 = 0; rho0 < p.GR; rho0 += kRowStep<G>) {
+                if constexpr (G == 64) {
+                    uint32_t bq[KT][2];
+#pragma unroll
+                    for (int kp = 0; kp < KT; kp += 2) {
+                        uint32_t r4[4];
+                        ldmatrix_x4(r4, base + swz_off<G>(rho0 + (lane & 7), 2 * kp + (lane >> 3)));
+                        bq[kp][0] = r4[0];
+                        bq[kp][1] = r4[1];
+                        bq[kp + 1][0] = r4[2];
+                        bq[kp + 1][1] = r4[3];
+                    }
+                    float acc[MT][4];
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
 #pragma unroll
                     for (int kt = 0; kt < KT; ++kt)
-                        ldmatrix_x4(afr[kt], base + swz_off<G>(rho, kt * 2 + cadd));
-                }
-                float acc[NT][4];
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+                        for (int mt = 0; mt < MT; ++mt) MmaOp<T>::run(acc[mt], ra[mt][kt], bq[kt][0], bq[kt][1]);
+                    // this lane's group-rows rho0 + 2 (lane % 4) + {0, 1}: absmax mask per half
+                    const int rr = rho0 + 2 * (lane & 3);
+                    const uint32_t keep = (rr < p.GR ? 0x0000FFFFu : 0u) | (rr + 1 < p.GR ? 0xFFFF0000u : 0u);
 #pragma unroll
-                for (int kt = 0; kt < KT; ++kt) {
-#pragma unroll
-                    for (int nt = 0; nt < NT; nt += 2) {
-                        uint32_t b4[4];
-                        const int n = nt * 8 + ((lane >> 4) << 3) + (lane & 7);
-                        ldmatrix_x4(b4, rt_base + rt_off<G>(n, kt * 2 + ((lane >> 3) & 1)));
-                        MmaOp<T>::run(acc[nt], afr[kt], b4[0], b4[1]);
-                        MmaOp<T>::run(acc[nt + 1], afr[kt], b4[2], b4[3]);
+                    for (int mt = 0; mt < MT; mt += 2) {
+                        const uint32_t q0 = MmaOp<T>::pack(acc[mt][0], acc[mt][1]);
+                        const uint32_t q1 = MmaOp<T>::pack(acc[mt][2], acc[mt][3]);
+                        const uint32_t q2 = MmaOp<T>::pack(acc[mt + 1][0], acc[mt + 1][1]);
+                        const uint32_t q3 = MmaOp<T>::pack(acc[mt + 1][2], acc[mt + 1][3]);
+                        m2 = MmaOp<T>::absmax2(m2, q0 & keep);
+                        m2 = MmaOp<T>::absmax2(m2, q1 & keep);
+                        m2 = MmaOp<T>::absmax2(m2, q2 & keep);
+                        m2 = MmaOp<T>::absmax2(m2, q3 & keep);
+                        stmatrix_x4_trans(base + swz_off<G>(rho0 + (lane & 7), 2 * mt + (lane >> 3)),
+                                          q0, q1, q2, q3);
                     }
-                }
-                const bool okA = rho0 + (lane >> 2) < p.GR, okB = rho0 + 8 + (lane >> 2) < p.GR;
-                const int srow = rho0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-                const int sn = (lane >> 4) & 1;
+                } else {
+                    // G = 16: one ldmatrix.x4 gives the B fragments of two n-tiles (rows
+                    // rho0..+7 and rho0+8..+15); the same lane addresses serve the store
+                    const uint32_t addr =
+                        base + swz_off<G>(rho0 + ((lane >> 4) << 3) + (lane & 7), (lane >> 3) & 1);
+                    uint32_t r4[4];
+                    ldmatrix_x4(r4, addr);
+                    float acc[2][4];
 #pragma unroll
-                for (int nt = 0; nt < NT; nt += 2) {
-                    const uint32_t pA0 = MmaOp<T>::pack(acc[nt][0], acc[nt][1]);
-                    const uint32_t pB0 = MmaOp<T>::pack(acc[nt][2], acc[nt][3]);
-                    const uint32_t pA1 = MmaOp<T>::pack(acc[nt + 1][0], acc[nt + 1][1]);
-                    const uint32_t pB1 = MmaOp<T>::pack(acc[nt + 1][2], acc[nt + 1][3]);
-                    if (okA) m2 = MmaOp<T>::absmax2(MmaOp<T>::absmax2(m2, pA0), pA1);
-                    if (okB) m2 = MmaOp<T>::absmax2(MmaOp<T>::absmax2(m2, pB0), pB1);
-                    stmatrix_x4(base + swz_off<G>(srow, nt + sn), pA0, pB0, pA1, pB1);
+                    for (int nt = 0; nt < 2; ++nt) {
+                        acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+                        MmaOp<T>::run(acc[nt], ra[0][0], r4[2 * nt], r4[2 * nt + 1]);
+                    }
+                    uint32_t q[2][2];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const int rr = rho0 + 8 * nt + 2 * (lane & 3);
+                        const uint32_t keep =
+                            (rr < p.GR ? 0x0000FFFFu : 0u) | (rr + 1 < p.GR ? 0xFFFF0000u : 0u);
+                        q[nt][0] = MmaOp<T>::pack(acc[nt][0], acc[nt][1]);
+                        q[nt][1] = MmaOp<T>::pack(acc[nt][2], acc[nt][3]);
+                        m2 = MmaOp<T>::absmax2(m2, q[nt][0] & keep);
+                        m2 = MmaOp<T>::absmax2(m2, q[nt][1] & keep);
+                    }
+                    stmatrix_x4_trans(addr, q[0][0], q[0][1], q[1][0], q[1][1]);
                 }
             }
             // ---- row scale (every lane of the warp holds the row's absmax)
@@ -631,16 +685,22 @@ __global__ void __launch_bounds__((kRowMaxWarps + 1) * 32, 1)
                 const uint4 u0 = *reinterpret_cast<const uint4*>(buf + swz_off<G>(rho, e / 8));
                 const uint4 u1 = *reinterpret_cast<const uint4*>(buf + swz_off<G>(rho, e / 8 + 1));
                 const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-                float y[16];
-#pragma unroll
-                for (int h = 0; h < 8; ++h) {
-                    const float2 a = MmaOp<T>::unpack(w[h]);
-                    y[2 * h] = a.x;
-                    y[2 * h + 1] = a.y;
-                }
                 uint32_t out[4];
-                if (DYN) quant16_dyn(y, dv, out);
-                else quant16(y, dv, out);
+                if (DYN) {
+                    unsigned long long y2[8];
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) y2[h] = MmaOp<T>::unpack2(w[h]);
+                    quant16_dyn2(y2, dv, out);
+                } else {
+                    float y[16];
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) {
+                        const float2 a = MmaOp<T>::unpack(w[h]);
+                        y[2 * h] = a.x;
+                        y[2 * h + 1] = a.y;
+                    }
+                    quant16(y, dv, out);
+                }
                 int8_t* dst = dst_row + k;
                 if (p.vec_codes) {
                     *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);

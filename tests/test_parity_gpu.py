@@ -372,3 +372,26 @@ def test_quantizer_exact_ties_with_inexact_reciprocal(dt, g):
     np.testing.assert_array_equal(codes.cpu().numpy(), np.array(want * (g // 16) * 2)[None].repeat(40, 0))
     oc, os_ = oracle.rotate_quant(x, R, g)
     np.testing.assert_array_equal(codes.cpu().numpy(), oc)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("g", [16, 64, 256])
+def test_quantizer_codes_bit_exact_with_identity_rotation(dt, g):
+    """With R = I the rotation is exact in every path, so the codes depend on the quantizer
+    alone and must equal the oracle's IEEE-division codes bit for bit, ties included: half of
+    the rows are random normals with outliers, half hold multiples of 1.5 next to an absmax
+    of 21 (s = 3, an inexact reciprocal, so many quotients are exact half-integers)."""
+    rng = np.random.default_rng(1000 + g)
+    M, K = 300, 3840
+    x = rng.standard_normal((M, K))
+    x[:, rng.choice(K, K // 100, replace=False)] *= 20.0
+    x[M // 2:] = 1.5 * rng.integers(-14, 15, size=(M - M // 2, K))
+    x[M // 2:, 0] = 21.0
+    xt = torch.from_numpy(x).to(DT[dt])
+    R = torch.eye(g, dtype=torch.float64).to(DT[dt])
+    codes, scales = ck.ck_rotate_quant(xt.cuda(), R.cuda(), g)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.rotate_quant(xt, R, g)
+    np.testing.assert_array_equal(scales.cpu().numpy(), os_)
+    np.testing.assert_array_equal(codes.cpu().numpy(), oc)
