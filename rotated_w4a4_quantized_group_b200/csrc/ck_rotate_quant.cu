@@ -492,14 +492,14 @@ __global__ void __launch_bounds__(kRqThreads, 1)
 
 // ===================================================================== row kernel
 
-// One persistent CTA per SM whose compute warps own whole rows.  The last warp streams rows
-// into per-warp double buffers with TMA (3-D boxes of group-rows, swizzled like the ring
-// kernel's); each compute warp rotates its row in place (mma.sync m16n8k16, R^T in shared
-// memory, results rounded to T and written back with stmatrix), reduces the row absmax with
-// warp shuffles, writes the row scale, quantizes from shared memory and stores the codes
-// 16 bytes per lane.  No barrier is shared between compute warps: each buffer has its own
-// full / empty mbarrier pair with the producer.
-constexpr int kRowMaxWarps = 12;   // compute warps
+// One persistent CTA per SM whose warps own whole rows.  Each warp keeps two row buffers
+// filled by its own TMA copies (3-D boxes of group-rows, swizzled like the ring kernel's):
+// as soon as it has quantized a row it refills that buffer with its row after next.  It
+// rotates each row in place (mma.sync m16n8k16 with R^T in shared memory, results rounded to
+// T and written back with stmatrix), reduces the row absmax with warp shuffles, writes the row
+// scale, quantizes from shared memory and stores the codes 16 bytes per lane.  No barrier is
+// shared between warps.
+constexpr int kRowMaxWarps = 12;   // warps
 constexpr int kRowBufs = 2;        // row buffers per compute warp
 
 struct RqRowParams {
@@ -514,7 +514,7 @@ struct RqRowParams {
 };
 
 template <typename T, int G, bool DYN>
-__global__ void __launch_bounds__((kRowMaxWarps + 1) * 32, 1)
+__global__ void __launch_bounds__(kRowMaxWarps * 32, 1)
     rq_row_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ R,
                   const float* __restrict__ scale_in, int8_t* __restrict__ codes,
                   float* __restrict__ scales, RqRowParams p, int* dev_status) {
@@ -524,7 +524,6 @@ __global__ void __launch_bounds__((kRowMaxWarps + 1) * 32, 1)
     unsigned char* bufs = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(row_smem) + 1023) & ~uintptr_t(1023));
     __shared__ __align__(8) uint64_t full_bar[kRowMaxWarps * kRowBufs];
-    __shared__ __align__(8) uint64_t empty_bar[kRowMaxWarps * kRowBufs];
     __shared__ int abort_flag;
     __shared__ __align__(128) unsigned char rt_sh[G * G * 2];
 
@@ -535,10 +534,7 @@ __global__ void __launch_bounds__((kRowMaxWarps + 1) * 32, 1)
         (int64_t)blockIdx.x < p.M ? (p.M - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
     if (tid == 0) {
-        for (int b = 0; b < W * kRowBufs; ++b) {
-            mbar_init(&full_bar[b], 1);
-            mbar_init(&empty_bar[b], 1);
-        }
+        for (int b = 0; b < W * kRowBufs; ++b) mbar_init(&full_bar[b], 1);
         abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&xmap);
@@ -549,39 +545,27 @@ __global__ void __launch_bounds__((kRowMaxWarps + 1) * 32, 1)
     }
     __syncthreads();
 
-    if (warp == W) {
-        // ---------------------------------------------------------------- TMA producer
+    if (warp < W) {
+        // ---------------------------------------------------------------- row warps
+        // row i of this warp is this CTA's row warp + i W, in buffer i % 2
+        auto issue = [&](int64_t i) {   // lane 0: start the copy of the warp's row i
+            const int64_t j = warp + i * W;
+            if (j >= my_rows) return;
+            const int bi = warp * kRowBufs + (int)(i % kRowBufs);
+            unsigned char* dst = bufs + (size_t)bi * p.buf_bytes;
+            mbar_arrive_expect_tx(&full_bar[bi], p.box_bytes * (uint32_t)p.NB);
+            const int32_t row = (int32_t)(blockIdx.x + j * gridDim.x);
+            for (int bx = 0; bx < p.NB; ++bx)
+                tma_load_3d(dst + (size_t)bx * p.GB * G * 2, &xmap, &full_bar[bi], 0, bx * p.GB, row);
+        };
         if (lane == 0) {
-            int64_t issued = 0;
-            for (int64_t j = 0; j < my_rows; ++j) {
-                const int64_t i = j / W;
-                const int bi = (int)(j % W) * kRowBufs + (int)(i % kRowBufs);
-                const int64_t f = i / kRowBufs;   // fill number of this buffer
-                if (f >= 1 &&
-                    !mbar_wait(&empty_bar[bi], (uint32_t)(f - 1) & 1u, &abort_flag, dev_status))
-                    break;
-                unsigned char* dst = bufs + (size_t)bi * p.buf_bytes;
-                mbar_arrive_expect_tx(&full_bar[bi], p.box_bytes * (uint32_t)p.NB);
-                const int32_t row = (int32_t)(blockIdx.x + j * gridDim.x);
-                for (int bx = 0; bx < p.NB; ++bx)
-                    tma_load_3d(dst + (size_t)bx * p.GB * G * 2, &xmap, &full_bar[bi], 0,
-                                bx * p.GB, row);
-                ++issued;
-            }
-            // copies still in flight land before the CTA leaves
-            const int64_t first = issued > (int64_t)W * kRowBufs ? issued - (int64_t)W * kRowBufs : 0;
-            if (abort_flag)
-                for (int64_t j = first; j < issued; ++j) {
-                    const int64_t i = j / W;
-                    const int bi = (int)(j % W) * kRowBufs + (int)(i % kRowBufs);
-                    mbar_wait(&full_bar[bi], (uint32_t)(i / kRowBufs) & 1u, nullptr, nullptr);
-                }
+            issue(0);
+            issue(1);
         }
-    } else if (warp < W) {
-        // ---------------------------------------------------------------- compute warps
         const uint32_t rt_base = smem_u32(rt_sh);
         const int units = (int)(p.K / 16);             // 16-element quantize units per row
-        for (int64_t i = 0;; ++i) {
+        int64_t i = 0;
+        for (;; ++i) {
             const int64_t j = warp + i * W;
             if (j >= my_rows) break;
             const int bi = warp * kRowBufs + (int)(i % kRowBufs);
@@ -709,10 +693,20 @@ __global__ void __launch_bounds__((kRowMaxWarps + 1) * 32, 1)
                     for (int q = 0; q < 16; ++q) dst[q] = (int8_t)((out[q / 4] >> (8 * (q % 4))) & 0xFF);
                 }
             }
-            // the buffer is no longer read by this warp
+            // the buffer is no longer read by this warp: refill it with row i + 2 (the proxy
+            // fence orders this warp's shared-memory accesses before the async copy's writes)
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty_bar[bi]);
+            if (lane == 0) {
+                fence_proxy_async_smem();
+                issue(i + kRowBufs);
+            }
         }
+        // after an expired wait, copies still in flight land before the CTA leaves
+        if (lane == 0)
+            for (int64_t k = i; k < i + kRowBufs; ++k)
+                if (warp + k * W < my_rows)
+                    mbar_wait(&full_bar[warp * kRowBufs + (int)(k % kRowBufs)],
+                              (uint32_t)(k / kRowBufs) & 1u, nullptr, nullptr);
     }
     __syncthreads();
 }
@@ -755,7 +749,7 @@ static ck_status launch_row(const void* x, int64_t M, int64_t K, int64_t sm, con
 
     const size_t smem = (size_t)p.W * kRowBufs * p.buf_bytes + 1024;
     const int grid = (int)(M < num_sms() ? M : num_sms());
-    const int threads = (p.W + 1) * 32;
+    const int threads = p.W * 32;
     auto run = [&](auto kern) -> ck_status {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
