@@ -196,7 +196,10 @@ def test_rotate_quant_is_deterministic():
 @pytest.mark.parametrize("M,N,K,out_dt", [(1, 1, 2, torch.float32), (200, 300, 448, torch.float32),
                                           (129, 257, 128, torch.bfloat16),
                                           (77, 513, 3840, torch.float16),
-                                          (300, 100, 48, torch.float32)])
+                                          (300, 100, 48, torch.float32),
+                                          # several tiles per CTA with an odd number of
+                                          # 128-deep K blocks per tile
+                                          (4000, 2000, 384, torch.float32)])
 def test_gemm_accumulators_bit_exact(M, N, K, out_dt):
     """Unit scales, no bias, fp32 out: the output is the INT32 accumulator exactly."""
     g = torch.Generator().manual_seed(M + N + K)
