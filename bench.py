@@ -148,22 +148,32 @@ class ClockSampler:
                 "source": "nvml" if self._nvml is not None else "nvidia-smi"}
 
 
-def dist_setup():
+def dist_setup(backend: str = "nccl"):
+    """Process group from torchrun's environment (RANK, WORLD_SIZE, LOCAL_RANK, MASTER_*),
+    with a short timeout so that ranks waiting on a lost peer end with an error.  NCCL binds
+    each rank to its local GPU; gloo (CPU) serves the host-side tests."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
 
 
+def _reduce_device():
+    return "cpu" if torch.distributed.get_backend() == "gloo" else "cuda"
+
+
 def max_over_ranks(v: float, world: int) -> float:
+    """The largest value over all ranks (every rank receives it)."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_reduce_device())
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -171,7 +181,8 @@ def max_over_ranks(v: float, world: int) -> float:
 def barrier(world: int):
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 # ----------------------------------------------------------------------------- oracle (CPU)
@@ -202,7 +213,7 @@ def run_reference(args, case, world, rank):
     inp = W.make_linear_inputs(case)
     vals = []
     rows_used = 0
-    per_step = max(0.5, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    per_step = max(0.05, min(args.cpu_budget, 120.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup + args.steps):
         v, rows, dt = oracle_sample(case, inp, per_step)
         if i >= args.warmup:
