@@ -17,6 +17,7 @@
 //   rq_generic_kernel  every dtype, g and stride: one row per CTA step, fp32 FFMA with R
 //                      in shared memory (or read through L1 when it does not fit).
 #include <algorithm>
+#include <type_traits>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -761,6 +762,253 @@ static ck_status launch_row(const void* x, int64_t M, int64_t K, int64_t sm, con
     return scale_in ? run(rq_row_kernel<T, G, false>) : run(rq_row_kernel<T, G, true>);
 }
 
+// ===================================================================== tensor-core kernel (g = 64)
+
+// One persistent CTA per SM for g = 64 with a row of at most 128 groups.  A tile is the RB
+// rows (RB = floor(128 / (K / 64))) whose group-rows fill the 128 lanes of one
+// tcgen05.mma.kind::f16: D[group-row, c] = sum_i x[group-row, i] R[i, c], M = 128, N = 64,
+// K = 64 (four instructions), fp32 in TMEM.
+//   warp 0       TMA producer: one 3-D box (64 channels x K/64 groups x RB rows) per tile
+//                into a ring of 16 KB stages (128-byte swizzle)
+//   warp 1       TMEM allocation and the MMA-issuing thread; R^T is the B operand, resident
+//                in shared memory; four 64-column accumulators in flight
+//   warps 2-17   four groups of four warps (one per TMEM lane quarter); group k finishes the
+//                tiles i = k (mod 4), whose accumulator is k, so four tiles are in flight:
+//                tcgen05.ld of the lane's group-row (64 channels), round to the dtype, row
+//                absmax through shared atomics and a 4-warp barrier, then the row scale and
+//                the 64 codes of the group-row in four 16-byte stores
+constexpr int kTcXStages = 6;
+constexpr int kTcAcc = 4;                  // TMEM accumulators of 64 columns
+constexpr int kTcEpiWarp0 = 2, kTcEpiWarps = 16;
+constexpr int kTcThreads = (kTcEpiWarp0 + kTcEpiWarps) * 32;
+constexpr int kTcSlots = 3;                // row-absmax slots per group: its j-th tile uses j % 3
+constexpr uint32_t kTcStageBytes = 128 * 128;
+
+struct RqTcParams {
+    int64_t M, K, ldq;
+    int GR;            // group-rows per row (K / 64), at most 128
+    int RB;            // rows per tile, RB * GR <= 128
+    int tiles;
+    uint32_t box_bytes;
+    uint32_t idesc;
+    int vec_codes;
+};
+
+template <typename T, bool DYN>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    rq_tc_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ R,
+                 const float* __restrict__ scale_in, int8_t* __restrict__ codes,
+                 float* __restrict__ scales, RqTcParams p, int* dev_status) {
+    extern __shared__ __align__(1024) unsigned char tc_smem[];
+    unsigned char* base = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(tc_smem) + 1023) & ~uintptr_t(1023));
+    unsigned char* xring = base;
+    unsigned char* rt = base + (size_t)kTcXStages * kTcStageBytes;   // R^T, 8 KB, 1024-aligned
+    __shared__ __align__(8) uint64_t x_full[kTcXStages], x_empty[kTcXStages];
+    __shared__ __align__(8) uint64_t d_full[kTcAcc], d_empty[kTcAcc], amax_bar[kTcAcc], drain_bar;
+    __shared__ unsigned int amax_sh[kTcAcc][kTcSlots][128];
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_flag;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int my_tiles = (int)blockIdx.x < p.tiles ? (p.tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+    if (tid == 0) {
+        for (int s = 0; s < kTcXStages; ++s) {
+            mbar_init(&x_full[s], 1);
+            mbar_init(&x_empty[s], 1);
+        }
+        for (int b = 0; b < kTcAcc; ++b) {
+            mbar_init(&d_full[b], 1);
+            mbar_init(&d_empty[b], 4);     // the four warps of group b
+            mbar_init(&amax_bar[b], 4);
+        }
+        mbar_init(&drain_bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&xmap);
+    }
+    for (int i = tid; i < kTcAcc * kTcSlots * 128; i += kTcThreads) (&amax_sh[0][0][0])[i] = 0u;
+    for (int i = tid; i < 64 * 64; i += kTcThreads) {
+        const int n = i / 64, k = i % 64;   // R^T[n][k] = R[k][n]: the MMA's B operand (N = c)
+        *reinterpret_cast<T*>(rt + rt_off<64>(n, k / 8) + (k % 8) * 2) = R[k * 64 + n];
+    }
+    fence_proxy_async_smem();   // R^T, written by threads, is read by the tensor core
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, kTcAcc * 64);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_sh;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int i = 0; i < my_tiles; ++i) {
+                const int s = i % kTcXStages, f = i / kTcXStages;
+                if (f >= 1 && !mbar_wait(&x_empty[s], (uint32_t)(f - 1) & 1u, &abort_flag, dev_status))
+                    break;
+                mbar_arrive_expect_tx(&x_full[s], p.box_bytes);
+                const int t = (int)blockIdx.x + i * (int)gridDim.x;
+                tma_load_3d(xring + (size_t)s * kTcStageBytes, &xmap, &x_full[s], 0, 0, t * p.RB);
+                ++issued;
+            }
+            if (abort_flag)
+                for (int j = issued > kTcXStages ? issued - kTcXStages : 0; j < issued; ++j)
+                    mbar_wait(&x_full[j % kTcXStages], (uint32_t)(j / kTcXStages) & 1u, nullptr, nullptr);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint64_t adesc0 = smem_desc_k_sw128(smem_u32(xring));
+            const uint64_t bdesc = smem_desc_k_sw128(smem_u32(rt));
+            for (int i = 0; i < my_tiles; ++i) {
+                const int s = i % kTcXStages, b = i % kTcAcc;
+                if (!mbar_wait(&x_full[s], (uint32_t)(i / kTcXStages) & 1u, &abort_flag, dev_status))
+                    break;
+                if (i >= kTcAcc &&
+                    !mbar_wait(&d_empty[b], (uint32_t)((i / kTcAcc) - 1) & 1u, &abort_flag, dev_status))
+                    break;
+                tc_fence_after();
+                const uint64_t adesc = adesc0 + (uint64_t)(s * (kTcStageBytes >> 4));
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)   // K = 16 (32 bytes) per instruction
+                    tc_mma_f16(tmem_base + (uint32_t)(b * 64), adesc + (uint64_t)(kk * 2),
+                               bdesc + (uint64_t)(kk * 2), p.idesc, kk > 0 ? 1u : 0u);
+                tc_commit(&x_empty[s]);
+                tc_commit(&d_full[b]);
+            }
+            tc_commit(&drain_bar);
+            mbar_wait(&drain_bar, 0, nullptr, dev_status);
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue warps
+        const int q = warp & 3;                          // TMEM lanes 32q .. 32q + 31
+        const int grp = (warp - kTcEpiWarp0) >> 2;       // tiles i = grp (mod 4), accumulator grp
+        const int L = q * 32 + lane;                     // the lane's group-row of the tile
+        const bool valid = L < p.RB * p.GR;
+        const int r = valid ? L / p.GR : 0, rho = valid ? L - r * p.GR : 0;
+        const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(grp * 64);
+        int slot = 0;
+        for (int i = grp, j = 0; i < my_tiles; i += kTcAcc, ++j) {
+            const int t = (int)blockIdx.x + i * (int)gridDim.x;
+            const int64_t row = (int64_t)t * p.RB + r;
+            const bool row_ok = valid && row < p.M;
+            if (!__all_sync(0xffffffffu, mbar_wait(&d_full[grp], (uint32_t)j & 1u, &abort_flag,
+                                                   dev_status)))
+                break;
+            tc_fence_after();
+            uint32_t v[64];
+            tc_ld_32x32b_x32(tacc, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+            tc_ld_32x32b_x32(tacc + 32u, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+            tc_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&d_empty[grp]);   // the accumulator is in registers
+            // round to T (the rotation's result dtype) and fold |y| into the row absmax
+            uint32_t yp[32];
+            uint32_t m2 = 0u;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                yp[k] = MmaOp<T>::pack(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+                m2 = MmaOp<T>::absmax2(m2, yp[k]);
+            }
+            // slot (j + 1) % 3 was read during tile j - 2, before any warp of the group arrived
+            // for tile j - 1; it is next written by tile j + 1, after this warp arrives for j
+            if (q == 0)
+                for (int k = lane; k < p.RB; k += 32) amax_sh[grp][slot == 2 ? 0 : slot + 1][k] = 0u;
+            const float2 mf = MmaOp<T>::unpack(m2);
+            if (row_ok) atomicMax(&amax_sh[grp][slot][r], __float_as_uint(fmax_nan(mf.x, mf.y)));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&amax_bar[grp]);
+            if (!__all_sync(0xffffffffu, mbar_wait(&amax_bar[grp], (uint32_t)j & 1u, &abort_flag,
+                                                   dev_status)))
+                break;
+            const unsigned int amax_bits = amax_sh[grp][slot][r];
+            slot = slot == 2 ? 0 : slot + 1;
+            if (!row_ok) continue;
+            const float sc = row_scale(__uint_as_float(amax_bits), DYN ? nullptr : scale_in);
+            const RowDivisor dv(sc);
+            if (rho == 0) scales[row] = sc;
+            int8_t* dst = codes + row * p.ldq + rho * 64;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                uint32_t out[4];
+                if (DYN) {
+                    unsigned long long y2[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) y2[k] = MmaOp<T>::unpack2(yp[8 * u + k]);
+                    quant16_dyn2(y2, dv, out);
+                } else {
+                    float y[16];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const float2 a = MmaOp<T>::unpack(yp[8 * u + k]);
+                        y[2 * k] = a.x;
+                        y[2 * k + 1] = a.y;
+                    }
+                    quant16(y, dv, out);
+                }
+                if (p.vec_codes) {
+                    *reinterpret_cast<uint4*>(dst + 16 * u) = make_uint4(out[0], out[1], out[2], out[3]);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        dst[16 * u + k] = (int8_t)((out[k / 4] >> (8 * (k % 4))) & 0xFF);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTcAcc * 64);
+    }
+}
+
+// Tensor-core kernel for bf16/fp16, g = 64, K / 64 <= 128.  Returns CK_ERR_UNSUPPORTED otherwise.
+template <typename T>
+static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, const void* R,
+                           const float* scale_in, int8_t* codes, int64_t ldq, float* scales,
+                           int* dev_status, cudaStream_t stream, CUtensorMapDataType tdt) {
+    RqTcParams p;
+    p.M = M;
+    p.K = K;
+    p.ldq = ldq;
+    p.GR = (int)(K / 64);
+    if (p.GR < 1 || p.GR > 128) return CK_ERR_UNSUPPORTED;
+    p.RB = 128 / p.GR;
+    const int64_t tiles = (M + p.RB - 1) / p.RB;
+    if (tiles >= (1LL << 31) / p.RB) return CK_ERR_UNSUPPORTED;
+    p.tiles = (int)tiles;
+    p.box_bytes = (uint32_t)(p.RB * p.GR * 128);
+    p.idesc = idesc_f16(128, 64, std::is_same<T, __nv_bfloat16>::value);
+    p.vec_codes = (aligned(codes, 16) && ldq % 16 == 0) ? 1 : 0;
+
+    CUtensorMap map;
+    const uint64_t dims[3] = {64u, (uint64_t)p.GR, (uint64_t)M};
+    const uint64_t strides[2] = {128u, (uint64_t)sm * 2};
+    const uint32_t box[3] = {64u, (uint32_t)p.GR, (uint32_t)p.RB};
+    ck_status st = encode_tma(&map, tdt, 3, x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != CK_OK) return st;
+
+    const size_t smem = (size_t)kTcXStages * kTcStageBytes + 64 * 64 * 2 + 1024;
+    const int grid = (int)(p.tiles < num_sms() ? p.tiles : num_sms());
+    auto run = [&](auto kern) -> ck_status {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return CK_ERR_CUDA;
+        kern<<<grid, kTcThreads, smem, stream>>>(map, static_cast<const T*>(R), scale_in, codes,
+                                                 scales, p, dev_status);
+        return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+    };
+    return scale_in ? run(rq_tc_kernel<T, false>) : run(rq_tc_kernel<T, true>);
+}
+
 // ===================================================================== host launch
 
 template <typename T, int G>
@@ -855,6 +1103,13 @@ ck_status launch_rotate_quant(const void* x, ck_dtype dt, int64_t M, int64_t K, 
                         K / g <= (1LL << 31);
     if (mma_ok) {
         ck_status st = CK_ERR_UNSUPPORTED;
+        if (g == 64)
+            st = dt == CK_BF16 ? launch_tc<__nv_bfloat16>(x, M, K, sm, R, scale_in, codes, ldq, scales,
+                                                          dev_status, stream,
+                                                          CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
+                               : launch_tc<__half>(x, M, K, sm, R, scale_in, codes, ldq, scales,
+                                                   dev_status, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+        if (st != CK_ERR_UNSUPPORTED) return st;
         if (dt == CK_BF16)
             st = g == 64 ? launch_row<__nv_bfloat16, 64>(x, M, K, sm, R, scale_in, codes, ldq, scales,
                                                           dev_status, stream,
