@@ -762,31 +762,47 @@ static ck_status launch_row(const void* x, int64_t M, int64_t K, int64_t sm, con
     return scale_in ? run(rq_row_kernel<T, G, false>) : run(rq_row_kernel<T, G, true>);
 }
 
-// ===================================================================== tensor-core kernel (g = 64)
+// ===================================================================== tensor-core kernel (g = 64, 256)
 
-// One persistent CTA per SM for g = 64 with a row of at most 128 groups.  A tile is the RB
-// rows (RB = floor(128 / (K / 64))) whose group-rows fill the 128 lanes of one
-// tcgen05.mma.kind::f16: D[group-row, c] = sum_i x[group-row, i] R[i, c], M = 128, N = 64,
-// K = 64 (four instructions), fp32 in TMEM.
-//   warp 0       TMA producer: one 3-D box (64 channels x K/64 groups x RB rows) per tile
-//                into a ring of 16 KB stages (128-byte swizzle)
+// One persistent CTA per SM for g in {64, 256} with a row of at most 128 groups.  A tile is
+// the RB rows (RB = floor(128 / (K / g))) whose group-rows fill the 128 lanes of a
+// tcgen05.mma.kind::f16 chain: D[group-row, c] = sum_i x[group-row, i] R[i, c], M = 128,
+// N = g, K = g (g / 16 instructions), fp32 in TMEM.
+//   warp 0       TMA producer: per tile g / 64 boxes (64 channels x K/g groups x RB rows),
+//                each into a 16 KB stage of a ring (128-byte swizzle)
 //   warp 1       TMEM allocation and the MMA-issuing thread; R^T is the B operand, resident
-//                in shared memory; four 64-column accumulators in flight
-//   warps 2-17   four groups of four warps (one per TMEM lane quarter); group k finishes the
-//                tiles i = k (mod 4), whose accumulator is k, so four tiles are in flight:
-//                tcgen05.ld of the lane's group-row (64 channels), round to the dtype, row
-//                absmax through shared atomics and a 4-warp barrier, then the row scale and
-//                the 64 codes of the group-row in four 16-byte stores
-constexpr int kTcXStages = 6;
-constexpr int kTcAcc = 4;                  // TMEM accumulators of 64 columns
+//                in shared memory; kTcAcc<G> accumulators of g columns in flight
+//   warps 2-17   kTcAcc<G> groups of warps; group k finishes the tiles i = k (mod kTcAcc<G>),
+//                whose accumulator is k.  Each warp owns one TMEM lane quarter (its warp
+//                index mod 4) and a column range of the accumulator: tcgen05.ld of the
+//                lane's group-row, round to the dtype, row absmax through shared atomics and
+//                a barrier of the group's warps, then the row scale and the codes in 16-byte
+//                stores.  For g = 64 the rounded values stay in registers between the two
+//                steps; for g = 256 (128 columns a warp) the accumulator is read twice.
+template <int G> constexpr int kTcAcc = G == 64 ? 4 : 2;         // kTcAcc * G <= 512 columns
+template <int G> constexpr int kTcXStages = G == 64 ? 6 : 5;     // 16 KB stages
 constexpr int kTcEpiWarp0 = 2, kTcEpiWarps = 16;
 constexpr int kTcThreads = (kTcEpiWarp0 + kTcEpiWarps) * 32;
 constexpr int kTcSlots = 3;                // row-absmax slots per group: its j-th tile uses j % 3
 constexpr uint32_t kTcStageBytes = 128 * 128;
 
+template <int G>
+constexpr size_t tc_smem_bytes() {
+    return (size_t)kTcXStages<G> * kTcStageBytes + (size_t)G * G * 2 + 1024;
+}
+
+// R^T (B operand, K-major, 128-byte swizzle) in shared memory: K in atoms of 64 values, atom a
+// holds the G rows n (output channel) of 128 bytes with K = 64a .. 64a + 63; the 16-byte chunk
+// of row n is XOR-swizzled by n % 8.
+template <int G>
+__device__ __forceinline__ uint32_t tc_rt_off(int n, int k) {
+    return (uint32_t)(k >> 6) * (uint32_t)(G * 128) + (uint32_t)n * 128u +
+           (uint32_t)((((k & 63) >> 3) ^ (n & 7)) << 4) + (uint32_t)(k & 7) * 2u;
+}
+
 struct RqTcParams {
     int64_t M, K, ldq;
-    int GR;            // group-rows per row (K / 64), at most 128
+    int GR;            // group-rows per row (K / g), at most 128
     int RB;            // rows per tile, RB * GR <= 128
     int tiles;
     uint32_t box_bytes;
@@ -795,47 +811,109 @@ struct RqTcParams {
 };
 
 template <typename T, bool DYN>
+__device__ __forceinline__ void tc_quant_store(const uint32_t (&yp)[8], const RowDivisor& dv,
+                                               const float* scale_in, int8_t* dst, bool vec) {
+    uint32_t out[4];
+    if (DYN) {
+        unsigned long long y2[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) y2[k] = MmaOp<T>::unpack2(yp[k]);
+        quant16_dyn2(y2, dv, out);
+    } else {
+        float y[16];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float2 a = MmaOp<T>::unpack(yp[k]);
+            y[2 * k] = a.x;
+            y[2 * k + 1] = a.y;
+        }
+        quant16(y, dv, out);
+    }
+    if (vec) {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) dst[k] = (int8_t)((out[k / 4] >> (8 * (k % 4))) & 0xFF);
+    }
+}
+
+template <typename T, int G, bool DYN>
 __global__ void __launch_bounds__(kTcThreads, 1)
     rq_tc_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ R,
                  const float* __restrict__ scale_in, int8_t* __restrict__ codes,
                  float* __restrict__ scales, RqTcParams p, int* dev_status) {
+    constexpr int kAcc = kTcAcc<G>, kStages = kTcXStages<G>, kAtoms = G / 64;
+    constexpr int kGrpWarps = kTcEpiWarps / kAcc;   // 4 or 8
+    constexpr int kCols = G / (kGrpWarps / 4);      // accumulator columns a warp finishes
     extern __shared__ __align__(1024) unsigned char tc_smem[];
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(tc_smem) + 1023) & ~uintptr_t(1023));
     unsigned char* xring = base;
-    unsigned char* rt = base + (size_t)kTcXStages * kTcStageBytes;   // R^T, 8 KB, 1024-aligned
-    __shared__ __align__(8) uint64_t x_full[kTcXStages], x_empty[kTcXStages];
-    __shared__ __align__(8) uint64_t d_full[kTcAcc], d_empty[kTcAcc], amax_bar[kTcAcc], drain_bar;
-    __shared__ unsigned int amax_sh[kTcAcc][kTcSlots][128];
+    unsigned char* rt = base + (size_t)kStages * kTcStageBytes;   // R^T, 1024-aligned
+    __shared__ __align__(8) uint64_t x_full[kStages], x_empty[kStages];
+    __shared__ __align__(8) uint64_t d_full[kAcc], d_empty[kAcc], amax_bar[kAcc], drain_bar;
+    __shared__ unsigned int amax_sh[kAcc][kTcSlots][128];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int my_tiles = (int)blockIdx.x < p.tiles ? (p.tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int my_boxes = my_tiles * kAtoms;
+    // box n of this CTA: atom n % kAtoms of its tile n / kAtoms, into stage n % kStages
+    auto issue = [&](int n) {
+        const int s = n % kStages, a = n % kAtoms;
+        const int t = (int)blockIdx.x + (n / kAtoms) * (int)gridDim.x;
+        mbar_arrive_expect_tx(&x_full[s], p.box_bytes);
+        tma_load_3d(xring + (size_t)s * kTcStageBytes, &xmap, &x_full[s], 64 * a, 0, t * p.RB);
+    };
 
     if (tid == 0) {
-        for (int s = 0; s < kTcXStages; ++s) {
+        for (int s = 0; s < kStages; ++s) {
             mbar_init(&x_full[s], 1);
             mbar_init(&x_empty[s], 1);
         }
-        for (int b = 0; b < kTcAcc; ++b) {
+        for (int b = 0; b < kAcc; ++b) {
             mbar_init(&d_full[b], 1);
-            mbar_init(&d_empty[b], 4);     // the four warps of group b
-            mbar_init(&amax_bar[b], 4);
+            mbar_init(&d_empty[b], kGrpWarps);   // the warps of group b
+            mbar_init(&amax_bar[b], kGrpWarps);
         }
         mbar_init(&drain_bar, 1);
         abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&xmap);
+        // the first ring's worth of boxes goes out while the CTA stages R^T
+        for (int n = 0; n < kStages && n < my_boxes; ++n) issue(n);
     }
-    for (int i = tid; i < kTcAcc * kTcSlots * 128; i += kTcThreads) (&amax_sh[0][0][0])[i] = 0u;
-    for (int i = tid; i < 64 * 64; i += kTcThreads) {
-        const int n = i / 64, k = i % 64;   // R^T[n][k] = R[k][n]: the MMA's B operand (N = c)
-        *reinterpret_cast<T*>(rt + rt_off<64>(n, k / 8) + (k % 8) * 2) = R[k * 64 + n];
+    for (int i = tid; i < kAcc * kTcSlots * 128; i += kTcThreads) (&amax_sh[0][0][0])[i] = 0u;
+    // R^T[n][k] = R[k][n] is the MMA's B operand (N = c), staged in 8 x 8 blocks: a thread
+    // loads rows k0 .. k0 + 7 of R at columns n0 .. n0 + 7 (16 bytes each), transposes them in
+    // registers and stores the 16-byte chunks of rows n0 .. n0 + 7 of R^T.  Consecutive
+    // threads take consecutive k0, so a warp's stores cover distinct swizzled chunks.
+    for (int blk = tid; blk < (G / 8) * (G / 8); blk += kTcThreads) {
+        const int k0 = (blk % (G / 8)) * 8, n0 = (blk / (G / 8)) * 8;
+        uint32_t a[8][4];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(R + (size_t)(k0 + r) * G + n0));
+            a[r][0] = v.x;
+            a[r][1] = v.y;
+            a[r][2] = v.z;
+            a[r][3] = v.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            // word w of row n0 + j: (R[k0 + 2w][n0 + j], R[k0 + 2w + 1][n0 + j])
+            const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
+            const uint4 o = make_uint4(__byte_perm(a[0][j / 2], a[1][j / 2], sel),
+                                       __byte_perm(a[2][j / 2], a[3][j / 2], sel),
+                                       __byte_perm(a[4][j / 2], a[5][j / 2], sel),
+                                       __byte_perm(a[6][j / 2], a[7][j / 2], sel));
+            *reinterpret_cast<uint4*>(rt + tc_rt_off<G>(n0 + j, k0)) = o;
+        }
     }
     fence_proxy_async_smem();   // R^T, written by threads, is read by the tensor core
     if (warp == 1) {
-        tmem_alloc(&tmem_base_sh, kTcAcc * 64);
+        tmem_alloc(&tmem_base_sh, kAcc * G);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -846,40 +924,43 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
-            int issued = 0;
-            for (int i = 0; i < my_tiles; ++i) {
-                const int s = i % kTcXStages, f = i / kTcXStages;
-                if (f >= 1 && !mbar_wait(&x_empty[s], (uint32_t)(f - 1) & 1u, &abort_flag, dev_status))
-                    break;
-                mbar_arrive_expect_tx(&x_full[s], p.box_bytes);
-                const int t = (int)blockIdx.x + i * (int)gridDim.x;
-                tma_load_3d(xring + (size_t)s * kTcStageBytes, &xmap, &x_full[s], 0, 0, t * p.RB);
-                ++issued;
+            int issued = my_boxes < kStages ? my_boxes : kStages;
+            for (; issued < my_boxes; ++issued) {
+                const int s = issued % kStages, f = issued / kStages;
+                if (!mbar_wait(&x_empty[s], (uint32_t)(f - 1) & 1u, &abort_flag, dev_status)) break;
+                issue(issued);
             }
             if (abort_flag)
-                for (int j = issued > kTcXStages ? issued - kTcXStages : 0; j < issued; ++j)
-                    mbar_wait(&x_full[j % kTcXStages], (uint32_t)(j / kTcXStages) & 1u, nullptr, nullptr);
+                for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
+                    mbar_wait(&x_full[j % kStages], (uint32_t)(j / kStages) & 1u, nullptr, nullptr);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint64_t adesc0 = smem_desc_k_sw128(smem_u32(xring));
-            const uint64_t bdesc = smem_desc_k_sw128(smem_u32(rt));
-            for (int i = 0; i < my_tiles; ++i) {
-                const int s = i % kTcXStages, b = i % kTcAcc;
-                if (!mbar_wait(&x_full[s], (uint32_t)(i / kTcXStages) & 1u, &abort_flag, dev_status))
+            const uint64_t bdesc0 = smem_desc_k_sw128(smem_u32(rt));
+            bool ok = true;
+            for (int i = 0; i < my_tiles && ok; ++i) {
+                const int b = i % kAcc;
+                if (i >= kAcc &&
+                    !mbar_wait(&d_empty[b], (uint32_t)((i / kAcc) - 1) & 1u, &abort_flag, dev_status))
                     break;
-                if (i >= kTcAcc &&
-                    !mbar_wait(&d_empty[b], (uint32_t)((i / kTcAcc) - 1) & 1u, &abort_flag, dev_status))
-                    break;
-                tc_fence_after();
-                const uint64_t adesc = adesc0 + (uint64_t)(s * (kTcStageBytes >> 4));
+                for (int a = 0; a < kAtoms; ++a) {
+                    const int n = i * kAtoms + a, s = n % kStages;
+                    if (!mbar_wait(&x_full[s], (uint32_t)(n / kStages) & 1u, &abort_flag, dev_status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t adesc = adesc0 + (uint64_t)(s * (kTcStageBytes >> 4));
+                    const uint64_t bdesc = bdesc0 + (uint64_t)(a * ((G * 128) >> 4));
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)   // K = 16 (32 bytes) per instruction
-                    tc_mma_f16(tmem_base + (uint32_t)(b * 64), adesc + (uint64_t)(kk * 2),
-                               bdesc + (uint64_t)(kk * 2), p.idesc, kk > 0 ? 1u : 0u);
-                tc_commit(&x_empty[s]);
-                tc_commit(&d_full[b]);
+                    for (int kk = 0; kk < 4; ++kk)   // K = 16 (32 bytes) per instruction
+                        tc_mma_f16(tmem_base + (uint32_t)(b * G), adesc + (uint64_t)(kk * 2),
+                                   bdesc + (uint64_t)(kk * 2), p.idesc, (a > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&x_empty[s]);
+                }
+                if (ok) tc_commit(&d_full[b]);
             }
             tc_commit(&drain_bar);
             mbar_wait(&drain_bar, 0, nullptr, dev_status);
@@ -887,13 +968,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else {
         // ---------------------------------------------------------------- epilogue warps
         const int q = warp & 3;                          // TMEM lanes 32q .. 32q + 31
-        const int grp = (warp - kTcEpiWarp0) >> 2;       // tiles i = grp (mod 4), accumulator grp
+        const int e = warp - kTcEpiWarp0;
+        const int grp = e / kGrpWarps;                   // tiles i = grp (mod kAcc), accumulator grp
+        const int h = (e % kGrpWarps) >> 2;              // column range h * kCols .. + kCols
         const int L = q * 32 + lane;                     // the lane's group-row of the tile
         const bool valid = L < p.RB * p.GR;
         const int r = valid ? L / p.GR : 0, rho = valid ? L - r * p.GR : 0;
-        const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(grp * 64);
+        const uint32_t tacc =
+            tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(grp * G + h * kCols);
+        const bool zeroer = q == 0 && h == 0;
         int slot = 0;
-        for (int i = grp, j = 0; i < my_tiles; i += kTcAcc, ++j) {
+        for (int i = grp, j = 0; i < my_tiles; i += kAcc, ++j) {
             const int t = (int)blockIdx.x + i * (int)gridDim.x;
             const int64_t row = (int64_t)t * p.RB + r;
             const bool row_ok = valid && row < p.M;
@@ -901,24 +986,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                                    dev_status)))
                 break;
             tc_fence_after();
-            uint32_t v[64];
-            tc_ld_32x32b_x32(tacc, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-            tc_ld_32x32b_x32(tacc + 32u, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-            tc_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&d_empty[grp]);   // the accumulator is in registers
             // round to T (the rotation's result dtype) and fold |y| into the row absmax
-            uint32_t yp[32];
+            uint32_t yp[kCols == 64 ? 32 : 1];
             uint32_t m2 = 0u;
+            if constexpr (kCols == 64) {
+                uint32_t v[64];
+                tc_ld_32x32b_x32(tacc, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                tc_ld_32x32b_x32(tacc + 32u, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                tc_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&d_empty[grp]);   // the accumulator is in registers
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                yp[k] = MmaOp<T>::pack(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
-                m2 = MmaOp<T>::absmax2(m2, yp[k]);
+                for (int k = 0; k < 32; ++k) {
+                    yp[k] = MmaOp<T>::pack(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+                    m2 = MmaOp<T>::absmax2(m2, yp[k]);
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < kCols; c += 32) {
+                    uint32_t v[32];
+                    tc_ld_32x32b_x32(tacc + (uint32_t)c, v);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        m2 = MmaOp<T>::absmax2(
+                            m2, MmaOp<T>::pack(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1])));
+                }
             }
             // slot (j + 1) % 3 was read during tile j - 2, before any warp of the group arrived
             // for tile j - 1; it is next written by tile j + 1, after this warp arrives for j
-            if (q == 0)
+            if (zeroer)
                 for (int k = lane; k < p.RB; k += 32) amax_sh[grp][slot == 2 ? 0 : slot + 1][k] = 0u;
             const float2 mf = MmaOp<T>::unpack(m2);
             if (row_ok) atomicMax(&amax_sh[grp][slot][r], __float_as_uint(fmax_nan(mf.x, mf.y)));
@@ -929,36 +1027,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 break;
             const unsigned int amax_bits = amax_sh[grp][slot][r];
             slot = slot == 2 ? 0 : slot + 1;
-            if (!row_ok) continue;
             const float sc = row_scale(__uint_as_float(amax_bits), DYN ? nullptr : scale_in);
             const RowDivisor dv(sc);
-            if (rho == 0) scales[row] = sc;
-            int8_t* dst = codes + row * p.ldq + rho * 64;
+            if (row_ok && rho == 0 && h == 0) scales[row] = sc;
+            int8_t* dst = codes + row * p.ldq + rho * G + h * kCols;
+            if constexpr (kCols == 64) {
+                if (row_ok) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                uint32_t out[4];
-                if (DYN) {
-                    unsigned long long y2[8];
+                    for (int u = 0; u < 4; ++u)
+                        tc_quant_store<T, DYN>(*reinterpret_cast<const uint32_t(*)[8]>(&yp[8 * u]),
+                                               dv, scale_in, dst + 16 * u, p.vec_codes != 0);
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < kCols; c += 32) {
+                    uint32_t v[32];
+                    tc_ld_32x32b_x32(tacc + (uint32_t)c, v);
+                    tc_wait_ld();
+                    if (row_ok) {
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) y2[k] = MmaOp<T>::unpack2(yp[8 * u + k]);
-                    quant16_dyn2(y2, dv, out);
-                } else {
-                    float y[16];
+                        for (int u = 0; u < 2; ++u) {
+                            uint32_t y8[8];
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const float2 a = MmaOp<T>::unpack(yp[8 * u + k]);
-                        y[2 * k] = a.x;
-                        y[2 * k + 1] = a.y;
+                            for (int k = 0; k < 8; ++k)
+                                y8[k] = MmaOp<T>::pack(__uint_as_float(v[16 * u + 2 * k]),
+                                                       __uint_as_float(v[16 * u + 2 * k + 1]));
+                            tc_quant_store<T, DYN>(y8, dv, scale_in, dst + c + 16 * u,
+                                                   p.vec_codes != 0);
+                        }
                     }
-                    quant16(y, dv, out);
                 }
-                if (p.vec_codes) {
-                    *reinterpret_cast<uint4*>(dst + 16 * u) = make_uint4(out[0], out[1], out[2], out[3]);
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        dst[16 * u + k] = (int8_t)((out[k / 4] >> (8 * (k % 4))) & 0xFF);
-                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&d_empty[grp]);   // done reading the accumulator
             }
         }
     }
@@ -966,12 +1067,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTcAcc * 64);
+        tmem_dealloc(tmem_base, kTcAcc<G> * G);
     }
 }
 
-// Tensor-core kernel for bf16/fp16, g = 64, K / 64 <= 128.  Returns CK_ERR_UNSUPPORTED otherwise.
-template <typename T>
+// Tensor-core kernel for bf16/fp16, g in {64, 256}, K / g <= 128.  Returns
+// CK_ERR_UNSUPPORTED otherwise.
+template <typename T, int G>
 static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, const void* R,
                            const float* scale_in, int8_t* codes, int64_t ldq, float* scales,
                            int* dev_status, cudaStream_t stream, CUtensorMapDataType tdt) {
@@ -979,24 +1081,26 @@ static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, cons
     p.M = M;
     p.K = K;
     p.ldq = ldq;
-    p.GR = (int)(K / 64);
-    if (p.GR < 1 || p.GR > 128) return CK_ERR_UNSUPPORTED;
+    if (K % G != 0 || K / G < 1 || K / G > 128) return CK_ERR_UNSUPPORTED;
+    p.GR = (int)(K / G);
     p.RB = 128 / p.GR;
     const int64_t tiles = (M + p.RB - 1) / p.RB;
     if (tiles >= (1LL << 31) / p.RB) return CK_ERR_UNSUPPORTED;
     p.tiles = (int)tiles;
     p.box_bytes = (uint32_t)(p.RB * p.GR * 128);
-    p.idesc = idesc_f16(128, 64, std::is_same<T, __nv_bfloat16>::value);
+    p.idesc = idesc_f16(128, G, std::is_same<T, __nv_bfloat16>::value);
     p.vec_codes = (aligned(codes, 16) && ldq % 16 == 0) ? 1 : 0;
 
+    // x as (channel within group, group, row); each box is 64 channels (128 bytes) of every
+    // group of RB rows, fetched at channel offsets 0, 64, .. G - 64
     CUtensorMap map;
-    const uint64_t dims[3] = {64u, (uint64_t)p.GR, (uint64_t)M};
-    const uint64_t strides[2] = {128u, (uint64_t)sm * 2};
+    const uint64_t dims[3] = {(uint64_t)G, (uint64_t)p.GR, (uint64_t)M};
+    const uint64_t strides[2] = {(uint64_t)G * 2, (uint64_t)sm * 2};
     const uint32_t box[3] = {64u, (uint32_t)p.GR, (uint32_t)p.RB};
     ck_status st = encode_tma(&map, tdt, 3, x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != CK_OK) return st;
 
-    const size_t smem = (size_t)kTcXStages * kTcStageBytes + 64 * 64 * 2 + 1024;
+    const size_t smem = tc_smem_bytes<G>();
     const int grid = (int)(p.tiles < num_sms() ? p.tiles : num_sms());
     auto run = [&](auto kern) -> ck_status {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -1006,7 +1110,7 @@ static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, cons
                                                  scales, p, dev_status);
         return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
     };
-    return scale_in ? run(rq_tc_kernel<T, false>) : run(rq_tc_kernel<T, true>);
+    return scale_in ? run(rq_tc_kernel<T, G, false>) : run(rq_tc_kernel<T, G, true>);
 }
 
 // ===================================================================== host launch
@@ -1101,15 +1205,27 @@ ck_status launch_rotate_quant(const void* x, ck_dtype dt, int64_t M, int64_t K, 
     const bool mma_ok = (dt == CK_BF16 || dt == CK_F16) && (g == 16 || g == 64) && sk == 1 &&
                         aligned(x, 16) && sm % 8 == 0 && sm > 0 && M < (1LL << 31) &&
                         K / g <= (1LL << 31);
-    if (mma_ok) {
-        ck_status st = CK_ERR_UNSUPPORTED;
-        if (g == 64)
-            st = dt == CK_BF16 ? launch_tc<__nv_bfloat16>(x, M, K, sm, R, scale_in, codes, ldq, scales,
+    const bool tc_ok = (dt == CK_BF16 || dt == CK_F16) && (g == 64 || g == 256) && sk == 1 &&
+                       aligned(x, 16) && aligned(R, 16) && sm % 8 == 0 && sm > 0 &&
+                       M < (1LL << 31);
+    if (tc_ok) {
+        ck_status st;
+        if (dt == CK_BF16)
+            st = g == 64 ? launch_tc<__nv_bfloat16, 64>(x, M, K, sm, R, scale_in, codes, ldq, scales,
+                                                         dev_status, stream,
+                                                         CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
+                         : launch_tc<__nv_bfloat16, 256>(x, M, K, sm, R, scale_in, codes, ldq, scales,
                                                           dev_status, stream,
-                                                          CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
-                               : launch_tc<__half>(x, M, K, sm, R, scale_in, codes, ldq, scales,
+                                                          CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+        else
+            st = g == 64 ? launch_tc<__half, 64>(x, M, K, sm, R, scale_in, codes, ldq, scales,
+                                                  dev_status, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)
+                         : launch_tc<__half, 256>(x, M, K, sm, R, scale_in, codes, ldq, scales,
                                                    dev_status, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
         if (st != CK_ERR_UNSUPPORTED) return st;
+    }
+    if (mma_ok) {
+        ck_status st = CK_ERR_UNSUPPORTED;
         if (dt == CK_BF16)
             st = g == 64 ? launch_row<__nv_bfloat16, 64>(x, M, K, sm, R, scale_in, codes, ldq, scales,
                                                           dev_status, stream,

@@ -135,6 +135,26 @@ def test_rotate_quant_small_every_row(dt, g, layout):
     compare_stage1(codes.cpu().numpy(), scales.cpu().numpy(), oc, os_, DT[dt], case.name, g)
 
 
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+@pytest.mark.parametrize("g,groups,M", [(64, 1, 1000), (64, 127, 200), (64, 128, 160), (64, 129, 20),
+                                        (256, 1, 1000), (256, 43, 333), (256, 128, 150),
+                                        (256, 129, 3)])
+def test_rotate_quant_tile_shapes(dt, g, groups, M):
+    """Rows of 1 to 129 groups: a tile packs floor(128 / groups) rows, so these cover a tile of
+    128 one-group rows, one row of 127 or 128 groups, a ragged last tile, more tiles than SMs
+    (150 rows of 128 groups), and the first row length past 128 groups, which another kernel
+    takes.  R is a non-symmetric orthogonal matrix, so R and R^T give different results.
+    Every output is compared."""
+    case = W.RotateCase(f"tiles_{dt}_{g}_{groups}", M=M, K=g * groups, g=g, dtype=dt,
+                        seed=groups + g)
+    x = W.make_rotate_inputs(case)["x"]
+    R = W.haar_orthogonal(g, torch.Generator().manual_seed(g + groups)).to(DT[dt]).contiguous()
+    codes, scales = ck.ck_rotate_quant(to_device(x), R.cuda(), g)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.rotate_quant(x, R, g)
+    compare_stage1(codes.cpu().numpy(), scales.cpu().numpy(), oc, os_, DT[dt], case.name, g)
+
+
 @pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
 def test_rotate_quant_zero_rows_and_caller_zero_scale(dt):
     x = torch.randn(20, 128, generator=torch.Generator().manual_seed(5)).to(DT[dt])
