@@ -310,22 +310,31 @@ __device__ __forceinline__ int quant_code(float y, float s) {
 // With r correctly rounded and t within a few ulps of y / s, q is the correctly rounded
 // quotient fl(y / s) as long as the remainder e is not subnormal.  The quotients needed
 // here are below 2^23 and y is at least 2^-24 |q| s, so s >= 2^-64 keeps e far above the
-// subnormal range.  `fast` is false when s is below that bound, not finite, or NaN, or when
-// r is not a normal number; every code of such a row takes the IEEE division.
+// subnormal range.  A power of two s (for instance the FLT_MIN of an all-zero row) is fast at
+// any size: r = 1 / s exactly, so t = y r is the exact quotient whenever it is a normal
+// number (then e = 0 and q = t), and a quotient below the normal range gives code 0 either way.
+// Where t overflows or is at least 16 (a caller's scale far below the values), the code
+// saturates by the sign of t, which the callers take instead of q (the correction would turn
+// an infinite t into NaN).  `fast` is false when s is below 2^-64 and not a power of two, not
+// finite, or NaN, or when r is not a normal number; every code of such a row takes the IEEE
+// division.
 struct RowDivisor {
     float s, r;
     bool fast;
     __device__ __forceinline__ explicit RowDivisor(float s_) : s(s_) {
         r = __frcp_rn(s_);
-        fast = (s_ >= 0x1p-64f) && (r >= 1.17549435e-38f) && (r <= 3.40282347e38f);
+        const bool pow2 = (__float_as_uint(s_) & 0x007FFFFFu) == 0u;
+        fast = (s_ >= 0x1p-64f || pow2) && (r >= 1.17549435e-38f) && (r <= 3.40282347e38f);
     }
 };
 
-// fl(y / s) for a fast RowDivisor (Markstein's correction, see RowDivisor).
+// fl(y / s) for a fast RowDivisor (Markstein's correction, see RowDivisor), or y r where
+// |y r| >= 16, which saturates the code the same way.
 __device__ __forceinline__ float quotient_fast(float y, float s, float r) {
     const float t = __fmul_rn(y, r);
     const float e = __fmaf_rn(-t, s, y);
-    return __fmaf_rn(e, r, t);
+    const float q = __fmaf_rn(e, r, t);
+    return fabsf(t) < 16.0f ? q : t;
 }
 
 // The same code as quant_code(y, d.s): the IEEE quotient from a reciprocal multiply and
@@ -355,8 +364,9 @@ __device__ __forceinline__ void quant16(const float (&y)[16], const RowDivisor& 
             const unsigned long long t = mul2s_rn(y2, d.r);
             const unsigned long long e = fma2_rn(t, ns, y2);
             const float2 qq = f2_unpack(fma2_rn(e, r2, t));
-            q[i] = __float2int_rn(qq.x);          // NaN -> 0; +-inf saturates
-            q[i + 1] = __float2int_rn(qq.y);
+            const float2 tt = f2_unpack(t);       // |t| >= 16: the code saturates by sign
+            q[i] = __float2int_rn(fabsf(tt.x) < 16.0f ? qq.x : tt.x);   // NaN -> 0
+            q[i + 1] = __float2int_rn(fabsf(tt.y) < 16.0f ? qq.y : tt.y);
         }
     } else {
 #pragma unroll

@@ -418,3 +418,29 @@ def test_quantizer_codes_bit_exact_with_identity_rotation(dt, g):
     oc, os_ = oracle.rotate_quant(xt, R, g)
     np.testing.assert_array_equal(scales.cpu().numpy(), os_)
     np.testing.assert_array_equal(codes.cpu().numpy(), oc)
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("g", [16, 64, 256])
+def test_quantizer_caller_scale_extremes_with_identity_rotation(dt, g):
+    """A caller's scale far from the data, R = I so that y = x exactly.  With s = 1e-10 and
+    values up to 3e35, y / s overflows fp32 and every nonzero code saturates by sign; with
+    s = 2^-100 (a power of two below 2^-64) and x = k/2 * 2^-100, the quotients are exact
+    half-integers and the codes are their ties rounded half to even."""
+    rng = np.random.default_rng(77 + g)
+    M, K = 24, g * 8
+    x = rng.standard_normal((M, K))
+    x[1, 5] = 1e30
+    x[2, 7] = -3e35
+    x[3] = 1e20
+    x[4] = 0.0
+    xt = torch.from_numpy(x).to(DT[dt])
+    R = torch.eye(g, dtype=DT[dt])
+    for sc, xs in ((1e-10, xt), (2.0 ** -100, (torch.from_numpy(rng.integers(-20, 21, size=(M, K)) / 2.0)
+                                             * 2.0 ** -100).to(DT[dt]))):
+        scale = torch.tensor([sc], dtype=torch.float32)
+        codes, scales = ck.ck_rotate_quant(xs.cuda(), R.cuda(), g, scale_in=scale.cuda())
+        torch.cuda.synchronize()
+        oc, os_ = oracle.rotate_quant(xs, R, g, scale_in=float(scale))
+        np.testing.assert_array_equal(scales.cpu().numpy(), os_)
+        np.testing.assert_array_equal(codes.cpu().numpy(), oc)
