@@ -155,6 +155,21 @@ def test_rotate_quant_tile_shapes(dt, g, groups, M):
     compare_stage1(codes.cpu().numpy(), scales.cpu().numpy(), oc, os_, DT[dt], case.name, g)
 
 
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+@pytest.mark.parametrize("g,K", [(16, 16384), (16, 32768), (64, 16384), (64, 32768), (256, 16384)])
+def test_rotate_quant_long_rows(dt, g, K):
+    """Rows longer than the row kernel's two double-buffered rows per warp hold (K > 12800 for
+    16-bit inputs at g = 16 and 64), which the block-ring kernel takes, and a g = 256 row of 64
+    groups (tensor-core kernel, two rows per tile).  Every output is compared."""
+    case = W.RotateCase(f"long_{dt}_{g}_{K}", M=45, K=K, g=g, dtype=dt, seed=K // g)
+    x = W.make_rotate_inputs(case)["x"]
+    R = W.haar_orthogonal(g, torch.Generator().manual_seed(K + g)).to(DT[dt]).contiguous()
+    codes, scales = ck.ck_rotate_quant(to_device(x), R.cuda(), g)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.rotate_quant(x, R, g)
+    compare_stage1(codes.cpu().numpy(), scales.cpu().numpy(), oc, os_, DT[dt], case.name, g)
+
+
 @pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
 def test_rotate_quant_zero_rows_and_caller_zero_scale(dt):
     x = torch.randn(20, 128, generator=torch.Generator().manual_seed(5)).to(DT[dt])
