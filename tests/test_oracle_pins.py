@@ -242,6 +242,31 @@ def test_caller_zero_scale_follows_eager_semantics():
     np.testing.assert_array_equal(codes[xv < 0], -8)
 
 
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_caller_scale_far_from_the_data(dt):
+    """Closed forms for a caller's scale, with R = I so that y = x.  Below the data (s = 1e-10,
+    values up to 3e35, where y / s overflows fp32) every code is the sign's saturated value.  A
+    power of two (s = 2^-100) divides exactly, so the codes of x = k/2 * 2^-100 are the
+    half-integers k/2 rounded half to even and clamped, computed here with Python's round()."""
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((6, 64))
+    x[1, 5] = 1e30
+    x[2, 7] = -3e35
+    x[4] = 0.0
+    R = torch.eye(16, dtype=TORCH_DT[dt])
+    xt = torch.from_numpy(x).to(TORCH_DT[dt])
+    codes, scales = oracle.rotate_quant(xt, R, 16, scale_in=1e-10)
+    assert (scales == np.float32(1e-10)).all()
+    xv = xt.double().numpy()
+    np.testing.assert_array_equal(codes, np.where(xv > 0, 7, np.where(xv < 0, -8, 0)))
+
+    k = rng.integers(-20, 21, size=(6, 64))
+    xt = torch.from_numpy(k / 2.0 * 2.0 ** -100).to(TORCH_DT[dt])
+    codes, _ = oracle.rotate_quant(xt, R, 16, scale_in=2.0 ** -100)
+    want = np.vectorize(lambda v: max(-8, min(7, round(v / 2))))(k)   # round(): half to even
+    np.testing.assert_array_equal(codes, want)
+
+
 @pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
 def test_dynamic_codes_reach_seven_and_never_minus_eight(dt):
     case = W.RotateCase("t", M=40, K=512, g=64, dtype=dt, seed=11)
