@@ -8,14 +8,22 @@
 //   s[m] = max(fp32(max_k |y[m, k]|) / 7, FLT_MIN)   or the caller's tensor-wise scale
 //   q[m, k] = clamp(round_half_even(y[m, k] / s[m]), -8, 7)
 //
-// Two kernels:
-//   rq_mma_kernel      bf16/fp16, g in {16, 64}, unit K stride, 16-byte aligned rows.
-//                      A block of rows arrives by one TMA tensor copy (swizzled, so the
-//                      warp-level MMA fragment loads are bank-conflict free), is rotated
-//                      in place by mma.sync with R held in registers, and then quantized
-//                      from shared memory with 16-byte coalesced code stores.
+// Four kernels, tried in this order:
+//   rq_tc_kernel       bf16/fp16, g in {64, 256}, rows of at most 128 groups, unit K stride,
+//                      16-byte aligned x and R.  Whole rows fill the 128 lanes of a
+//                      tcgen05.mma.kind::f16 chain against R^T resident in shared memory; the
+//                      fp32 result in tensor memory is rounded, reduced and quantized by
+//                      sixteen epilogue warps, several tiles in flight.
+//   rq_row_kernel      bf16/fp16, g in {16, 64}, rows that fit two buffers per warp.  Each warp
+//                      owns whole rows, filled by its own TMA copies, and rotates them with
+//                      mma.sync (y^T = R^T x^T) in place.
+//   rq_mma_kernel      bf16/fp16, g in {16, 64}, longer rows.  A TMA producer fills a ring of
+//                      row blocks; two groups of compute warps rotate them with mma.sync and
+//                      quantize from shared memory.
 //   rq_generic_kernel  every dtype, g and stride: one row per CTA step, fp32 FFMA with R
 //                      in shared memory (or read through L1 when it does not fit).
+// The TMA-fed kernels store 16 codes at a time where the code rows are 16-byte aligned; the
+// generic kernel stores 4.
 #include <algorithm>
 #include <type_traits>
 
