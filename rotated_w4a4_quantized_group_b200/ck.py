@@ -82,10 +82,15 @@ def _stream(stream) -> int | None:
 
 
 def _ptr(t) -> int | None:
+    """Device address of a tensor argument (None stays NULL, an int is taken as an address).
+    A tensor outside GPU memory is refused here: the library would hand its host address to
+    the device."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_cuda:
+        raise ValueError(f"ck: tensor arguments must live on a CUDA device, got one on {t.device}")
     return t.data_ptr()
 
 

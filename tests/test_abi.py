@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from rotated_w4a4_quantized_group_b200 import build as ck_build
 from rotated_w4a4_quantized_group_b200 import ck
@@ -140,3 +141,13 @@ def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(ck, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         ck.lib()
+
+
+def test_binding_refuses_host_tensors(L):
+    """A CPU tensor never reaches the library: its address would be read by the device."""
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    R = torch.eye(64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA device"):
+        ck.ck_rotate_quant(x, R, 64)
+    with pytest.raises(ValueError, match="CUDA device"):
+        ck.ck_unpack_w4(torch.zeros(4, 32, dtype=torch.int8), 64)
