@@ -152,12 +152,18 @@ ck_status ck_unpack_w4(const int8_t* packed, int64_t N, int64_t K, int64_t ld_pa
  * Scratch memory comes from an array compiled into the library: 32 MiB of device memory
  * that every GPU which loads the library holds until the process exits.  The call allocates
  * nothing (no cudaMalloc, cudaFree or allocating library routine).
- *   - Limit: calls whose scratch need (ck_w4a4_linear_workspace_bytes for the same sizes,
- *     or 0 for 16-byte-aligned int8 codes with 16-byte-pitched weights) exceeds 32 MiB
- *     return CK_ERR_WORKSPACE and launch nothing (e.g. 8192 x 3840 activations fit,
- *     8192 x 10240 do not).
+ *   - Limit: calls whose scratch need exceeds 32 MiB return CK_ERR_WORKSPACE and launch
+ *     nothing (e.g. 8192 x 3840 activations fit, 8192 x 10240 do not).  The need is the
+ *     scratch ck_w4a4_linear uses for this call: the stage-1 codes and scales of
+ *     floating-point input (ck_workspace_scales_offset(M, K) + 4 M, rounded up to 256), the
+ *     same for int8 codes whose rows are not 16-byte aligned (0 for aligned ones), plus a
+ *     16-byte-pitched weight copy when w_packed is not 16-byte aligned and pitched.
  *   - The first call on each device looks up the array's device address (with that device
- *     current); make that first call before any stream capture.
+ *     current) and caches it; after a device reset, which ends the context and may move the
+ *     array, the next call looks it up again.  Make the first call on a device before any
+ *     stream capture.
+ *   - Every pointer must refer to memory of the calling thread's current device (the array
+ *     used is the current device's).
  *   - Every call on a device shares the one array and nothing in it needs clearing between
  *     calls; calls whose GPU work overlaps in time (different streams) race on it.
  */

@@ -74,6 +74,8 @@ def _check(status: int, where: str):
 
 
 def _stream(stream) -> int | None:
+    """The caller's stream, or torch's current stream of the current device (every entry
+    point makes its tensors' device current before asking)."""
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
     if isinstance(stream, torch.cuda.Stream):
@@ -119,15 +121,46 @@ def ck_rotate_quant(x: torch.Tensor, R: torch.Tensor, g: int, scale_in: torch.Te
     """Stage 1 on a 2-D (M, K) CUDA view; returns (codes int8 (M, K), scales fp32 (M,))."""
     M, K = x.shape
     _check_rotation(x, R, g)
+    _same_device(x, R, scale_in, codes, scales, dev_status)
     if codes is None:
         codes = torch.empty(M, K, dtype=torch.int8, device=x.device)
     if scales is None:
         scales = torch.empty(M, dtype=torch.float32, device=x.device)
-    st = lib().ck_rotate_quant(_ptr(x), DTYPE_CODE[x.dtype], M, K, x.stride(0), x.stride(1),
-                               _ptr(R), g, _ptr(scale_in), _ptr(codes), codes.stride(0),
-                               _ptr(scales), _ptr(dev_status), _stream(stream))
+    if codes.dtype != torch.int8 or tuple(codes.shape) != (M, K) or codes.stride(1) != 1:
+        raise ValueError(f"codes must be an int8 ({M}, {K}) view with unit inner stride")
+    if scales.dtype != torch.float32 or scales.numel() < M or not scales.is_contiguous():
+        raise ValueError(f"scales must be a contiguous fp32 tensor of at least {M} values")
+    with torch.cuda.device(x.device):
+        st = lib().ck_rotate_quant(_ptr(x), DTYPE_CODE[x.dtype], M, K, x.stride(0), x.stride(1),
+                                   _ptr(R), g, _ptr(scale_in), _ptr(codes), codes.stride(0),
+                                   _ptr(scales), _ptr(dev_status), _stream(stream))
     _check(st, "ck_rotate_quant")
     return codes, scales
+
+
+def _check_weights(w_packed: torch.Tensor, N: int, K: int):
+    # the library reads N rows of K/2 bytes through the row pitch w_packed.stride(0)
+    if w_packed.dtype != torch.int8 or w_packed.dim() != 2 or w_packed.stride(1) != 1 or \
+            tuple(w_packed.shape) != (N, K // 2):
+        raise ValueError(f"w_packed must be an int8 (N, K/2) = ({N}, {K // 2}) view with unit inner "
+                         f"stride; got {tuple(w_packed.shape)} {w_packed.dtype} strides "
+                         f"{w_packed.stride()}")
+
+
+def _check_out(out: torch.Tensor, M: int, N: int, x: torch.Tensor):
+    # the library writes M rows of N values through the row pitch out.stride(0)
+    if tuple(out.shape) != (M, N) or out.stride(1) != 1 or out.device != x.device:
+        raise ValueError(f"out must be an (M, N) = ({M}, {N}) view with unit inner stride on "
+                         f"{x.device}; got {tuple(out.shape)} strides {out.stride()} on {out.device}")
+
+
+def _same_device(x: torch.Tensor, *ts):
+    """Every tensor argument on x's CUDA device (a host tensor's address would be read by the
+    device; a tensor on another GPU would be read through the wrong device's memory)."""
+    _ptr(x)
+    for t in ts:
+        if t is not None and not isinstance(t, int) and t.device != x.device:
+            raise ValueError(f"every tensor must be on {x.device}; got one on {t.device}")
 
 
 def ck_w4a4_linear(x: torch.Tensor, R: torch.Tensor | None, g: int, w_packed: torch.Tensor,
@@ -141,19 +174,21 @@ def ck_w4a4_linear(x: torch.Tensor, R: torch.Tensor | None, g: int, w_packed: to
     N = w_packed.shape[0]
     if x.dtype != torch.int8:
         _check_rotation(x, R, g)
-    if w_packed.stride(1) != 1 or tuple(w_packed.shape) != (N, K // 2):
-        raise ValueError("w_packed must be (N, K/2) with unit inner stride")
+    _check_weights(w_packed, N, K)
+    _same_device(x, R, w_packed, w_scale, bias, a_scale, workspace, dev_status)
     if out is None:
         odt = out_dtype or (x.dtype if x.dtype != torch.int8 else w_scale.dtype)
         out = torch.empty(M, N, dtype=odt, device=x.device)
-    if workspace is None:
-        nbytes = workspace_bytes(M, N, K, w_packed.stride(0))
-        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
-    st = lib().ck_w4a4_linear(
-        _ptr(x), DTYPE_CODE[x.dtype], M, K, x.stride(0), x.stride(1), _ptr(R), int(g),
-        _ptr(a_scale), _ptr(w_packed), N, w_packed.stride(0), _ptr(w_scale),
-        DTYPE_CODE[w_scale.dtype], _ptr(bias), _ptr(out), DTYPE_CODE[out.dtype], out.stride(0),
-        _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream))
+    _check_out(out, M, N, x)
+    with torch.cuda.device(x.device):
+        if workspace is None:
+            nbytes = workspace_bytes(M, N, K, w_packed.stride(0))
+            workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+        st = lib().ck_w4a4_linear(
+            _ptr(x), DTYPE_CODE[x.dtype], M, K, x.stride(0), x.stride(1), _ptr(R), int(g),
+            _ptr(a_scale), _ptr(w_packed), N, w_packed.stride(0), _ptr(w_scale),
+            DTYPE_CODE[w_scale.dtype], _ptr(bias), _ptr(out), DTYPE_CODE[out.dtype],
+            out.stride(0), _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream))
     _check(st, "ck_w4a4_linear")
     return out
 
@@ -169,11 +204,15 @@ def ck_w4a4_linear_noalloc(x: torch.Tensor, R: torch.Tensor | None, g: int,
     N = w_packed.shape[0]
     if x.dtype != torch.int8:
         _check_rotation(x, R, g)
-    st = lib().ck_w4a4_linear_noalloc(
-        _ptr(x), DTYPE_CODE[x.dtype], M, K, x.stride(0), x.stride(1), _ptr(R), int(g),
-        _ptr(a_scale), _ptr(w_packed), N, w_packed.stride(0), _ptr(w_scale),
-        DTYPE_CODE[w_scale.dtype], _ptr(bias), _ptr(out), DTYPE_CODE[out.dtype], out.stride(0),
-        _ptr(dev_status), _stream(stream))
+    _check_weights(w_packed, N, K)
+    _same_device(x, R, w_packed, w_scale, bias, a_scale, dev_status)
+    _check_out(out, M, N, x)
+    with torch.cuda.device(x.device):
+        st = lib().ck_w4a4_linear_noalloc(
+            _ptr(x), DTYPE_CODE[x.dtype], M, K, x.stride(0), x.stride(1), _ptr(R), int(g),
+            _ptr(a_scale), _ptr(w_packed), N, w_packed.stride(0), _ptr(w_scale),
+            DTYPE_CODE[w_scale.dtype], _ptr(bias), _ptr(out), DTYPE_CODE[out.dtype],
+            out.stride(0), _ptr(dev_status), _stream(stream))
     _check(st, "ck_w4a4_linear_noalloc")
     return out
 
@@ -184,7 +223,12 @@ def ck_unpack_w4(packed: torch.Tensor, K: int, out: torch.Tensor | None = None,
     N = packed.shape[0]
     if out is None:
         out = torch.empty(N, K, dtype=torch.int8, device=packed.device)
-    st = lib().ck_unpack_w4(_ptr(packed), N, K, packed.stride(0), _ptr(out), out.stride(0),
-                            _stream(stream))
+    if packed.dim() != 2 or packed.stride(1) != 1 or packed.shape[1] < K // 2 or \
+            out.dim() != 2 or out.stride(1) != 1 or tuple(out.shape) != (N, K):
+        raise ValueError("ck_unpack_w4: packed must be (N, >= K/2) and out (N, K), unit inner strides")
+    _same_device(packed, out)
+    with torch.cuda.device(packed.device):
+        st = lib().ck_unpack_w4(_ptr(packed), N, K, packed.stride(0), _ptr(out), out.stride(0),
+                                _stream(stream))
     _check(st, "ck_unpack_w4")
     return out

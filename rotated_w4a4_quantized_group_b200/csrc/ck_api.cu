@@ -64,6 +64,20 @@ static int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 // The largest K for which |acc| <= 8 * 8 * K fits in int32.
 static constexpr int64_t kMaxK = 2147483647LL / 64;
 
+size_t linear_scratch_need(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                           int64_t stride_m, const int8_t* w_packed, int64_t N, int64_t w_ld) {
+    const bool codes_in = x_dtype == CK_I8;
+    const bool codes_aligned = codes_in && aligned(x, 16) && stride_m % 16 == 0;
+    const bool w_aligned = aligned(w_packed, 16) && w_ld % 16 == 0;
+    const int64_t P = K <= 0 ? 0 : round_up(K, 16);
+    const size_t scales_off = (size_t)round_up(M * P, 256);
+    const size_t wcopy_off = scales_off + (size_t)round_up(4 * M, 256);
+    size_t need = 0;
+    if (!codes_in || !codes_aligned) need = wcopy_off;
+    if (!w_aligned) need = wcopy_off + (size_t)round_up(N * round_up(K / 2, 16), 256);
+    return need;
+}
+
 }  // namespace ck
 
 using namespace ck;
@@ -148,9 +162,7 @@ ck_status ck_w4a4_linear(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
     const size_t wcopy_off = scales_off + (size_t)round_up(4 * M, 256);
     const bool codes_aligned = codes_in && aligned(x, 16) && stride_m % 16 == 0;
     const bool w_aligned = aligned(w_packed, 16) && w_ld % 16 == 0;
-    size_t need = 0;
-    if (!codes_in || !codes_aligned) need = wcopy_off;
-    if (!w_aligned) need = wcopy_off + (size_t)round_up(N * round_up(K / 2, 16), 256);
+    const size_t need = linear_scratch_need(x, x_dtype, M, K, stride_m, w_packed, N, w_ld);
     if (need) {
         if (!ws || workspace_bytes < need || !aligned(ws, 256)) return CK_ERR_WORKSPACE;
     }

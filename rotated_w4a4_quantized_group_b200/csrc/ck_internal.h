@@ -35,6 +35,13 @@ ck_status launch_w4a4_gemm(const int8_t* codes, int64_t ldq, const float* a_scal
 ck_status launch_unpack_w4(const int8_t* packed, int64_t N, int64_t K, int64_t ld_packed,
                            int8_t* out, int64_t ld_out, cudaStream_t stream);
 
+// Scratch bytes one ck_w4a4_linear call needs (0 when it needs none): the stage-1 codes and
+// row scales for floating-point input, or a 16-byte-pitched copy of int8 codes whose rows are
+// not 16-byte aligned, then (offset past them) a 16-byte-pitched copy of packed weights that
+// are not 16-byte aligned and pitched.  Arguments as in ck_w4a4_linear, already validated.
+size_t linear_scratch_need(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                           int64_t stride_m, const int8_t* w_packed, int64_t N, int64_t w_ld);
+
 // Copy a (rows, cols) byte matrix between pitches (used to re-pitch misaligned inputs).
 ck_status launch_copy_rows(const int8_t* src, int64_t ld_src, int8_t* dst, int64_t ld_dst,
                            int64_t rows, int64_t cols, cudaStream_t stream);

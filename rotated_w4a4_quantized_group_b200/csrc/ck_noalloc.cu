@@ -8,12 +8,14 @@
 // cudaMalloc (which may synchronise the device).  This entry point uses a scratch array
 // compiled into the library instead: a file-scope __device__ array of kNoAllocScratchBytes,
 // which every GPU that loads the library holds until the process exits.
+#include <cuda.h>
 #include <cuda_runtime_api.h>
 #include <stdint.h>
 
 #include <mutex>
 
 #include "ck.h"
+#include "ck_internal.h"
 
 namespace ck {
 
@@ -27,19 +29,53 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void* g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if the driver cannot say).  A device
+// reset ends the context and reloads the module, which may move the array; the new context has
+// a new id, so an address cached under the old one is looked up again.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_ctx = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_ctx = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_ctx && get_id && get_ctx(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, &id) == CUDA_SUCCESS)
+        return id;
+    return 0;
+}
 }  // namespace
 
 // Device address of the scratch array on the current device.  In host code the array's name
-// is only a host-side stand-in, so the address is looked up once per device (with that
-// device current) and cached.
+// is only a host-side stand-in, so the address is looked up (with that device current) once
+// per device and context, and cached.
 static ck_status scratch_address(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CK_ERR_CUDA;
+    unsigned long long ctx = current_context_id();
+    if (ctx == 0) {   // no context current yet: make the device's primary context current
+        if (cudaSetDevice(dev) != cudaSuccess) return CK_ERR_CUDA;
+        ctx = current_context_id();
+    }
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_addr[dev]) {
+    if (!g_scratch_addr[dev] || g_scratch_ctx[dev] != ctx) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return CK_ERR_CUDA;
         g_scratch_addr[dev] = p;
+        g_scratch_ctx[dev] = ctx;
     }
     *out = g_scratch_addr[dev];
     return CK_OK;
@@ -54,13 +90,13 @@ extern "C" ck_status ck_w4a4_linear_noalloc(const void* x, ck_dtype x_dtype, int
                                             const void* w_scale, ck_dtype scale_dtype,
                                             const void* bias, void* out, ck_dtype out_dtype,
                                             int64_t ldo, int* dev_status, cudaStream_t stream) {
-    // scratch is used for the stage-1 result of activation input, for int8 codes whose rows
-    // are not 16-byte aligned, and for weight rows that are not 16-byte pitched
-    const bool codes_direct = x_dtype == CK_I8 && (reinterpret_cast<uintptr_t>(x) % 16) == 0 &&
-                              stride_m % 16 == 0;
-    const bool w_direct = (reinterpret_cast<uintptr_t>(w_packed) % 16) == 0 && w_ld % 16 == 0;
-    const size_t need = (codes_direct && w_direct) ? 0 : ck_w4a4_linear_workspace_bytes(M, N, K, w_ld);
-    if (need > ck::kNoAllocScratchBytes) return CK_ERR_WORKSPACE;
+    // the same scratch calculation ck_w4a4_linear enforces (pointer alignments included);
+    // sizes it would reject are passed on for it to reject
+    if (M > 0 && N > 0 && K > 0 && K % 2 == 0 && w_ld >= K / 2) {
+        const size_t need =
+            ck::linear_scratch_need(x, x_dtype, M, K, stride_m, w_packed, N, w_ld);
+        if (need > ck::kNoAllocScratchBytes) return CK_ERR_WORKSPACE;
+    }
     void* scratch = nullptr;
     if (M > 0 && N > 0) {
         const ck_status st = ck::scratch_address(&scratch);

@@ -13,8 +13,8 @@ import pytest
 import torch
 
 import oracle
-from parity_util import (assert_close, compare_stage1, oracle_on_codes, sample_cols, sample_rows,
-                         to_device, workspace_stage1)
+from parity_util import (assert_close, compare_stage1, mismatch_widening, oracle_on_codes,
+                         sample_cols, sample_rows, to_device, workspace_stage1)
 from rotated_w4a4_quantized_group_b200 import ck
 from rotated_w4a4_quantized_group_b200 import workloads as W
 
@@ -61,7 +61,7 @@ def _check_linear(case, rows, cols):
     # full oracle on the sampled rows / columns
     ref, oc, os_ = oracle.linear(inp["x"], inp["R"], case.g, inp["w_packed"], inp["w_scale"],
                                  inp["bias"], rows=rows, cols=cols)
-    compare_stage1(gc, gs, oc, os_, dtype, case.name, case.g)
+    compare_stage1(gc, gs, oc, os_, dtype, case.name, case.g, x=inp["x"], R=inp["R"], rows=rows)
     got = out.cpu()[torch.from_numpy(rows)][:, torch.from_numpy(cols)]
     # bit-exact: the oracle's unpack + GEMM + epilogue on the GPU's own codes and scales
     exact = oracle_on_codes(gc, gs, inp["w_packed"], case.K, cols, inp["w_scale"], inp["bias"],
@@ -69,11 +69,11 @@ def _check_linear(case, rows, cols):
     assert torch.equal(got.view(torch.int16 if dtype != torch.float32 else torch.int32),
                        exact.view(torch.int16 if dtype != torch.float32 else torch.int32)), \
         f"{case.name}: output differs from oracle GEMM+epilogue on identical codes"
-    # tolerance against the whole oracle path, on rows whose codes agree with the oracle
-    same = (gc == oc).all(axis=1)
-    assert same.mean() >= 0.9
-    b = None if inp["bias"] is None else inp["bias"][torch.from_numpy(cols)]
-    assert_close(got[torch.from_numpy(same)], ref[torch.from_numpy(same)], dtype, case.name, b)
+    # tolerance against the whole oracle path on every sampled output; a row whose codes
+    # differ from the oracle's at ties gets its bound widened by those codes' effect
+    extra = mismatch_widening(gc, oc, os_, inp["w_packed"], case.K, cols, inp["w_scale"])
+    assert_close(got, ref, dtype, case.name, extra)
+    return gc, oc
 
 
 # ------------------------------------------------------------------- weight unpack
@@ -112,7 +112,7 @@ def _rq_case(case: W.RotateCase, rows=None):
     oc, os_ = oracle.rotate_quant(inp["x"], inp["R"], case.g, rows=rows)
     idx = torch.from_numpy(rows).cuda()
     return compare_stage1(codes[idx].cpu().numpy(), scales[idx].cpu().numpy(), oc, os_,
-                          DT[case.dtype], case.name, case.g)
+                          DT[case.dtype], case.name, case.g, x=inp["x"], R=inp["R"], rows=rows)
 
 
 @pytest.mark.parametrize("case", W.sweep_cases(), ids=lambda c: c.name)
@@ -132,7 +132,8 @@ def test_rotate_quant_small_every_row(dt, g, layout):
     codes, scales = ck.ck_rotate_quant(to_device(x), inp["R"].cuda(), g)
     torch.cuda.synchronize()
     oc, os_ = oracle.rotate_quant(x, inp["R"], g)
-    compare_stage1(codes.cpu().numpy(), scales.cpu().numpy(), oc, os_, DT[dt], case.name, g)
+    compare_stage1(codes.cpu().numpy(), scales.cpu().numpy(), oc, os_, DT[dt], case.name, g,
+                   x=x, R=inp["R"])
 
 
 @pytest.mark.parametrize("dt", ["f16", "bf16"])
@@ -152,7 +153,8 @@ def test_rotate_quant_tile_shapes(dt, g, groups, M):
     codes, scales = ck.ck_rotate_quant(to_device(x), R.cuda(), g)
     torch.cuda.synchronize()
     oc, os_ = oracle.rotate_quant(x, R, g)
-    compare_stage1(codes.cpu().numpy(), scales.cpu().numpy(), oc, os_, DT[dt], case.name, g)
+    compare_stage1(codes.cpu().numpy(), scales.cpu().numpy(), oc, os_, DT[dt], case.name, g,
+                   x=x, R=R)
 
 
 @pytest.mark.parametrize("dt", ["f16", "bf16"])
@@ -167,7 +169,8 @@ def test_rotate_quant_long_rows(dt, g, K):
     codes, scales = ck.ck_rotate_quant(to_device(x), R.cuda(), g)
     torch.cuda.synchronize()
     oc, os_ = oracle.rotate_quant(x, R, g)
-    compare_stage1(codes.cpu().numpy(), scales.cpu().numpy(), oc, os_, DT[dt], case.name, g)
+    compare_stage1(codes.cpu().numpy(), scales.cpu().numpy(), oc, os_, DT[dt], case.name, g,
+                   x=x, R=R)
 
 
 @pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
@@ -185,7 +188,8 @@ def test_rotate_quant_zero_rows_and_caller_zero_scale(dt):
     torch.cuda.synchronize()
     oc, os_ = oracle.rotate_quant(x, R, 64, scale_in=0.0)
     np.testing.assert_array_equal(scales0.cpu().numpy(), os_)
-    compare_stage1(codes0.cpu().numpy(), scales0.cpu().numpy(), oc, os_, DT[dt], "zero scale", 64)
+    compare_stage1(codes0.cpu().numpy(), scales0.cpu().numpy(), oc, os_, DT[dt], "zero scale", 64,
+                   x=x, R=R, scale_in=0.0)
 
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
@@ -201,7 +205,8 @@ def test_rotate_quant_non_finite_follows_the_oracle_convention(dt):
     assert math.isnan(gs[1]) and math.isnan(os_[1])
     assert math.isinf(gs[2]) and math.isinf(os_[2])
     np.testing.assert_array_equal(codes.cpu().numpy()[1:3], oc[1:3])
-    compare_stage1(codes.cpu().numpy()[[0, 3]], gs[[0, 3]], oc[[0, 3]], os_[[0, 3]], DT[dt], "", 16)
+    compare_stage1(codes.cpu().numpy()[[0, 3]], gs[[0, 3]], oc[[0, 3]], os_[[0, 3]], DT[dt], "", 16,
+                   x=x, R=R, rows=[0, 3])
 
 
 def test_rotate_quant_unaligned_and_strided_views():
@@ -212,7 +217,8 @@ def test_rotate_quant_unaligned_and_strided_views():
     codes, scales = ck.ck_rotate_quant(to_device(x), R.cuda(), 64, codes=codes_buf[:, 3:131])
     torch.cuda.synchronize()
     oc, os_ = oracle.rotate_quant(x, R, 64)
-    compare_stage1(codes.cpu().numpy(), scales.cpu().numpy(), oc, os_, torch.bfloat16, "", 64)
+    compare_stage1(codes.cpu().numpy(), scales.cpu().numpy(), oc, os_, torch.bfloat16, "", 64,
+                   x=x, R=R)
     assert (codes_buf[:, :3] == 55).all() and (codes_buf[:, 131:] == 55).all()
 
 
