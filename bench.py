@@ -11,8 +11,10 @@ launches from activations) so each kernel's duration is measured with CUDA event
 
 Rank 0 prints one JSON line.  With N > 1 (torchrun) every rank runs its own replica of
 the workload (the path has no exchange step): weak scaling, max device time over ranks.
-`--impl reference` times the CPU oracle (test infrastructure, plain single-threaded C) on
-a bounded sample of the same workload.
+`--impl reference` times the CPU oracle (test infrastructure, plain single-threaded C, its
+rows spread over the host's cores by threads) on a bounded sample of the same workload.
+`--sweep` times stage 1 alone on the 72 rotate+quantize cases (M x K x g x dtype x layout)
+and prints one JSON object with a line per case (microseconds, GB/s, fraction of HBM).
 """
 from __future__ import annotations
 
@@ -58,22 +60,34 @@ def source_sha(path: str) -> str:
 
 
 def recorded_traffic(kernel_file: str, workload: str):
-    """DRAM bytes per launch recorded (profiles/traffic.md) from an ncu capture of this exact
+    """DRAM bytes per launch recorded in profiles/traffic.json from an ncu capture of this exact
     kernel source; None when no row matches the current source."""
-    p = os.path.join(ROOT, "profiles", "traffic.md")
+    p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     sha = source_sha(kernel_file)
     name = os.path.basename(kernel_file)
     with open(p) as f:
-        for line in f:
-            cells = [c.strip() for c in line.strip().strip("|").split("|")]
-            if len(cells) >= 4 and cells[0] == name and cells[1] == workload and cells[2] == sha:
-                try:
-                    return int(cells[3])
-                except ValueError:
-                    return None
+        rows = json.load(f).get("rows", [])
+    for r in rows:
+        if r.get("kernel_file") == name and r.get("workload") == workload and \
+                r.get("source_sha16") == sha:
+            try:
+                return int(r["dram_bytes_per_launch"])
+            except (KeyError, TypeError, ValueError):
+                return None
     return None
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 class ClockSampler:
@@ -187,52 +201,167 @@ def barrier(world: int):
 
 # ----------------------------------------------------------------------------- oracle (CPU)
 
-def oracle_sample(case, inp, budget_s: float):
-    """Time the CPU oracle on the first rows of the workload (all N output channels), sized
-    so that it takes about budget_s seconds.  Returns (ops/s, rows, seconds)."""
-    import oracle  # test infrastructure: only this CPU-baseline leg uses it
+def host_cores() -> list[int]:
+    try:
+        return sorted(os.sched_getaffinity(0))
+    except AttributeError:
+        return list(range(os.cpu_count() or 1))
+
+
+def _run_threads(fn, parts):
+    """Call fn(part) for every part on its own thread.  The oracle is called through ctypes,
+    which releases the interpreter lock, so the threads run on separate cores."""
+    ts = [threading.Thread(target=fn, args=(pt,)) for pt in parts]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+
+
+def oracle_linear_sample(case, inp, budget_s: float, threads: int, pin_core: int | None = None):
+    """Time the CPU oracle's whole linear (stage 1, unpack, GEMM, epilogue) on the first rows
+    of the workload, all N output channels, with the rows split over `threads` threads, sized
+    to about budget_s seconds.  With pin_core the process runs on that one core.  Returns
+    (ops per second, rows, seconds)."""
+    import oracle  # test infrastructure: only the CPU-baseline and reference legs use it
     oracle.lib()
-    rows = 1
-    t0 = time.perf_counter()
-    oracle.linear(inp["x"], inp["R"], case.g, inp["w_packed"], inp["w_scale"], inp["bias"],
-                  rows=list(range(rows)))
-    dt = time.perf_counter() - t0
-    rows = max(1, min(case.M, int(budget_s / max(dt, 1e-6))))
-    t0 = time.perf_counter()
-    oracle.linear(inp["x"], inp["R"], case.g, inp["w_packed"], inp["w_scale"], inp["bias"],
-                  rows=list(range(rows)))
-    dt = time.perf_counter() - t0
+    saved = host_cores()
+    if pin_core is not None:
+        os.sched_setaffinity(0, {pin_core})
+    try:
+        def run(rows):
+            parts = [rows[i::threads] for i in range(threads)]
+            parts = [p for p in parts if p]
+            _run_threads(lambda pr: oracle.linear(inp["x"], inp["R"], case.g, inp["w_packed"],
+                                                  inp["w_scale"], inp["bias"], rows=pr), parts)
+        t0 = time.perf_counter()
+        run(list(range(min(threads, case.M))))
+        dt = time.perf_counter() - t0
+        per_row = dt / min(threads, case.M) * threads      # seconds per row per thread
+        rows = max(1, min(case.M, int(budget_s * threads / max(per_row, 1e-6))))
+        t0 = time.perf_counter()
+        run(list(range(rows)))
+        dt = time.perf_counter() - t0
+    finally:
+        if pin_core is not None:
+            os.sched_setaffinity(0, set(saved))
     return 2.0 * rows * case.N * case.K / dt, rows, dt
+
+
+def oracle_stage1_sample(case, inp, budget_s: float, threads: int, pin_core: int | None = None):
+    """Time the CPU oracle's stage 1 (rotate + quantize) on the first rows; returns (bytes per
+    second of the stage's algorithmic traffic, rows, seconds)."""
+    import oracle
+    oracle.lib()
+    saved = host_cores()
+    if pin_core is not None:
+        os.sched_setaffinity(0, {pin_core})
+    try:
+        def run(rows):
+            parts = [p for p in (rows[i::threads] for i in range(threads)) if p]
+            _run_threads(lambda pr: oracle.rotate_quant(inp["x"], inp["R"], case.g, rows=pr), parts)
+        t0 = time.perf_counter()
+        run(list(range(min(threads, case.M))))
+        per_row = (time.perf_counter() - t0) / min(threads, case.M) * threads
+        rows = max(1, min(case.M, int(budget_s * threads / max(per_row, 1e-6))))
+        t0 = time.perf_counter()
+        run(list(range(rows)))
+        dt = time.perf_counter() - t0
+    finally:
+        if pin_core is not None:
+            os.sched_setaffinity(0, set(saved))
+    per_row_bytes = W.algorithmic_bytes_rotate_quant(1, case.K, case.g, case.dtype) - \
+        case.g * case.g * W.ELEM_BYTES[case.dtype]
+    return per_row_bytes * rows / dt, rows, dt
+
+
+def cpu_baseline(case, inp, budget_s: float):
+    """The oracle as it stands on the host: the whole linear on all cores (rows split across
+    threads) and on one pinned core, and stage 1 alone in GB/s on all cores."""
+    cores = host_cores()
+    n = len(cores)
+    v_all, rows_all, dt_all = oracle_linear_sample(case, inp, budget_s, n)
+    v_one, rows_one, dt_one = oracle_linear_sample(case, inp, budget_s / 2, 1, pin_core=cores[0])
+    b_all, rows_s1, dt_s1 = oracle_stage1_sample(case, inp, budget_s / 3, n)
+    return {
+        "value": v_all / 1e12, "unit": UNIT, "cores": n, "kind": "oracle",
+        "sample": (f"oracle linear on the first {rows_all} of {case.M} rows x all {case.N} output "
+                   f"channels ({dt_all:.1f} s), rows split over {n} threads on {n} cores"),
+        "cpu_model": cpu_model(), "hardware_concurrency": os.cpu_count(),
+        "single_core_pinned": {"value": v_one / 1e12, "unit": UNIT, "cores": 1,
+                               "core": cores[0], "rows": rows_one, "seconds": dt_one},
+        "stage1": {"value": b_all / 1e9, "unit": "GB/s", "cores": n, "rows": rows_s1,
+                   "seconds": dt_s1},
+    }
 
 
 # ----------------------------------------------------------------------------- arms
 
+def config_of(case, world: int) -> dict:
+    """The workload description both arms print (identical for the same case)."""
+    return {"workload": case.name, "M": case.M, "K": case.K, "N": case.N, "g": case.g,
+            "x_dtype": case.dtype, "rotation": case.rotation, "layout": case.layout,
+            "l2": "GPU arm: flushed (512 MiB write) before every step, outside the timed events",
+            "parallelism": f"replicas x{world}"}
+
+
 def run_reference(args, case, world, rank):
+    """The oracle, as it stands, on the host's cores: each step is a bounded sample of the
+    workload's rows (all output channels), timed by the wall clock."""
     if rank != 0:
         return None
     inp = W.make_linear_inputs(case)
-    vals = []
-    rows_used = 0
+    cores = host_cores()
     per_step = max(0.05, min(args.cpu_budget, 120.0 / max(1, args.steps + args.warmup)))
+    vals, times, rows_used = [], [], 0
     for i in range(args.warmup + args.steps):
-        v, rows, dt = oracle_sample(case, inp, per_step)
+        v, rows, dt = oracle_linear_sample(case, inp, per_step, len(cores))
         if i >= args.warmup:
             vals.append(v)
+            times.append(dt)
             rows_used = rows
     value = statistics.mean(vals) / 1e12
-    ms = 2.0 * case.M * case.N * case.K / (value * 1e12) * 1e3
     sample = (f"oracle linear on the first {rows_used} of {case.M} rows x all {case.N} output "
-              f"channels per step (stage 1 + unpack + GEMM + epilogue), single-threaded C")
+              f"channels per step (stage 1 + unpack + GEMM + epilogue), rows split over "
+              f"{len(cores)} threads")
     return {
         "metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
-        "config": {"workload": case.name, "M": case.M, "K": case.K, "N": case.N, "g": case.g,
-                   "x_dtype": case.dtype},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": sample},
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(times) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8",
+        "data": "synthetic", "config": config_of(case, args.gpus),
+        "sample_rows_per_step": rows_used,
+        "full_step_ms_extrapolated": 2.0 * case.M * case.N * case.K / (value * 1e12) * 1e3,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": len(cores), "kind": "oracle",
+                         "sample": sample, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+
+
+def gemm_roofline(M, N, K, case, gemm_ms, pk, pk_kind, sm_mhz, traffic):
+    """Roofline of the GEMM launch: tensor-bound when its operation intensity is above the
+    ridge (INT8 peak / HBM bandwidth), HBM-bound below it (small M)."""
+    ops = 2.0 * M * N * K
+    nbytes = W.algorithmic_bytes_gemm(M, K, N, case.dtype, case.has_bias)
+    int8_peak = pk["bf16_tflops"] * INT8_OVER_BF16
+    ridge = int8_peak * 1e12 / (pk["hbm_gbs"] * 1e9)
+    mma_rate = None
+    if sm_mhz:
+        # tcgen05.mma kind::i8 issues 8192 MACs per clock per SM (148 SMs)
+        mma_rate = 148 * 8192 * 2 * sm_mhz * 1e6 / 1e12
+    if ops / nbytes >= ridge:
+        achieved = ops / (gemm_ms * 1e-3) / 1e12
+        r = {"bound": "tensor", "kernel": "w4a4_gemm_kernel", "achieved": achieved,
+             "peak": int8_peak, "unit": "TOPS", "frac": achieved / int8_peak, "traffic": traffic,
+             "peak_source": f"{pk_kind} bf16 burst x {INT8_OVER_BF16} (INT8:BF16 nominal)"}
+        if mma_rate:
+            r["frac_of_kind_i8_rate"] = achieved / mma_rate
+            r["kind_i8_rate_tops"] = mma_rate
+        return r
+    achieved = nbytes / (gemm_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": "w4a4_gemm_kernel", "achieved": achieved,
+            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+            "traffic": traffic, "algorithmic_bytes": nbytes,
+            "tops": ops / (gemm_ms * 1e-3) / 1e12, "peak_source": f"{pk_kind} HBM copy"}
 
 
 def run_ck(args, case, world, rank, local):
@@ -241,7 +370,10 @@ def run_ck(args, case, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     inp = W.make_linear_inputs(case)
-    x = inp["x"].to(dev)
+    if case.layout == "colmajor":       # keep the column-major layout on the device
+        x = inp["x"].t().contiguous().to(dev).t()
+    else:
+        x = inp["x"].contiguous().to(dev)
     R = inp["R"].to(dev)
     wp = inp["w_packed"].to(dev)
     wsc = inp["w_scale"].to(dev)
@@ -272,6 +404,14 @@ def run_ck(args, case, world, rank, local):
 
     evs = []
     with ClockSampler(local) as clk:
+        # clock soak: back-to-back steps for about a second under the sampler, so the clock
+        # record covers the same load the timed steps see (untimed, before them)
+        t_soak = time.perf_counter()
+        while time.perf_counter() - t_soak < args.clock_soak_s:
+            for _ in range(20):
+                flush.zero_()
+                step()
+            torch.cuda.synchronize()
         barrier(world)
         t_wall = time.perf_counter()
         for _ in range(args.steps):
@@ -295,20 +435,20 @@ def run_ck(args, case, world, rank, local):
     value = flops * world / (ms_per_step * 1e-3) / 1e12
 
     pk, pk_kind = peaks()
-    int8_peak = pk["bf16_tflops"] * INT8_OVER_BF16
     gemm_ms = statistics.mean(gemm)
     s1_ms = statistics.mean(stage1)
-    achieved = flops / (gemm_ms * 1e-3) / 1e12
     s1_bytes = W.algorithmic_bytes_rotate_quant(M, K, g, case.dtype)
     s1_gbs = s1_bytes / (s1_ms * 1e-3) / 1e9
     gemm_file = os.path.join(ROOT, "rotated_w4a4_quantized_group_b200", "csrc", "ck_w4a4_gemm.cu")
-    traffic = recorded_traffic(gemm_file, case.name)
+    rq_file = os.path.join(ROOT, "rotated_w4a4_quantized_group_b200", "csrc", "ck_rotate_quant.cu")
+    clocks = clk.summary()
+    roof = gemm_roofline(M, N, K, case, gemm_ms, pk, pk_kind, clocks.get("sm_mhz"),
+                         recorded_traffic(gemm_file, case.name))
 
     # ---- end to end through the public call with host buffers (pinned), copies timed
-    xh = torch.empty_like(inp["x"], device="cpu").pin_memory() if inp["x"].is_contiguous() \
-        else inp["x"].contiguous().pin_memory()
-    xh.copy_(inp["x"])
-    xd = torch.empty_like(xh, device=dev)
+    xh = inp["x"].contiguous().pin_memory() if case.layout != "colmajor" else \
+        inp["x"].t().contiguous().pin_memory().t()
+    xd = x.clone() if case.layout != "colmajor" else x.t().clone().t()
     oh = torch.empty(M, N, dtype=out.dtype).pin_memory()
     e2e_steps = max(3, min(args.steps, 20))
     for i in range(2 + e2e_steps):
@@ -332,29 +472,75 @@ def run_ck(args, case, world, rank, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
-        "config": {"workload": case.name, "M": M, "K": K, "N": N, "g": g, "x_dtype": case.dtype,
-                   "rotation": case.rotation, "l2": "flushed (512 MiB write) before every step, "
-                   "outside the timed events", "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "tensor", "kernel": "w4a4_gemm_kernel", "achieved": achieved,
-                     "peak": int8_peak, "unit": "TOPS", "frac": achieved / int8_peak,
-                     "traffic": traffic,
-                     "peak_source": f"{pk_kind} bf16 burst x {INT8_OVER_BF16} (INT8:BF16 nominal)"},
+        "config": config_of(case, world),
+        "roofline": roof,
         "stage1": {"kernel": "rotate_quant", "ms": s1_ms, "algorithmic_bytes": s1_bytes,
-                   "gbs": s1_gbs, "hbm_peak_gbs": pk["hbm_gbs"], "frac": s1_gbs / pk["hbm_gbs"]},
+                   "gbs": s1_gbs, "hbm_peak_gbs": pk["hbm_gbs"], "frac": s1_gbs / pk["hbm_gbs"],
+                   "traffic": recorded_traffic(rq_file, case.name)},
         "gemm_ms": gemm_ms,
         "e2e": {"value": e2e_val, "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": xh.numel() * xh.element_size(),
                 "d2h_bytes_per_step": oh.numel() * oh.element_size()},
         "gpu_launches": 2 * args.steps,
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "wall_s_timed_region": t_wall,
     }
     if not args.no_cpu_baseline and world == 1:
-        v, rows, dt = oracle_sample(case, inp, args.cpu_budget)
-        res["cpu_baseline"] = {"value": v / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
-                               "sample": f"oracle linear on the first {rows} of {M} rows x all "
-                                         f"{N} output channels ({dt:.1f} s, single-threaded C)"}
+        res["cpu_baseline"] = cpu_baseline(case, inp, args.cpu_budget)
     return res
+
+
+def run_sweep(args, local):
+    """Stage 1 alone on the 72 rotate+quantize cases: median event time over the timed
+    iterations (L2 flushed before each, outside the events), GB/s of the algorithmic bytes."""
+    from rotated_w4a4_quantized_group_b200 import ck
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pk, pk_kind = peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = []
+    for case in W.sweep_cases():
+        if args.sweep_filter and args.sweep_filter not in case.name:
+            continue
+        inp = W.make_rotate_inputs(case)
+        xc = inp["x"]
+        if case.layout == "pitch2k":
+            buf = torch.zeros(case.M, 2 * case.K, dtype=xc.dtype, device=dev)
+            buf[:, :case.K] = xc.to(dev)
+            x = buf[:, :case.K]
+        else:
+            x = xc.to(dev)
+        R = inp["R"].to(dev)
+        codes = torch.empty(case.M, case.K, dtype=torch.int8, device=dev)
+        scales = torch.empty(case.M, dtype=torch.float32, device=dev)
+        for _ in range(3):
+            ck.ck_rotate_quant(x, R, case.g, codes=codes, scales=scales, dev_status=status)
+        ts = []
+        for _ in range(args.steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            ck.ck_rotate_quant(x, R, case.g, codes=codes, scales=scales, dev_status=status,
+                               stream=stream)
+            e1.record(stream)
+            ts.append((e0, e1))
+        torch.cuda.synchronize()
+        ms = statistics.median(a.elapsed_time(b) for a, b in ts)
+        nbytes = W.algorithmic_bytes_rotate_quant(case.M, case.K, case.g, case.dtype)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out.append({"case": case.name, "us": ms * 1e3, "algorithmic_bytes": nbytes, "gbs": gbs,
+                    "frac_hbm": gbs / pk["hbm_gbs"]})
+        del x, codes, scales
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()}")
+    return {"sweep": "rotate+quantize, stage 1 alone", "unit": "GB/s", "steps": args.steps,
+            "hbm_peak_gbs": pk["hbm_gbs"], "peak_source": f"{pk_kind} HBM copy",
+            "l2": "flushed (512 MiB write) before every timed launch, outside the events",
+            "cases": out}
 
 
 def main():
@@ -364,8 +550,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ck", choices=["ck", "reference"])
     ap.add_argument("--workload", default=W.HEADLINE, choices=list(W.LINEAR_CASES))
-    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-soak-s", type=float, default=1.0)
+    ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--sweep-filter", default="")
     args = ap.parse_args()
     case = W.LINEAR_CASES[args.workload]
 
@@ -378,6 +567,10 @@ def main():
 
     world, rank, local = dist_setup()
     try:
+        if args.sweep:
+            if rank == 0:
+                print(json.dumps(run_sweep(args, local)), flush=True)
+            return
         res = run_ck(args, case, world, rank, local)
         if res is not None:
             print(json.dumps(res), flush=True)

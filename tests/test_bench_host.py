@@ -1,8 +1,10 @@
 """Host-side helpers of bench.py, on CPU: the per-launch DRAM traffic lookup keyed by kernel
-source, and the clock sampler's summary (the bench rejects runs with thermal or hardware
-slowdowns, so the reasons it reports must be exact)."""
+source, the clock sampler's summary (the bench rejects runs with thermal or hardware
+slowdowns, so the reasons it reports must be exact), the workload description both arms
+print, the roofline bound chosen per workload, and the CPU baseline's structure."""
 from __future__ import annotations
 
+import json
 import os
 import sys
 
@@ -10,6 +12,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
 import bench  # noqa: E402
+from rotated_w4a4_quantized_group_b200 import workloads as W  # noqa: E402
 
 
 def _fake_tree(tmp_path, kernel_src: bytes):
@@ -19,12 +22,18 @@ def _fake_tree(tmp_path, kernel_src: bytes):
     return str(k)
 
 
+def _table(tmp_path, rows):
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"rows": rows}))
+
+
 def test_traffic_is_read_only_for_the_captured_source(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     k = _fake_tree(tmp_path, b"kernel v1")
     sha = bench.source_sha(k)
-    (tmp_path / "profiles" / "traffic.md").write_text(
-        "| kern.cu | wl | %s | 1234 |\n| kern.cu | other | %s | 99 |\n" % (sha, sha))
+    _table(tmp_path, [{"kernel_file": "kern.cu", "workload": "wl", "source_sha16": sha,
+                       "dram_bytes_per_launch": 1234},
+                      {"kernel_file": "kern.cu", "workload": "other", "source_sha16": sha,
+                       "dram_bytes_per_launch": 99}])
     assert bench.recorded_traffic(k, "wl") == 1234
     assert bench.recorded_traffic(k, "other") == 99
     assert bench.recorded_traffic(k, "missing") is None
@@ -40,14 +49,44 @@ def test_traffic_without_a_table_is_none(tmp_path, monkeypatch):
     assert bench.recorded_traffic(str(k), "wl") is None
 
 
-def test_committed_traffic_row_parses():
-    """The committed table has a well-formed row for the GEMM on the headline workload."""
-    rows = [l for l in open(os.path.join(ROOT, "profiles", "traffic.md"))
-            if l.startswith("| ck_w4a4_gemm.cu")]
-    assert rows
-    cells = [c.strip() for c in rows[0].strip().strip("|").split("|")]
-    assert cells[1] == "zimage_m8192_k3840_n3840_g64_bf16"
-    assert len(cells[2]) == 16 and int(cells[3]) > 0
+def test_committed_traffic_rows_parse():
+    """Every committed row names a kernel source file of the package and a known workload."""
+    d = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    assert d["rows"]
+    csrc = os.path.join(ROOT, "rotated_w4a4_quantized_group_b200", "csrc")
+    for r in d["rows"]:
+        assert os.path.exists(os.path.join(csrc, r["kernel_file"]))
+        assert len(r["source_sha16"]) == 16 and int(r["dram_bytes_per_launch"]) > 0
+        assert r["command"]
+
+
+def test_both_arms_print_the_same_config():
+    case = W.LINEAR_CASES[W.HEADLINE]
+    assert bench.config_of(case, 1) == bench.config_of(case, 1)
+    assert bench.config_of(case, 2)["parallelism"] == "replicas x2"
+    assert bench.config_of(case, 1)["workload"] == case.name
+
+
+def test_roofline_bound_follows_operation_intensity():
+    pk = {"hbm_gbs": 6550.0, "bf16_tflops": 1640.0}
+    small = W.LINEAR_CASES["zimage_m32_k3840_n3840_g64_bf16"]
+    big = W.LINEAR_CASES[W.HEADLINE]
+    r0 = bench.gemm_roofline(small.M, small.N, small.K, small, 0.01, pk, "measured", 1965.0, None)
+    assert r0["bound"] == "hbm" and r0["unit"] == "GB/s"
+    assert abs(r0["achieved"] - r0["algorithmic_bytes"] / 1e-5 / 1e9) < 1e-6 * r0["achieved"]
+    r1 = bench.gemm_roofline(big.M, big.N, big.K, big, 0.1, pk, "measured", 1965.0, None)
+    assert r1["bound"] == "tensor" and r1["peak"] == 3280.0
+    assert abs(r1["kind_i8_rate_tops"] - 148 * 8192 * 2 * 1.965e9 / 1e12) < 1e-6
+
+
+def test_cpu_baseline_reports_all_cores_pinned_core_and_stage1():
+    case = W.LINEAR_CASES["zimage_m32_k3840_n3840_g64_bf16"].replace(N=64)
+    inp = W.make_linear_inputs(case)
+    cb = bench.cpu_baseline(case, inp, 0.2)
+    assert cb["kind"] == "oracle" and cb["cores"] == len(bench.host_cores())
+    assert cb["value"] > 0 and cb["single_core_pinned"]["cores"] == 1
+    assert cb["stage1"]["unit"] == "GB/s" and cb["stage1"]["value"] > 0
+    assert cb["cpu_model"] and cb["hardware_concurrency"] >= 1
 
 
 def test_clock_summary_reports_median_and_every_reason():
