@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from parity_util import (assert_close, compare_stage1, mismatch_widening, oracle_on_codes,
+from parity_util import (assert_close, compare_stage1, oracle_on_codes, output_widening,
                          sample_cols, sample_rows, to_device, workspace_stage1)
 from rotated_w4a4_quantized_group_b200 import ck
 from rotated_w4a4_quantized_group_b200 import workloads as W
@@ -70,8 +70,9 @@ def _check_linear(case, rows, cols):
                        exact.view(torch.int16 if dtype != torch.float32 else torch.int32)), \
         f"{case.name}: output differs from oracle GEMM+epilogue on identical codes"
     # tolerance against the whole oracle path on every sampled output; a row whose codes
-    # differ from the oracle's at ties gets its bound widened by those codes' effect
-    extra = mismatch_widening(gc, oc, os_, inp["w_packed"], case.K, cols, inp["w_scale"])
+    # differ from the oracle's at ties, or whose scale differs within its bound, gets its bound
+    # widened by exactly that difference's effect
+    extra = output_widening(gc, oc, gs, os_, inp["w_packed"], case.K, cols, inp["w_scale"])
     assert_close(got, ref, dtype, case.name, extra)
     return gc, oc
 

@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import oracle
-from parity_util import (assert_close, compare_stage1, mismatch_widening, oracle_on_codes,
+from parity_util import (assert_close, compare_stage1, oracle_on_codes, output_widening,
                          tie_distance_bound)
 from rotated_w4a4_quantized_group_b200 import workloads as W
 
@@ -114,9 +114,30 @@ def test_output_widening_covers_exactly_a_tie_flip(out_dt):
     gc[2, 17] += 1 if gc[2, 17] < 7 else -1
     got = oracle_on_codes(gc, os_, inp["w_packed"], case.K, cols, inp["w_scale"], inp["bias"],
                           out_dt)
-    extra = mismatch_widening(gc, oc, os_, inp["w_packed"], case.K, cols, inp["w_scale"])
+    extra = output_widening(gc, oc, os_, os_, inp["w_packed"], case.K, cols, inp["w_scale"])
     assert (extra[2] > 0).any() and not extra[[0, 1, 3, 4, 5]].any()
     assert_close(got, ref, out_dt, "widened", extra)
     if out_dt == torch.float32:
         with pytest.raises(AssertionError):
             assert_close(got, ref, out_dt, "plain")
+
+
+def test_output_widening_covers_a_scale_one_ulp_off():
+    """fp32 output with bias: a row scale one fp32 ulp from the oracle's (allowed for fp32
+    inputs) moves outputs by |acc| * ulp * |ws|.  Where acc * a * ws cancels against the bias
+    that exceeds rtol 1e-5 of |ref|; the widened bound accepts exactly that."""
+    case = W.LinearCase("ulp", M=8, K=512, N=300, g=16, dtype="f32", rotation="haar",
+                        bias_std=1.0, seed=31)
+    inp = W.make_linear_inputs(case)
+    rows, cols = np.arange(case.M), np.arange(case.N)
+    ref, oc, os_ = oracle.linear(inp["x"], inp["R"], case.g, inp["w_packed"], inp["w_scale"],
+                                 inp["bias"], rows=rows, cols=cols)
+    gs = os_.copy()
+    gs[3] = np.nextafter(gs[3], np.float32(np.inf))
+    got = oracle_on_codes(oc, gs, inp["w_packed"], case.K, cols, inp["w_scale"], inp["bias"],
+                          torch.float32)
+    extra = output_widening(oc, oc, gs, os_, inp["w_packed"], case.K, cols, inp["w_scale"])
+    assert not extra[[0, 1, 2, 4, 5, 6, 7]].any() and (extra[3] > 0).all()
+    assert_close(got, ref, torch.float32, "scale ulp", extra)
+    # the planted difference is real: some outputs of that row moved
+    assert (got[3] != ref[3]).any()
