@@ -337,3 +337,175 @@ done:
     free(q); free(s); free(wsel); free(acc); free(wsc); free(bsel);
     return rc;
 }
+
+/* ---------------------------------------------------------------- W8A8 variant */
+
+/* INT8 row-wise quantizer: the same steps as ck_oracle_quantize with the INT8 grid, qmax 127
+ * (PR #155, fused RotateQuant emitting INT8 codes). */
+int ck_oracle_quantize_int8(const double* y, int64_t nrows, int64_t K, const float* scale_in,
+                            int8_t* codes, float* scales) {
+    if (nrows < 0 || K <= 0) return -1;
+    for (int64_t r = 0; r < nrows; ++r) {
+        const double* row = y + r * K;
+        float s;
+        if (scale_in) {
+            s = *scale_in;
+        } else {
+            double amax = 0.0;
+            int has_nan = 0;
+            for (int64_t k = 0; k < K; ++k) {
+                if (isnan(row[k])) has_nan = 1;
+                else if (fabs(row[k]) > amax) amax = fabs(row[k]);
+            }
+            s = has_nan ? NAN : (float)amax / 127.0f;
+        }
+        if (s < FLT_MIN) s = FLT_MIN;
+        scales[r] = s;
+        for (int64_t k = 0; k < K; ++k) {
+            float t = (float)row[k] / s;
+            int8_t q;
+            if (isnan(t)) {
+                q = 0;
+            } else {
+                t = rintf(t);
+                if (t > 127.0f) t = 127.0f;
+                if (t < -128.0f) t = -128.0f;
+                q = (int8_t)t;
+            }
+            codes[r * K + k] = q;
+        }
+    }
+    return 0;
+}
+
+int ck_oracle_rotate_quant_int8(const void* x, int dtype, int64_t M, int64_t K,
+                                int64_t stride_m, int64_t stride_k, const void* R, int g,
+                                const float* scale_in, const int64_t* rows, int64_t nrows,
+                                int8_t* codes, float* scales) {
+    if (nrows < 0 || K <= 0) return -1;
+    if (nrows == 0) return 0;
+    double* y = (double*)malloc(sizeof(double) * (size_t)nrows * (size_t)K);
+    if (!y) return -3;
+    int rc = ck_oracle_rotate(x, dtype, M, K, stride_m, stride_k, R, g, rows, nrows, y);
+    if (rc == 0) rc = ck_oracle_quantize_int8(y, nrows, K, scale_in, codes, scales);
+    free(y);
+    return rc;
+}
+
+int ck_oracle_linear_w8a8(const void* x, int dtype, int64_t M, int64_t K, int64_t stride_m,
+                          int64_t stride_k, const void* R, int g, const int8_t* w, int64_t N,
+                          int64_t w_ld, const void* w_scale, const void* bias, int scale_dtype,
+                          int out_dtype, const int64_t* rows, int64_t nrows, const int64_t* cols,
+                          int64_t ncols, void* out, int8_t* codes, float* scales) {
+    if (nrows < 0 || ncols < 0 || K <= 0 || w_ld < K) return -1;
+    int rc = 0;
+    int8_t* q = (int8_t*)malloc((size_t)(nrows ? nrows : 1) * (size_t)K);
+    float* s = (float*)malloc(sizeof(float) * (size_t)(nrows ? nrows : 1));
+    int8_t* wsel = (int8_t*)malloc((size_t)(ncols ? ncols : 1) * (size_t)K);
+    int32_t* acc = (int32_t*)malloc(sizeof(int32_t) * (size_t)(nrows ? nrows : 1) *
+                                    (size_t)(ncols ? ncols : 1));
+    unsigned char* wsc = (unsigned char*)malloc(4 * (size_t)(ncols ? ncols : 1));
+    unsigned char* bsel = (unsigned char*)malloc(4 * (size_t)(ncols ? ncols : 1));
+    if (!q || !s || !wsel || !acc || !wsc || !bsel) { rc = -3; goto done; }
+    rc = ck_oracle_rotate_quant_int8(x, dtype, M, K, stride_m, stride_k, R, g, NULL, rows,
+                                     nrows, q, s);
+    if (rc) goto done;
+    int eb = scale_dtype == OR_F32 ? 4 : 2;
+    for (int64_t c = 0; c < ncols; ++c) {
+        int64_t n = cols[c];
+        if (n < 0 || n >= N) { rc = -1; goto done; }
+        memcpy(wsel + c * K, w + n * w_ld, (size_t)K);
+        memcpy(wsc + c * eb, (const char*)w_scale + n * eb, (size_t)eb);
+        if (bias) memcpy(bsel + c * eb, (const char*)bias + n * eb, (size_t)eb);
+    }
+    rc = ck_oracle_gemm_s32(q, nrows, wsel, ncols, K, acc);
+    if (rc) goto done;
+    rc = ck_oracle_epilogue(acc, nrows, ncols, s, wsc, bias ? bsel : NULL, scale_dtype, out,
+                            out_dtype);
+    if (rc) goto done;
+    if (codes) memcpy(codes, q, (size_t)nrows * (size_t)K);
+    if (scales) memcpy(scales, s, sizeof(float) * (size_t)nrows);
+done:
+    free(q); free(s); free(wsel); free(acc); free(wsc); free(bsel);
+    return rc;
+}
+
+/* ---------------------------------------------------------------- packed quantizer */
+
+/* Philox4x32-10 as published (Salmon et al., SC 2011): each round multiplies two counter
+ * words by the constants 0xD2511F53 and 0xCD9E8D57 into 64-bit products and mixes their high
+ * halves with the other two words and the key; the key is bumped by the Weyl constants
+ * 0x9E3779B9 and 0xBB67AE85 between rounds. */
+int ck_oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]) {
+    uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        const uint32_t n0 = hi1 ^ c1 ^ k0;
+        const uint32_t n1 = lo1;
+        const uint32_t n2 = hi0 ^ c3 ^ k1;
+        const uint32_t n3 = lo0;
+        c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+    return 0;
+}
+
+int ck_oracle_quantize_packed(const double* y, int64_t nrows, int64_t K, const float* scale_in,
+                              int rounding, uint64_t seed, uint64_t offset, const int64_t* rows,
+                              uint8_t* packed, float* scales) {
+    if (nrows < 0 || K <= 0 || K % 2 || (rounding != 0 && rounding != 1) || !rows) return -1;
+    int8_t* q = (int8_t*)malloc((size_t)(K ? K : 1));
+    if (!q) return -3;
+    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    for (int64_t r = 0; r < nrows; ++r) {
+        const double* row = y + r * K;
+        float s;
+        if (scale_in) {
+            s = *scale_in;
+        } else {
+            double amax = 0.0;
+            int has_nan = 0;
+            for (int64_t k = 0; k < K; ++k) {
+                if (isnan(row[k])) has_nan = 1;
+                else if (fabs(row[k]) > amax) amax = fabs(row[k]);
+            }
+            s = has_nan ? NAN : (float)amax / 7.0f;
+        }
+        if (s < FLT_MIN) s = FLT_MIN;
+        scales[r] = s;
+        for (int64_t k = 0; k < K; ++k) {
+            float t = (float)row[k] / s;
+            if (isnan(t)) {
+                q[k] = 0;
+                continue;
+            }
+            if (rounding == 0) {
+                t = rintf(t);
+            } else {
+                const uint64_t e = (uint64_t)rows[r] * (uint64_t)K + (uint64_t)k;
+                const uint32_t ctr[4] = {(uint32_t)e, (uint32_t)(e >> 32), (uint32_t)offset,
+                                         (uint32_t)(offset >> 32)};
+                uint32_t rnd[4];
+                ck_oracle_philox4x32_10(ctr, key, rnd);
+                const float u = (float)(rnd[0] >> 8) * 0x1p-24f;
+                t = floorf(t + u);
+            }
+            if (t > 7.0f) t = 7.0f;
+            if (t < -8.0f) t = -8.0f;
+            q[k] = (int8_t)t;
+        }
+        for (int64_t i = 0; i < K / 2; ++i)
+            packed[r * (K / 2) + i] =
+                (uint8_t)(((uint8_t)q[2 * i] & 0xF) | (((uint8_t)q[2 * i + 1] & 0xF) << 4));
+    }
+    free(q);
+    return 0;
+}

@@ -29,6 +29,46 @@
 
 #ifdef __cplusplus
 extern "C" {
+/* ---------------------------------------------------------------- W8A8 variant
+ * The same rotation with INT8 codes (PR #155 "Add fused RotateQuant backend": the fused
+ * rotate-and-quantize operator emits INT8 codes with per-row scales; PR #198: the INT8
+ * linear): s = max(fp32(amax|y|) / 127, FLT_MIN) per row (or the caller's scale, clamped the
+ * same way), q = clamp(round_half_even(fp32(y) / s), -128, 127). */
+int ck_oracle_quantize_int8(const double* y, int64_t nrows, int64_t K, const float* scale_in,
+                            int8_t* codes, float* scales);
+
+int ck_oracle_rotate_quant_int8(const void* x, int dtype, int64_t M, int64_t K,
+                                int64_t stride_m, int64_t stride_k, const void* R, int g,
+                                const float* scale_in, const int64_t* rows, int64_t nrows,
+                                int8_t* codes, float* scales);
+
+/* W8A8 linear on the listed rows / cols: INT8 stage 1, INT8 weights w (N, K) with row pitch
+ * w_ld, exact INT32 GEMM, the same epilogue. */
+int ck_oracle_linear_w8a8(const void* x, int dtype, int64_t M, int64_t K, int64_t stride_m,
+                          int64_t stride_k, const void* R, int g, const int8_t* w, int64_t N,
+                          int64_t w_ld, const void* w_scale, const void* bias, int scale_dtype,
+                          int out_dtype, const int64_t* rows, int64_t nrows, const int64_t* cols,
+                          int64_t ncols, void* out, int8_t* codes, float* scales);
+
+/* ---------------------------------------------------------------- packed quantizer
+ * Philox4x32-10 (J. K. Salmon, M. A. Moraes, R. O. Dror, D. E. Shaw, "Parallel random
+ * numbers: as easy as 1, 2, 3", SC 2011): out = bijection of the 128-bit counter ctr under
+ * the 64-bit key, ten rounds. */
+int ck_oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
+
+/* The public signed-INT4 quantizer with nibble-packed output (PR #201 "Summary": the public
+ * packed quantizer keeps its signature, scales and stochastic rounding).  Scales as in
+ * ck_oracle_quantize.  t = fp32(y) / s (IEEE), then
+ *   rounding 0: q = clamp(round_half_even(t), -8, 7)
+ *   rounding 1: q = clamp(floor(fp32(t + u)), -8, 7), u = (r >> 8) * 2^-24 with r word 0 of
+ *               Philox4x32-10(counter {e, e >> 32, offset, offset >> 32}, key {seed, seed >> 32})
+ *               and e = rows[i] * K + k, the element's index in the (M, K) tensor
+ * (a NaN t gives 0).  packed (nrows, K / 2): byte k / 2 holds code k (even) in its low nibble
+ * and code k + 1 in its high nibble.  K must be even. */
+int ck_oracle_quantize_packed(const double* y, int64_t nrows, int64_t K, const float* scale_in,
+                              int rounding, uint64_t seed, uint64_t offset, const int64_t* rows,
+                              uint8_t* packed, float* scales);
+
 #endif
 
 /* Round each v[i] to the nearest value of the dtype (ties to even, IEEE overflow to inf). */
@@ -89,5 +129,85 @@ int ck_oracle_linear(const void* x, int dtype, int64_t M, int64_t K, int64_t str
 
 #ifdef __cplusplus
 }
+/* ---------------------------------------------------------------- W8A8 variant
+ * The same rotation with INT8 codes (PR #155 "Add fused RotateQuant backend": the fused
+ * rotate-and-quantize operator emits INT8 codes with per-row scales; PR #198: the INT8
+ * linear): s = max(fp32(amax|y|) / 127, FLT_MIN) per row (or the caller's scale, clamped the
+ * same way), q = clamp(round_half_even(fp32(y) / s), -128, 127). */
+int ck_oracle_quantize_int8(const double* y, int64_t nrows, int64_t K, const float* scale_in,
+                            int8_t* codes, float* scales);
+
+int ck_oracle_rotate_quant_int8(const void* x, int dtype, int64_t M, int64_t K,
+                                int64_t stride_m, int64_t stride_k, const void* R, int g,
+                                const float* scale_in, const int64_t* rows, int64_t nrows,
+                                int8_t* codes, float* scales);
+
+/* W8A8 linear on the listed rows / cols: INT8 stage 1, INT8 weights w (N, K) with row pitch
+ * w_ld, exact INT32 GEMM, the same epilogue. */
+int ck_oracle_linear_w8a8(const void* x, int dtype, int64_t M, int64_t K, int64_t stride_m,
+                          int64_t stride_k, const void* R, int g, const int8_t* w, int64_t N,
+                          int64_t w_ld, const void* w_scale, const void* bias, int scale_dtype,
+                          int out_dtype, const int64_t* rows, int64_t nrows, const int64_t* cols,
+                          int64_t ncols, void* out, int8_t* codes, float* scales);
+
+/* ---------------------------------------------------------------- packed quantizer
+ * Philox4x32-10 (J. K. Salmon, M. A. Moraes, R. O. Dror, D. E. Shaw, "Parallel random
+ * numbers: as easy as 1, 2, 3", SC 2011): out = bijection of the 128-bit counter ctr under
+ * the 64-bit key, ten rounds. */
+int ck_oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
+
+/* The public signed-INT4 quantizer with nibble-packed output (PR #201 "Summary": the public
+ * packed quantizer keeps its signature, scales and stochastic rounding).  Scales as in
+ * ck_oracle_quantize.  t = fp32(y) / s (IEEE), then
+ *   rounding 0: q = clamp(round_half_even(t), -8, 7)
+ *   rounding 1: q = clamp(floor(fp32(t + u)), -8, 7), u = (r >> 8) * 2^-24 with r word 0 of
+ *               Philox4x32-10(counter {e, e >> 32, offset, offset >> 32}, key {seed, seed >> 32})
+ *               and e = rows[i] * K + k, the element's index in the (M, K) tensor
+ * (a NaN t gives 0).  packed (nrows, K / 2): byte k / 2 holds code k (even) in its low nibble
+ * and code k + 1 in its high nibble.  K must be even. */
+int ck_oracle_quantize_packed(const double* y, int64_t nrows, int64_t K, const float* scale_in,
+                              int rounding, uint64_t seed, uint64_t offset, const int64_t* rows,
+                              uint8_t* packed, float* scales);
+
 #endif
+/* ---------------------------------------------------------------- W8A8 variant
+ * The same rotation with INT8 codes (PR #155 "Add fused RotateQuant backend": the fused
+ * rotate-and-quantize operator emits INT8 codes with per-row scales; PR #198: the INT8
+ * linear): s = max(fp32(amax|y|) / 127, FLT_MIN) per row (or the caller's scale, clamped the
+ * same way), q = clamp(round_half_even(fp32(y) / s), -128, 127). */
+int ck_oracle_quantize_int8(const double* y, int64_t nrows, int64_t K, const float* scale_in,
+                            int8_t* codes, float* scales);
+
+int ck_oracle_rotate_quant_int8(const void* x, int dtype, int64_t M, int64_t K,
+                                int64_t stride_m, int64_t stride_k, const void* R, int g,
+                                const float* scale_in, const int64_t* rows, int64_t nrows,
+                                int8_t* codes, float* scales);
+
+/* W8A8 linear on the listed rows / cols: INT8 stage 1, INT8 weights w (N, K) with row pitch
+ * w_ld, exact INT32 GEMM, the same epilogue. */
+int ck_oracle_linear_w8a8(const void* x, int dtype, int64_t M, int64_t K, int64_t stride_m,
+                          int64_t stride_k, const void* R, int g, const int8_t* w, int64_t N,
+                          int64_t w_ld, const void* w_scale, const void* bias, int scale_dtype,
+                          int out_dtype, const int64_t* rows, int64_t nrows, const int64_t* cols,
+                          int64_t ncols, void* out, int8_t* codes, float* scales);
+
+/* ---------------------------------------------------------------- packed quantizer
+ * Philox4x32-10 (J. K. Salmon, M. A. Moraes, R. O. Dror, D. E. Shaw, "Parallel random
+ * numbers: as easy as 1, 2, 3", SC 2011): out = bijection of the 128-bit counter ctr under
+ * the 64-bit key, ten rounds. */
+int ck_oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
+
+/* The public signed-INT4 quantizer with nibble-packed output (PR #201 "Summary": the public
+ * packed quantizer keeps its signature, scales and stochastic rounding).  Scales as in
+ * ck_oracle_quantize.  t = fp32(y) / s (IEEE), then
+ *   rounding 0: q = clamp(round_half_even(t), -8, 7)
+ *   rounding 1: q = clamp(floor(fp32(t + u)), -8, 7), u = (r >> 8) * 2^-24 with r word 0 of
+ *               Philox4x32-10(counter {e, e >> 32, offset, offset >> 32}, key {seed, seed >> 32})
+ *               and e = rows[i] * K + k, the element's index in the (M, K) tensor
+ * (a NaN t gives 0).  packed (nrows, K / 2): byte k / 2 holds code k (even) in its low nibble
+ * and code k + 1 in its high nibble.  K must be even. */
+int ck_oracle_quantize_packed(const double* y, int64_t nrows, int64_t K, const float* scale_in,
+                              int rounding, uint64_t seed, uint64_t offset, const int64_t* rows,
+                              uint8_t* packed, float* scales);
+
 #endif

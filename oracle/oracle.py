@@ -14,7 +14,8 @@ import torch
 from . import build as _build
 
 __all__ = ["lib", "round_to", "decode", "rotate", "quantize", "rotate_quant", "pack_w4",
-           "unpack_w4", "gemm_s32", "epilogue", "linear", "DT"]
+           "unpack_w4", "gemm_s32", "epilogue", "linear", "quantize_int8", "rotate_quant_int8",
+           "linear_w8a8", "philox4x32_10", "quantize_packed", "DT"]
 
 DT = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 DT_NAME = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
@@ -25,6 +26,7 @@ _lib = None
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
 _I = ctypes.c_int
+_U64 = ctypes.c_uint64
 
 _SIGS = {
     "ck_oracle_round": [_P, _I64, _I],
@@ -39,6 +41,12 @@ _SIGS = {
     "ck_oracle_epilogue": [_P, _I64, _I64, _P, _P, _P, _I, _P, _I],
     "ck_oracle_linear": [_P, _I, _I64, _I64, _I64, _I64, _P, _I, _P, _I64, _I64, _P, _P, _I, _I,
                          _P, _I64, _P, _I64, _P, _P, _P],
+    "ck_oracle_quantize_int8": [_P, _I64, _I64, _P, _P, _P],
+    "ck_oracle_rotate_quant_int8": [_P, _I, _I64, _I64, _I64, _I64, _P, _I, _P, _P, _I64, _P, _P],
+    "ck_oracle_linear_w8a8": [_P, _I, _I64, _I64, _I64, _I64, _P, _I, _P, _I64, _I64, _P, _P, _I,
+                              _I, _P, _I64, _P, _I64, _P, _P, _P],
+    "ck_oracle_philox4x32_10": [_P, _P, _P],
+    "ck_oracle_quantize_packed": [_P, _I64, _I64, _P, _I, _U64, _U64, _P, _P, _P],
 }
 
 
@@ -196,3 +204,78 @@ def linear(x: torch.Tensor, R: torch.Tensor, g: int, w_packed: torch.Tensor,
                                   _dtcode(ws), DT[out_dtype], _ptr(r), r.size, _ptr(c), c.size,
                                   _ptr(out), _ptr(codes), _ptr(scales)), "linear")
     return out, codes, scales
+
+
+# ---------------------------------------------------------------- W8A8 variant
+
+def quantize_int8(y: np.ndarray, scale_in: float | None = None):
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    n, K = y.shape
+    codes = np.empty((n, K), dtype=np.int8)
+    scales = np.empty(n, dtype=np.float32)
+    s_in = None if scale_in is None else np.array([scale_in], dtype=np.float32)
+    _check(lib().ck_oracle_quantize_int8(_ptr(y), n, K, _ptr(s_in), _ptr(codes), _ptr(scales)),
+           "quantize_int8")
+    return codes, scales
+
+
+def rotate_quant_int8(x: torch.Tensor, R: torch.Tensor, g: int, scale_in: float | None = None,
+                      rows=None):
+    M, K = x.shape
+    r = _rows(rows, M)
+    codes = np.empty((r.size, K), dtype=np.int8)
+    scales = np.empty(r.size, dtype=np.float32)
+    s_in = None if scale_in is None else np.array([scale_in], dtype=np.float32)
+    Rc = R.contiguous()
+    _check(lib().ck_oracle_rotate_quant_int8(_ptr(x), _dtcode(x), M, K, x.stride(0), x.stride(1),
+                                             _ptr(Rc), g, _ptr(s_in), _ptr(r), r.size,
+                                             _ptr(codes), _ptr(scales)), "rotate_quant_int8")
+    return codes, scales
+
+
+def linear_w8a8(x: torch.Tensor, R: torch.Tensor, g: int, w: torch.Tensor, w_scale: torch.Tensor,
+                bias: torch.Tensor | None, rows=None, cols=None, out_dtype=None):
+    """W8A8 linear (INT8 codes, INT8 weights (N, K)); returns (out, codes, scales)."""
+    M, K = x.shape
+    N = w.shape[0]
+    r = _rows(rows, M)
+    c = _rows(cols, N)
+    out_dtype = out_dtype or x.dtype
+    out = _out_tensor((r.size, c.size), out_dtype)
+    codes = np.empty((r.size, K), dtype=np.int8)
+    scales = np.empty(r.size, dtype=np.float32)
+    ws = w_scale.contiguous()
+    b = None if bias is None else bias.contiguous()
+    Rc = R.contiguous()
+    _check(lib().ck_oracle_linear_w8a8(_ptr(x), _dtcode(x), M, K, x.stride(0), x.stride(1),
+                                       _ptr(Rc), g, _ptr(w), N, w.stride(0), _ptr(ws), _ptr(b),
+                                       _dtcode(ws), DT[out_dtype], _ptr(r), r.size, _ptr(c),
+                                       c.size, _ptr(out), _ptr(codes), _ptr(scales)),
+           "linear_w8a8")
+    return out, codes, scales
+
+
+# ---------------------------------------------------------------- packed quantizer
+
+def philox4x32_10(ctr, key) -> np.ndarray:
+    c = np.ascontiguousarray(np.asarray(ctr, dtype=np.uint32))
+    k = np.ascontiguousarray(np.asarray(key, dtype=np.uint32))
+    out = np.empty(4, dtype=np.uint32)
+    _check(lib().ck_oracle_philox4x32_10(_ptr(c), _ptr(k), _ptr(out)), "philox4x32_10")
+    return out
+
+
+def quantize_packed(y: np.ndarray, rows, K: int, scale_in: float | None = None,
+                    stochastic: bool = False, seed: int = 0, offset: int = 0):
+    """Nibble-packed signed-INT4 codes of the rotated rows y (listed by their row index in the
+    (M, K) tensor, which the stochastic rounding's counter uses); returns (packed, scales)."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    n = y.shape[0]
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    packed = np.empty((n, K // 2), dtype=np.uint8)
+    scales = np.empty(n, dtype=np.float32)
+    s_in = None if scale_in is None else np.array([scale_in], dtype=np.float32)
+    _check(lib().ck_oracle_quantize_packed(_ptr(y), n, K, _ptr(s_in), 1 if stochastic else 0,
+                                           seed, offset, _ptr(r), _ptr(packed), _ptr(scales)),
+           "quantize_packed")
+    return packed, scales

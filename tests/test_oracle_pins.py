@@ -463,3 +463,138 @@ def test_linear_rows_cols_subset_matches_full():
     assert torch.equal(sub, full[rows][:, cols])
     np.testing.assert_array_equal(c2, codes[rows])
     np.testing.assert_array_equal(s2, scales[rows])
+
+
+# ------------------------------------------------------------------- W8A8 variant
+
+def _golden_int8_rows(golden_dir):
+    rows = []
+    for line in open(os.path.join(golden_dir, "quant_rows_int8.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        s_in, ys, s, qs = [c.strip() for c in line.split("|")]
+        rows.append((None if s_in == "dyn" else float(s_in), [float(v) for v in ys.split()],
+                     float(s), [int(v) for v in qs.split()]))
+    return rows
+
+
+def test_int8_quantizer_golden_rows(golden_dir):
+    for s_in, ys, s, qs in _golden_int8_rows(golden_dir):
+        codes, scales = oracle.quantize_int8(np.array([ys]), scale_in=s_in)
+        assert scales[0] == np.float32(s), (ys, scales[0])
+        np.testing.assert_array_equal(codes[0], qs)
+
+
+@pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
+def test_int8_dynamic_codes_reach_127_never_minus_128_and_reconstruct(dt):
+    rng = np.random.default_rng(41)
+    y = oracle.round_to(rng.standard_normal((64, 512)) * 3.0, W.DTYPES[dt])
+    y[5] = 0.0
+    codes, scales = oracle.quantize_int8(y)
+    amax = np.abs(y).max(axis=1)
+    live = amax > 0
+    np.testing.assert_array_equal(scales[live], (amax[live].astype(np.float32) / np.float32(127)))
+    assert (np.abs(codes[live]).max(axis=1) == 127).all()
+    assert (codes != -128).all()
+    # |y - q s| <= s / 2, plus the fp32 quotient's own rounding, which can move a value within
+    # |t| 2^-24 of a half-integer across it (|t| <= 127)
+    err = np.abs(y[live] - codes[live].astype(np.float64) * scales[live, None])
+    assert (err <= scales[live, None] * (0.5 + 127 * 2.0 ** -24) * (1 + 1e-9)).all()
+
+
+def test_w8a8_linear_tiny_brute_force():
+    """Independent numpy/torch evaluation of the W8A8 path on tiny shapes: group rotation in
+    float64 rounded to the dtype, INT8 grid, int64 matmul with INT8 weights, fp32 epilogue."""
+    rng = np.random.default_rng(43)
+    for dt, (M, N, K, g) in [("bf16", (5, 7, 64, 16)), ("f32", (3, 4, 128, 64)),
+                             ("f16", (2, 9, 256, 256))]:
+        tdt = W.DTYPES[dt]
+        x = torch.from_numpy(rng.standard_normal((M, K))).to(tdt)
+        R = W.haar_orthogonal(g, torch.Generator().manual_seed(g)).to(tdt)
+        w = torch.from_numpy(rng.integers(-128, 128, size=(N, K), dtype=np.int8))
+        ws = torch.from_numpy(rng.uniform(0.005, 0.02, N)).to(tdt)
+        b = torch.from_numpy(rng.standard_normal(N) * 0.1).to(tdt)
+        got, codes, scales = oracle.linear_w8a8(x, R, g, w, ws, b)
+        xd = x.double().numpy().reshape(M, K // g, g)
+        y = torch.from_numpy((xd @ R.double().numpy()).reshape(M, K)).to(tdt).double().numpy()
+        s = (np.abs(y).max(axis=1).astype(np.float32) / np.float32(127)).astype(np.float32)
+        s = np.maximum(s, np.float32(np.finfo(np.float32).tiny))
+        q = np.clip(np.rint(y.astype(np.float32) / s[:, None]), -128, 127).astype(np.int64)
+        np.testing.assert_array_equal(codes, q)
+        np.testing.assert_array_equal(scales, s)
+        acc = q @ w.numpy().astype(np.int64).T
+        o = acc.astype(np.float32) * s[:, None]
+        o = o * ws.float().numpy()[None, :]
+        o = o + b.float().numpy()[None, :]
+        assert torch.equal(got, torch.from_numpy(o).to(tdt))
+
+
+# ------------------------------------------------------------------- packed quantizer
+
+def test_philox_known_answer_vectors(golden_dir):
+    n = 0
+    for line in open(os.path.join(golden_dir, "philox4x32_10_kat.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        v = [int(t, 16) for t in line.split()]
+        np.testing.assert_array_equal(oracle.philox4x32_10(v[:4], v[4:6]), v[6:10])
+        n += 1
+    assert n == 3
+
+
+def test_packed_nearest_equals_packed_codes_of_the_quantizer():
+    rng = np.random.default_rng(44)
+    y = rng.standard_normal((9, 64)) * 2
+    y[3] = 0
+    packed, scales = oracle.quantize_packed(y, np.arange(9), 64)
+    codes, s2 = oracle.quantize(y)
+    np.testing.assert_array_equal(scales, s2)
+    np.testing.assert_array_equal(packed.view(np.int8), oracle.pack_w4(codes))
+
+
+def test_stochastic_rounding_first_draw_worked_by_hand():
+    """Element 0 of a tensor with seed 0 and offset 0 draws Philox(counter 0, key 0) word 0 =
+    0x6627e8d5, so u = 0x6627e8 * 2^-24 = 0.39904...; a row [2.7, 7, ...] has s = 1 and t = 2.7:
+    floor(2.7 + u) = 3; with 2.5 in its place floor(2.5 + u) = 2; with -0.7, floor(-0.3) = -1."""
+    u = np.float32(0x6627e8) * np.float32(2.0 ** -24)
+    assert abs(float(u) - 0.399) < 1e-3
+    for first, want in ((2.7, 3), (2.5, 2), (-0.7, -1)):
+        y = np.array([[first, 7.0] + [0.0] * 14])
+        packed, scales = oracle.quantize_packed(y, [0], 16, stochastic=True, seed=0, offset=0)
+        assert scales[0] == 1.0
+        lo = int(packed[0, 0]) & 0xF
+        assert (lo - 16 if lo >= 8 else lo) == want
+
+
+def _unpack_rows(packed):
+    lo = (packed & 0xF).astype(np.int64)
+    hi = (packed >> 4).astype(np.int64)
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    out = np.empty((packed.shape[0], packed.shape[1] * 2), dtype=np.int64)
+    out[:, 0::2] = lo
+    out[:, 1::2] = hi
+    return out
+
+
+def test_stochastic_rounding_brackets_the_quotient_and_is_unbiased():
+    rng = np.random.default_rng(45)
+    M, K = 64, 2048
+    y = rng.uniform(-6.5, 6.5, size=(M, K))
+    y[:, 0] = 7.0                                   # s = 1 in every row: t = y
+    y[:, 1::97] = np.round(y[:, 1::97])             # exact integers stay
+    packed, scales = oracle.quantize_packed(y, np.arange(M), K, stochastic=True, seed=1234)
+    assert (scales == 1.0).all()
+    q = _unpack_rows(packed)
+    t = y.astype(np.float32).astype(np.float64)
+    assert ((q == np.floor(t)) | (q == np.floor(t) + 1)).all()
+    ints = t == np.round(t)
+    np.testing.assert_array_equal(q[ints], t[ints])
+    frac = t - np.floor(t)
+    assert abs(float((q - np.floor(t)).mean() - frac.mean())) < 0.01   # E[q] = t
+    again, _ = oracle.quantize_packed(y, np.arange(M), K, stochastic=True, seed=1234)
+    np.testing.assert_array_equal(packed, again)
+    other, _ = oracle.quantize_packed(y, np.arange(M), K, stochastic=True, seed=1235)
+    assert (packed != other).any()
+    shifted, _ = oracle.quantize_packed(y, np.arange(M), K, stochastic=True, seed=1234, offset=1)
+    assert (packed != shifted).any()
