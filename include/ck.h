@@ -78,7 +78,9 @@ typedef enum { CK_F32 = 0, CK_F16 = 1, CK_BF16 = 2, CK_I8 = 3 } ck_dtype;
  * absmax, so a code may differ by one from an exact-arithmetic evaluation where
  * y / s lies within rounding of a half-integer.
  * Errors: CK_ERR_INVALID_ARG (null x/R/codes/scales, M < 0, K <= 0, K % g != 0,
- * bad g or dtype, ldq < K), CK_ERR_CUDA (launch failure).
+ * bad g or dtype, ldq < K, R not 16-byte aligned), CK_ERR_UNSUPPORTED (a shape no kernel of
+ * this build takes: an fp32 row above 56,000 channels that is neither row-major nor
+ * column-major with a 16-byte pitch), CK_ERR_CUDA (launch failure).
  */
 ck_status ck_rotate_quant(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
                           int64_t stride_m, int64_t stride_k, const void* R, int g,
@@ -120,6 +122,35 @@ ck_status ck_w4a4_linear(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
                          void* out, ck_dtype out_dtype, int64_t ldo,
                          void* workspace, size_t workspace_bytes, int* dev_status,
                          cudaStream_t stream);
+
+/*
+ * Several linears that read the same activations, as one call (comfy_kitchen/tensor/
+ * svdquant_w4a4.py: svdquant_w4a4_grouped_linear runs the projections that share one input,
+ * such as attention's Q, K and V, as one linear over their weights fused along N by
+ * svdquant_w4a4_fuse_linear_weights, and splits the result per projection).  Stage 1 runs
+ * once on x; one stage-2 GEMM covers the stacked weights; the channels of group i go to
+ * outs[i].
+ *
+ *   w_packed  (N, K/2) int8, the n_groups weights stacked along N in group order (row pitch
+ *             w_ld), N = group_n[0] + ... + group_n[n_groups - 1]
+ *   w_scale   (N,) stacked the same way; bias (N,) stacked, or NULL for no bias in any group
+ *   n_groups  1 to 8
+ *   group_n   host array: channels of each group (>= 0)
+ *   outs      host array of device pointers: group i's output (M, group_n[i]) of out_dtype
+ *   ldos      host array: group i's row pitch, >= group_n[i]
+ * Every other argument, the workspace size (for the stacked N) and the errors are those of
+ * ck_w4a4_linear, plus CK_ERR_INVALID_ARG for a bad n_groups, group_n or ldos, or a NULL
+ * outs[i] for a non-empty group.  Group i's output equals ck_w4a4_linear's with group i's
+ * weights, scales and bias alone, bit for bit: the same stage 1 and, per channel, the same
+ * arithmetic.
+ */
+ck_status ck_w4a4_grouped_linear(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                                 int64_t stride_m, int64_t stride_k, const void* R, int g,
+                                 const float* a_scale, const int8_t* w_packed, int64_t w_ld,
+                                 const void* w_scale, ck_dtype scale_dtype, const void* bias,
+                                 int n_groups, const int64_t* group_n, void* const* outs,
+                                 const int64_t* ldos, ck_dtype out_dtype, void* workspace,
+                                 size_t workspace_bytes, int* dev_status, cudaStream_t stream);
 
 /* Workspace ck_w4a4_linear needs for these sizes: the stage-1 codes and scales (also
  * used to re-pitch CK_I8 codes whose rows are not 16-byte aligned) and, when w_ld is
@@ -173,6 +204,64 @@ ck_status ck_w4a4_linear_noalloc(const void* x, ck_dtype x_dtype, int64_t M, int
                                  int64_t w_ld, const void* w_scale, ck_dtype scale_dtype,
                                  const void* bias, void* out, ck_dtype out_dtype, int64_t ldo,
                                  int* dev_status, cudaStream_t stream);
+
+/*
+ * The W8A8 variant (comfy-kitchen PR #155 "Add fused RotateQuant backend": the fused rotation
+ * and quantization emitting INT8 codes with per-row scales; PR #198 "Consolidate INT8,
+ * RotateQuant, RoPE and ConvRot W4A4 backends": the INT8 linear).  The same rotation, the INT8
+ * grid instead of INT4:
+ *   s[m] = max(fp32(max_k |y[m, k]|) / 127, FLT_MIN)   (or the caller's scale, clamped the same way)
+ *   q[m, k] = clamp(round_half_even(y[m, k] / s[m]), -128, 127)
+ * ck_rotate_quant_int8 takes and returns what ck_rotate_quant does.
+ */
+ck_status ck_rotate_quant_int8(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                               int64_t stride_m, int64_t stride_k, const void* R, int g,
+                               const float* scale_in, int8_t* codes, int64_t ldq, float* scales,
+                               int* dev_status, cudaStream_t stream);
+
+/*
+ * The W8A8 linear: ck_rotate_quant_int8 (or INT8 codes given with x_dtype == CK_I8 and their
+ * row scales in a_scale), then acc[m, n] = sum_k q[m, k] * w[n, k] in exact INT32 over INT8
+ * weights w (N, K) with row pitch w_ld >= K bytes (no unpack), and ck_w4a4_linear's epilogue.
+ * Every argument but w / w_ld means what it does for ck_w4a4_linear; the workspace is
+ * ck_w8a8_linear_workspace_bytes(M, N, K, w_ld).  CK_ERR_OVERFLOW when 128 * 128 * K > 2^31 - 1
+ * (K > 131071), the bound of |acc| on this grid.
+ */
+ck_status ck_w8a8_linear(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                         int64_t stride_m, int64_t stride_k, const void* R, int g,
+                         const float* a_scale, const int8_t* w, int64_t N, int64_t w_ld,
+                         const void* w_scale, ck_dtype scale_dtype, const void* bias,
+                         void* out, ck_dtype out_dtype, int64_t ldo,
+                         void* workspace, size_t workspace_bytes, int* dev_status,
+                         cudaStream_t stream);
+size_t ck_w8a8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t w_ld);
+
+/*
+ * The public packed-activation quantizer (comfy-kitchen PR #201 "Avoid activation pack/unpack
+ * in ConvRot W4A4", "Summary": the W4A4 path no longer packs activations, while the public
+ * packed quantizer keeps its signature, scales and stochastic rounding; "Correctness and
+ * tests": odd widths are rejected).  The rotation and row scale of ck_rotate_quant, then with
+ * t = y / s (the IEEE fp32 quotient):
+ *   stochastic == 0:  q = clamp(round_half_even(t), -8, 7)
+ *   stochastic == 1:  q = clamp(floor(t + u), -8, 7) with the sum rounded to fp32 and
+ *                     u = (r >> 8) * 2^-24, r = word 0 of Philox4x32-10 (Salmon et al., SC 2011)
+ *                     of counter {e, e >> 32, offset, offset >> 32} under key {seed, seed >> 32},
+ *                     e = m * K + k the element's index: the same (seed, offset) gives the same
+ *                     codes, and E[q] = t inside the grid.
+ * (NaN quotients give 0.)  The pages give no random-number specification; this one is the
+ * library's.
+ *   packed   (M, K / 2) bytes, row pitch ld_packed >= K / 2: byte k / 2 holds code k (even k) in
+ *            its low nibble and code k + 1 in its high nibble.
+ *   scales   (M,) fp32, as ck_rotate_quant.
+ * Errors: CK_ERR_INVALID_ARG (as ck_rotate_quant, plus odd K, ld_packed < K / 2, stochastic
+ * not 0 or 1), CK_ERR_UNSUPPORTED (rows whose fp32 copy and R exceed shared memory, about
+ * 56,000 channels), CK_ERR_CUDA.
+ */
+ck_status ck_rotate_quant_packed(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                                 int64_t stride_m, int64_t stride_k, const void* R, int g,
+                                 const float* scale_in, int stochastic, uint64_t seed,
+                                 uint64_t offset, uint8_t* packed, int64_t ld_packed,
+                                 float* scales, cudaStream_t stream);
 
 /* Static description of a status code (never NULL). */
 const char* ck_status_string(ck_status status);

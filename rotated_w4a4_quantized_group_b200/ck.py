@@ -34,7 +34,16 @@ SIGNATURES = {
     "ck_workspace_scales_offset": ([_I64, _I64], _SZ),
     "ck_w4a4_linear_noalloc": ([_P, _I, _I64, _I64, _I64, _I64, _P, _I, _P, _P, _I64, _I64, _P,
                                 _I, _P, _P, _I, _I64, _P, _P], _I),
+    "ck_w4a4_grouped_linear": ([_P, _I, _I64, _I64, _I64, _I64, _P, _I, _P, _P, _I64, _P, _I, _P,
+                                _I, _P, _P, _P, _I, _P, _SZ, _P, _P], _I),
     "ck_unpack_w4": ([_P, _I64, _I64, _I64, _P, _I64, _P], _I),
+    "ck_rotate_quant_int8": ([_P, _I, _I64, _I64, _I64, _I64, _P, _I, _P, _P, _I64, _P, _P, _P],
+                             _I),
+    "ck_w8a8_linear": ([_P, _I, _I64, _I64, _I64, _I64, _P, _I, _P, _P, _I64, _I64, _P, _I, _P,
+                        _P, _I, _I64, _P, _SZ, _P, _P], _I),
+    "ck_w8a8_linear_workspace_bytes": ([_I64, _I64, _I64, _I64], _SZ),
+    "ck_rotate_quant_packed": ([_P, _I, _I64, _I64, _I64, _I64, _P, _I, _P, _I, ctypes.c_uint64,
+                                ctypes.c_uint64, _P, _I64, _P, _P], _I),
     "ck_status_string": ([_I], ctypes.c_char_p),
 }
 
@@ -48,19 +57,24 @@ class CkError(RuntimeError):
 _lib = None
 
 
+def load_library(path: str) -> ctypes.CDLL:
+    """Load a build of the library at `path` with every entry point's ctypes signature set."""
+    if not os.path.exists(path):
+        raise ImportError(f"{os.path.basename(path)} not found at {path}; run "
+                          "`python -m rotated_w4a4_quantized_group_b200.build`")
+    L = ctypes.CDLL(path)
+    for name, (args, res) in SIGNATURES.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    return L
+
+
 def lib() -> ctypes.CDLL:
     """Load libck.so (raises if it is missing: build it with the package's build module)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise ImportError(f"libck.so not found at {LIB_PATH}; run "
-                              "`python -m rotated_w4a4_quantized_group_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
-        for name, (args, res) in SIGNATURES.items():
-            fn = getattr(L, name)
-            fn.argtypes = args
-            fn.restype = res
-        _lib = L
+        _lib = load_library(LIB_PATH)
     return _lib
 
 
@@ -215,6 +229,146 @@ def ck_w4a4_linear_noalloc(x: torch.Tensor, R: torch.Tensor | None, g: int,
             out.stride(0), _ptr(dev_status), _stream(stream))
     _check(st, "ck_w4a4_linear_noalloc")
     return out
+
+
+def fuse_linear_weights(parts):
+    """Stack the packed weights, weight scales and biases of several linears that share one
+    input along N (one-time weight preparation, done on the device by torch): parts is a list
+    of (w_packed (N_i, K/2) int8, w_scale (N_i,), bias (N_i,) or None).  Returns
+    (w_packed (N, K/2), w_scale (N,), bias (N,) or None, [N_i]); biases that are None become
+    zeros when another part has one."""
+    if not parts:
+        raise ValueError("fuse_linear_weights needs at least one linear")
+    ws = torch.cat([p[0] for p in parts], 0).contiguous()
+    sc = torch.cat([p[1] for p in parts], 0).contiguous()
+    if all(p[2] is None for p in parts):
+        bias = None
+    else:
+        bias = torch.cat([p[2] if p[2] is not None else torch.zeros_like(p[1]) for p in parts],
+                         0).contiguous()
+    return ws, sc, bias, [int(p[0].shape[0]) for p in parts]
+
+
+def ck_w4a4_grouped_linear(x: torch.Tensor, R: torch.Tensor | None, g: int,
+                           w_packed: torch.Tensor, w_scale: torch.Tensor,
+                           bias: torch.Tensor | None, group_n, *, outs=None,
+                           a_scale: torch.Tensor | None = None,
+                           out_dtype: torch.dtype | None = None,
+                           workspace: torch.Tensor | None = None,
+                           dev_status: torch.Tensor | None = None, stream=None):
+    """Several linears sharing x as one call: w_packed/w_scale/bias are the groups' weights
+    stacked along N (fuse_linear_weights), group_n the channels of each group.  Returns the
+    list of per-group outputs (M, N_i)."""
+    M, K = x.shape
+    N = int(sum(group_n))
+    if x.dtype != torch.int8:
+        _check_rotation(x, R, g)
+    _check_weights(w_packed, N, K)
+    _same_device(x, R, w_packed, w_scale, bias, a_scale, workspace, dev_status)
+    odt = out_dtype or (x.dtype if x.dtype != torch.int8 else w_scale.dtype)
+    if outs is None:
+        outs = [torch.empty(M, int(n), dtype=odt, device=x.device) for n in group_n]
+    if len(outs) != len(group_n):
+        raise ValueError("one output per group")
+    for o, n in zip(outs, group_n):
+        _check_out(o, M, int(n), x)
+        if o.dtype != outs[0].dtype:
+            raise ValueError("every group's output has the same dtype")
+    G = len(group_n)
+    gn = (ctypes.c_int64 * G)(*[int(n) for n in group_n])
+    ptrs = (ctypes.c_void_p * G)(*[o.data_ptr() for o in outs])
+    ldos = (ctypes.c_int64 * G)(*[o.stride(0) for o in outs])
+    with torch.cuda.device(x.device):
+        if workspace is None:
+            nbytes = workspace_bytes(M, N, K, w_packed.stride(0))
+            workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+        st = lib().ck_w4a4_grouped_linear(
+            _ptr(x), DTYPE_CODE[x.dtype], M, K, x.stride(0), x.stride(1), _ptr(R), int(g),
+            _ptr(a_scale), _ptr(w_packed), w_packed.stride(0), _ptr(w_scale),
+            DTYPE_CODE[w_scale.dtype], _ptr(bias), G, gn, ptrs, ldos, DTYPE_CODE[outs[0].dtype],
+            _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream))
+    _check(st, "ck_w4a4_grouped_linear")
+    return outs
+
+
+def ck_rotate_quant_int8(x: torch.Tensor, R: torch.Tensor, g: int,
+                         scale_in: torch.Tensor | None = None, codes: torch.Tensor | None = None,
+                         scales: torch.Tensor | None = None,
+                         dev_status: torch.Tensor | None = None, stream=None):
+    """The W8A8 variant's stage 1: INT8 codes (qmax 127) and fp32 row scales of a 2-D view."""
+    M, K = x.shape
+    _check_rotation(x, R, g)
+    _same_device(x, R, scale_in, codes, scales, dev_status)
+    if codes is None:
+        codes = torch.empty(M, K, dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty(M, dtype=torch.float32, device=x.device)
+    if codes.dtype != torch.int8 or tuple(codes.shape) != (M, K) or codes.stride(1) != 1:
+        raise ValueError(f"codes must be an int8 ({M}, {K}) view with unit inner stride")
+    if scales.dtype != torch.float32 or scales.numel() < M or not scales.is_contiguous():
+        raise ValueError(f"scales must be a contiguous fp32 tensor of at least {M} values")
+    with torch.cuda.device(x.device):
+        st = lib().ck_rotate_quant_int8(_ptr(x), DTYPE_CODE[x.dtype], M, K, x.stride(0),
+                                        x.stride(1), _ptr(R), g, _ptr(scale_in), _ptr(codes),
+                                        codes.stride(0), _ptr(scales), _ptr(dev_status),
+                                        _stream(stream))
+    _check(st, "ck_rotate_quant_int8")
+    return codes, scales
+
+
+def ck_w8a8_linear(x: torch.Tensor, R: torch.Tensor | None, g: int, w: torch.Tensor,
+                   w_scale: torch.Tensor, bias: torch.Tensor | None = None, *,
+                   a_scale: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                   out_dtype: torch.dtype | None = None, workspace: torch.Tensor | None = None,
+                   dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The W8A8 linear: x (M, K) activations (or INT8 codes with a_scale), w (N, K) int8."""
+    M, K = x.shape
+    N = w.shape[0]
+    if x.dtype != torch.int8:
+        _check_rotation(x, R, g)
+    if w.dtype != torch.int8 or w.dim() != 2 or w.stride(1) != 1 or tuple(w.shape) != (N, K):
+        raise ValueError(f"w must be an int8 (N, K) = ({N}, {K}) view with unit inner stride")
+    _same_device(x, R, w, w_scale, bias, a_scale, workspace, dev_status)
+    if out is None:
+        odt = out_dtype or (x.dtype if x.dtype != torch.int8 else w_scale.dtype)
+        out = torch.empty(M, N, dtype=odt, device=x.device)
+    _check_out(out, M, N, x)
+    with torch.cuda.device(x.device):
+        if workspace is None:
+            nbytes = int(lib().ck_w8a8_linear_workspace_bytes(M, N, K, w.stride(0)))
+            workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+        st = lib().ck_w8a8_linear(
+            _ptr(x), DTYPE_CODE[x.dtype], M, K, x.stride(0), x.stride(1), _ptr(R), int(g),
+            _ptr(a_scale), _ptr(w), N, w.stride(0), _ptr(w_scale), DTYPE_CODE[w_scale.dtype],
+            _ptr(bias), _ptr(out), DTYPE_CODE[out.dtype], out.stride(0), _ptr(workspace),
+            workspace.numel(), _ptr(dev_status), _stream(stream))
+    _check(st, "ck_w8a8_linear")
+    return out
+
+
+def ck_rotate_quant_packed(x: torch.Tensor, R: torch.Tensor, g: int, *, stochastic: bool = False,
+                           seed: int = 0, offset: int = 0, scale_in: torch.Tensor | None = None,
+                           packed: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                           stream=None):
+    """The public packed quantizer: (packed uint8 (M, K/2), scales fp32 (M,)); stochastic
+    rounding draws from Philox4x32-10 keyed by seed at counter (element index, offset)."""
+    M, K = x.shape
+    _check_rotation(x, R, g)
+    _same_device(x, R, scale_in, packed, scales)
+    if packed is None:
+        packed = torch.empty(M, K // 2, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(M, dtype=torch.float32, device=x.device)
+    if packed.dtype != torch.uint8 or tuple(packed.shape) != (M, K // 2) or packed.stride(1) != 1:
+        raise ValueError(f"packed must be a uint8 ({M}, {K // 2}) view with unit inner stride")
+    with torch.cuda.device(x.device):
+        st = lib().ck_rotate_quant_packed(_ptr(x), DTYPE_CODE[x.dtype], M, K, x.stride(0),
+                                          x.stride(1), _ptr(R), g, _ptr(scale_in),
+                                          1 if stochastic else 0, seed & (2 ** 64 - 1),
+                                          offset & (2 ** 64 - 1), _ptr(packed), packed.stride(0),
+                                          _ptr(scales), _stream(stream))
+    _check(st, "ck_rotate_quant_packed")
+    return packed, scales
 
 
 def ck_unpack_w4(packed: torch.Tensor, K: int, out: torch.Tensor | None = None,

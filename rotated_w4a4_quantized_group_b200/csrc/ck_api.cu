@@ -61,11 +61,14 @@ static bool float_dtype(ck_dtype d) { return d == CK_F32 || d == CK_F16 || d == 
 static bool group_ok(int g) { return g == 16 || g == 64 || g == 256; }
 static int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 
-// The largest K for which |acc| <= 8 * 8 * K fits in int32.
+// The largest K for which |acc| <= 8 * 8 * K fits in int32 (INT4 codes), and the same for
+// INT8 codes and weights (|acc| <= 128 * 128 * K).
 static constexpr int64_t kMaxK = 2147483647LL / 64;
+static constexpr int64_t kMaxK8 = 2147483647LL / (128 * 128);
 
 size_t linear_scratch_need(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
-                           int64_t stride_m, const int8_t* w_packed, int64_t N, int64_t w_ld) {
+                           int64_t stride_m, const int8_t* w_packed, int64_t N, int64_t w_ld,
+                           bool w8) {
     const bool codes_in = x_dtype == CK_I8;
     const bool codes_aligned = codes_in && aligned(x, 16) && stride_m % 16 == 0;
     const bool w_aligned = aligned(w_packed, 16) && w_ld % 16 == 0;
@@ -74,7 +77,7 @@ size_t linear_scratch_need(const void* x, ck_dtype x_dtype, int64_t M, int64_t K
     const size_t wcopy_off = scales_off + (size_t)round_up(4 * M, 256);
     size_t need = 0;
     if (!codes_in || !codes_aligned) need = wcopy_off;
-    if (!w_aligned) need = wcopy_off + (size_t)round_up(N * round_up(K / 2, 16), 256);
+    if (!w_aligned) need = wcopy_off + (size_t)round_up(N * round_up(w8 ? K : K / 2, 16), 256);
     return need;
 }
 
@@ -104,6 +107,13 @@ size_t ck_workspace_scales_offset(int64_t M, int64_t K) {
     return (size_t)round_up(M * ck_workspace_codes_pitch(K), 256);
 }
 
+size_t ck_w8a8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t w_ld) {
+    if (M < 0 || N < 0 || K <= 0 || K % 2 != 0 || w_ld < K) return 0;
+    size_t bytes = ck_workspace_scales_offset(M, K) + (size_t)round_up(4 * M, 256);
+    if (w_ld % 16 != 0) bytes += (size_t)round_up(N * round_up(K, 16), 256);
+    return bytes;
+}
+
 size_t ck_w4a4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t w_ld) {
     if (M < 0 || N < 0 || K <= 0 || K % 2 != 0 || w_ld < K / 2) return 0;
     size_t bytes = ck_workspace_scales_offset(M, K) + (size_t)round_up(4 * M, 256);
@@ -111,17 +121,49 @@ size_t ck_w4a4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t w
     return bytes;
 }
 
-ck_status ck_rotate_quant(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
-                          int64_t stride_m, int64_t stride_k, const void* R, int g,
-                          const float* scale_in, int8_t* codes, int64_t ldq, float* scales,
-                          int* dev_status, cudaStream_t stream) {
+static ck_status rotate_quant_checked(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                                      int64_t stride_m, int64_t stride_k, const void* R, int g,
+                                      const float* scale_in, int8_t* codes, int64_t ldq,
+                                      float* scales, int qmax, int* dev_status,
+                                      cudaStream_t stream) {
     if (!float_dtype(x_dtype) || !group_ok(g) || M < 0 || K <= 0 || K % g != 0 || ldq < K)
         return CK_ERR_INVALID_ARG;
     if (M == 0) return CK_OK;
     if (!x || !R || !codes || !scales) return CK_ERR_INVALID_ARG;
     if (!aligned(R, 16)) return CK_ERR_INVALID_ARG;
     return launch_rotate_quant(x, x_dtype, M, K, stride_m, stride_k, R, g, scale_in, codes, ldq,
-                               scales, dev_status, stream);
+                               scales, qmax, dev_status, stream);
+}
+
+ck_status ck_rotate_quant(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                          int64_t stride_m, int64_t stride_k, const void* R, int g,
+                          const float* scale_in, int8_t* codes, int64_t ldq, float* scales,
+                          int* dev_status, cudaStream_t stream) {
+    return rotate_quant_checked(x, x_dtype, M, K, stride_m, stride_k, R, g, scale_in, codes, ldq,
+                                scales, 7, dev_status, stream);
+}
+
+ck_status ck_rotate_quant_int8(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                               int64_t stride_m, int64_t stride_k, const void* R, int g,
+                               const float* scale_in, int8_t* codes, int64_t ldq, float* scales,
+                               int* dev_status, cudaStream_t stream) {
+    return rotate_quant_checked(x, x_dtype, M, K, stride_m, stride_k, R, g, scale_in, codes, ldq,
+                                scales, 127, dev_status, stream);
+}
+
+ck_status ck_rotate_quant_packed(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                                 int64_t stride_m, int64_t stride_k, const void* R, int g,
+                                 const float* scale_in, int stochastic, uint64_t seed,
+                                 uint64_t offset, uint8_t* packed, int64_t ld_packed,
+                                 float* scales, cudaStream_t stream) {
+    if (!float_dtype(x_dtype) || !group_ok(g) || M < 0 || K <= 0 || K % 2 != 0 || K % g != 0 ||
+        ld_packed < K / 2 || (stochastic != 0 && stochastic != 1))
+        return CK_ERR_INVALID_ARG;
+    if (M == 0) return CK_OK;
+    if (!x || !R || !packed || !scales) return CK_ERR_INVALID_ARG;
+    return launch_rotate_quant_packed(x, x_dtype, M, K, stride_m, stride_k, R, g, scale_in,
+                                      stochastic != 0, seed, offset, packed, ld_packed, scales,
+                                      stream);
 }
 
 ck_status ck_unpack_w4(const int8_t* packed, int64_t N, int64_t K, int64_t ld_packed,
@@ -133,26 +175,35 @@ ck_status ck_unpack_w4(const int8_t* packed, int64_t N, int64_t K, int64_t ld_pa
     return launch_unpack_w4(packed, N, K, ld_packed, out, ld_out, stream);
 }
 
-ck_status ck_w4a4_linear(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
-                         int64_t stride_m, int64_t stride_k, const void* R, int g,
-                         const float* a_scale, const int8_t* w_packed, int64_t N, int64_t w_ld,
-                         const void* w_scale, ck_dtype scale_dtype, const void* bias,
-                         void* out, ck_dtype out_dtype, int64_t ldo, void* workspace,
-                         size_t workspace_bytes, int* dev_status, cudaStream_t stream) {
+}  // extern "C"
+
+namespace ck {
+
+// The linear once its outputs' places are known (one segment, or one per group); every
+// argument check but the outputs' is here.
+static ck_status linear_impl(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                             int64_t stride_m, int64_t stride_k, const void* R, int g,
+                             const float* a_scale, const int8_t* w_packed, int64_t N, int64_t w_ld,
+                             const void* w_scale, ck_dtype scale_dtype, const void* bias,
+                             const OutSegs& segs, ck_dtype out_dtype, void* workspace,
+                             size_t workspace_bytes, bool w8, int* dev_status,
+                             cudaStream_t stream) {
     const bool codes_in = x_dtype == CK_I8;
     if (!(codes_in || float_dtype(x_dtype)) || !float_dtype(scale_dtype) ||
         !float_dtype(out_dtype))
         return CK_ERR_INVALID_ARG;
-    if (M < 0 || N < 0 || K <= 0 || K % 2 != 0 || w_ld < K / 2 || ldo < N)
+    if (M < 0 || N < 0 || K <= 0 || K % 2 != 0 || w_ld < (w8 ? K : K / 2))
         return CK_ERR_INVALID_ARG;
     if (codes_in) {
         if (stride_k != 1 || stride_m < K) return CK_ERR_INVALID_ARG;
     } else {
         if (!group_ok(g) || K % g != 0) return CK_ERR_INVALID_ARG;
     }
-    if (K > kMaxK) return CK_ERR_OVERFLOW;
+    if (K > (w8 ? kMaxK8 : kMaxK)) return CK_ERR_OVERFLOW;
     if (M == 0 || N == 0) return CK_OK;
-    if (!x || !w_packed || !w_scale || !out) return CK_ERR_INVALID_ARG;
+    if (!x || !w_packed || !w_scale) return CK_ERR_INVALID_ARG;
+    for (int s = 0; s < segs.n; ++s)
+        if (segs.start[s + 1] > segs.start[s] && !segs.ptr[s]) return CK_ERR_INVALID_ARG;
     if (codes_in ? !a_scale : (!R || !aligned(R, 16))) return CK_ERR_INVALID_ARG;
     if (M >= (1LL << 31) || N >= (1LL << 31)) return CK_ERR_UNSUPPORTED;
 
@@ -162,7 +213,7 @@ ck_status ck_w4a4_linear(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
     const size_t wcopy_off = scales_off + (size_t)round_up(4 * M, 256);
     const bool codes_aligned = codes_in && aligned(x, 16) && stride_m % 16 == 0;
     const bool w_aligned = aligned(w_packed, 16) && w_ld % 16 == 0;
-    const size_t need = linear_scratch_need(x, x_dtype, M, K, stride_m, w_packed, N, w_ld);
+    const size_t need = linear_scratch_need(x, x_dtype, M, K, stride_m, w_packed, N, w_ld, w8);
     if (need) {
         if (!ws || workspace_bytes < need || !aligned(ws, 256)) return CK_ERR_WORKSPACE;
     }
@@ -187,7 +238,7 @@ ck_status ck_w4a4_linear(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
         int8_t* wcodes = reinterpret_cast<int8_t*>(ws);
         float* wscales = reinterpret_cast<float*>(ws + scales_off);
         st = launch_rotate_quant(x, x_dtype, M, K, stride_m, stride_k, R, g, nullptr, wcodes, P,
-                                 wscales, dev_status, stream);
+                                 wscales, w8 ? 127 : 7, dev_status, stream);
         if (st != CK_OK) return st;
         codes = wcodes;
         ldq = P;
@@ -196,15 +247,74 @@ ck_status ck_w4a4_linear(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
     const int8_t* wp = w_packed;
     int64_t wld = w_ld;
     if (!w_aligned) {
-        const int64_t wp_pitch = round_up(K / 2, 16);
+        const int64_t wrow = w8 ? K : K / 2;
+        const int64_t wp_pitch = round_up(wrow, 16);
         int8_t* dst = reinterpret_cast<int8_t*>(ws + wcopy_off);
-        st = launch_copy_rows(w_packed, w_ld, dst, wp_pitch, N, K / 2, stream);
+        st = launch_copy_rows(w_packed, w_ld, dst, wp_pitch, N, wrow, stream);
         if (st != CK_OK) return st;
         wp = dst;
         wld = wp_pitch;
     }
+    if (w8)
+        return launch_w8a8_gemm(codes, ldq, row_scale, M, K, wp, wld, N, w_scale, scale_dtype,
+                                bias, segs, out_dtype, dev_status, stream);
     return launch_w4a4_gemm(codes, ldq, row_scale, M, K, wp, wld, N, w_scale, scale_dtype, bias,
-                            out, out_dtype, ldo, dev_status, stream);
+                            segs, out_dtype, dev_status, stream);
+}
+
+}  // namespace ck
+
+extern "C" {
+
+ck_status ck_w4a4_linear(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                         int64_t stride_m, int64_t stride_k, const void* R, int g,
+                         const float* a_scale, const int8_t* w_packed, int64_t N, int64_t w_ld,
+                         const void* w_scale, ck_dtype scale_dtype, const void* bias,
+                         void* out, ck_dtype out_dtype, int64_t ldo, void* workspace,
+                         size_t workspace_bytes, int* dev_status, cudaStream_t stream) {
+    if (ldo < N) return CK_ERR_INVALID_ARG;
+    if (M > 0 && N > 0 && !out) return CK_ERR_INVALID_ARG;
+    return linear_impl(x, x_dtype, M, K, stride_m, stride_k, R, g, a_scale, w_packed, N, w_ld,
+                       w_scale, scale_dtype, bias, single_segment(out, N, ldo), out_dtype,
+                       workspace, workspace_bytes, false, dev_status, stream);
+}
+
+ck_status ck_w8a8_linear(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                         int64_t stride_m, int64_t stride_k, const void* R, int g,
+                         const float* a_scale, const int8_t* w, int64_t N, int64_t w_ld,
+                         const void* w_scale, ck_dtype scale_dtype, const void* bias,
+                         void* out, ck_dtype out_dtype, int64_t ldo, void* workspace,
+                         size_t workspace_bytes, int* dev_status, cudaStream_t stream) {
+    if (ldo < N) return CK_ERR_INVALID_ARG;
+    if (M > 0 && N > 0 && !out) return CK_ERR_INVALID_ARG;
+    return linear_impl(x, x_dtype, M, K, stride_m, stride_k, R, g, a_scale, w, N, w_ld, w_scale,
+                       scale_dtype, bias, single_segment(out, N, ldo), out_dtype, workspace,
+                       workspace_bytes, true, dev_status, stream);
+}
+
+ck_status ck_w4a4_grouped_linear(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
+                                 int64_t stride_m, int64_t stride_k, const void* R, int g,
+                                 const float* a_scale, const int8_t* w_packed, int64_t w_ld,
+                                 const void* w_scale, ck_dtype scale_dtype, const void* bias,
+                                 int n_groups, const int64_t* group_n, void* const* outs,
+                                 const int64_t* ldos, ck_dtype out_dtype, void* workspace,
+                                 size_t workspace_bytes, int* dev_status, cudaStream_t stream) {
+    if (n_groups < 1 || n_groups > kMaxOutSegs || !group_n || !outs || !ldos)
+        return CK_ERR_INVALID_ARG;
+    OutSegs segs = {};
+    segs.n = n_groups;
+    int64_t N = 0;
+    for (int i = 0; i < n_groups; ++i) {
+        if (group_n[i] < 0 || ldos[i] < group_n[i]) return CK_ERR_INVALID_ARG;
+        segs.start[i] = N;
+        segs.ptr[i] = outs[i];
+        segs.ldo[i] = ldos[i];
+        N += group_n[i];
+    }
+    segs.start[n_groups] = N;
+    return linear_impl(x, x_dtype, M, K, stride_m, stride_k, R, g, a_scale, w_packed, N, w_ld,
+                       w_scale, scale_dtype, bias, segs, out_dtype, workspace, workspace_bytes,
+                       false, dev_status, stream);
 }
 
 }  // extern "C"

@@ -15,6 +15,16 @@ namespace ck {
 // B200's clocks) gives up, records CK_ERR_TIMEOUT and lets the kernel exit.
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
+// The limit of a role's waits on its ring (every wait given an abort flag); the waits for
+// copies and MMAs already in flight keep kWaitLimitCycles.  The library built for the expiry
+// test sets it to 0: such a wait then gives up unless its phase is already complete, so the
+// kernel takes its timeout path (record the status, stop issuing, drain what is in flight,
+// free tensor memory, return) on an ordinary input.
+#ifndef CK_ROLE_WAIT_LIMIT_CYCLES
+#define CK_ROLE_WAIT_LIMIT_CYCLES 2000000000LL
+#endif
+constexpr long long kRoleWaitLimitCycles = CK_ROLE_WAIT_LIMIT_CYCLES;
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -55,6 +65,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Whether the phase with the given parity has completed, without waiting at all.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // try_wait that may suspend the thread (up to about 20 us) until the phase completes, so a
 // waiting warp does not take issue slots from the working ones.
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
@@ -74,17 +97,67 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // *abort is seen set by another role of the CTA.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* dev_status) {
+    const long long limit = abort ? kRoleWaitLimitCycles : kWaitLimitCycles;
+    if (limit <= 0) {
+        // the expiry-test build: give up unless the phase is already complete (try_wait may
+        // suspend the thread for a while, during which most phases complete)
+        if (mbar_test_wait(bar, parity)) return true;
+        if (abort) *abort = 1;
+        record_timeout(dev_status);
+        return false;
+    }
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait_sleep(bar, parity)) return true;
         if (abort && *abort) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             if (abort) *abort = 1;
             record_timeout(dev_status);
             return false;
         }
     }
+}
+
+// ------------------------------------------------------------------ thread-block clusters
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+// All threads of every CTA of the cluster: shared-memory writes before it are visible to the
+// cluster's reads after it.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// A 32-bit word of CTA `rank`'s shared memory at the address of `local` in this CTA.
+__device__ __forceinline__ uint32_t dsmem_load_u32(const void* local, uint32_t rank) {
+    uint32_t remote, v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
+    return v;
+}
+
+// Sixteen bytes of CTA `rank`'s shared memory at the address of `local` in this CTA.
+__device__ __forceinline__ uint4 dsmem_load_v4(const void* local, uint32_t rank) {
+    uint32_t remote;
+    uint4 v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(remote)
+                 : "memory");
+    return v;
 }
 
 // ------------------------------------------------------------------ TMA
@@ -293,12 +366,13 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
     return r;
 }
 
-// Signed-INT4 code of one value: clamp(round_half_even(y / s), -8, 7); NaN -> 0.
-__device__ __forceinline__ int quant_code(float y, float s) {
+// Signed code of one value on the grid [-qmax - 1, qmax] (qmax = 7 for INT4, 127 for INT8):
+// clamp(round_half_even(y / s), -qmax - 1, qmax); NaN -> 0.
+__device__ __forceinline__ int quant_code(float y, float s, int qmax) {
     float t = __fdiv_rn(y, s);
     if (t != t) return 0;
     t = rintf(t);
-    t = fminf(fmaxf(t, -8.0f), 7.0f);
+    t = fminf(fmaxf(t, (float)(-qmax - 1)), (float)qmax);
     return (int)t;
 }
 
@@ -321,7 +395,8 @@ __device__ __forceinline__ int quant_code(float y, float s) {
 struct RowDivisor {
     float s, r;
     bool fast;
-    __device__ __forceinline__ explicit RowDivisor(float s_) : s(s_) {
+    int qmax;   // the code grid [-qmax - 1, qmax]: 7 (INT4) or 127 (INT8)
+    __device__ __forceinline__ RowDivisor(float s_, int qmax_) : s(s_), qmax(qmax_) {
         r = __frcp_rn(s_);
         const bool pow2 = (__float_as_uint(s_) & 0x007FFFFFu) == 0u;
         fast = (s_ >= 0x1p-64f || pow2) && (r >= 1.17549435e-38f) && (r <= 3.40282347e38f);
@@ -329,20 +404,20 @@ struct RowDivisor {
 };
 
 // fl(y / s) for a fast RowDivisor (Markstein's correction, see RowDivisor), or y r where
-// |y r| >= 16, which saturates the code the same way.
+// |y r| >= 1024, which saturates the code of either grid the same way.
 __device__ __forceinline__ float quotient_fast(float y, float s, float r) {
     const float t = __fmul_rn(y, r);
     const float e = __fmaf_rn(-t, s, y);
     const float q = __fmaf_rn(e, r, t);
-    return fabsf(t) < 16.0f ? q : t;
+    return fabsf(t) < 1024.0f ? q : t;
 }
 
 // The same code as quant_code(y, d.s): the IEEE quotient from a reciprocal multiply and
 // Markstein's correction (RowDivisor), rounded half to even by the conversion.  NaN
 // converts to 0 and +-inf saturates, as in quant_code.
 __device__ __forceinline__ int quant_code_fast(float y, const RowDivisor& d) {
-    if (!d.fast) return quant_code(y, d.s);
-    return min(max(__float2int_rn(quotient_fast(y, d.s, d.r)), -8), 7);
+    if (!d.fast) return quant_code(y, d.s, d.qmax);
+    return min(max(__float2int_rn(quotient_fast(y, d.s, d.r)), -d.qmax - 1), d.qmax);
 }
 
 // Sixteen codes of one row (divisor d) packed four per word, first code lowest: the
@@ -364,16 +439,16 @@ __device__ __forceinline__ void quant16(const float (&y)[16], const RowDivisor& 
             const unsigned long long t = mul2s_rn(y2, d.r);
             const unsigned long long e = fma2_rn(t, ns, y2);
             const float2 qq = f2_unpack(fma2_rn(e, r2, t));
-            const float2 tt = f2_unpack(t);       // |t| >= 16: the code saturates by sign
-            q[i] = __float2int_rn(fabsf(tt.x) < 16.0f ? qq.x : tt.x);   // NaN -> 0
-            q[i + 1] = __float2int_rn(fabsf(tt.y) < 16.0f ? qq.y : tt.y);
+            const float2 tt = f2_unpack(t);       // |t| >= 1024: the code saturates by sign
+            q[i] = __float2int_rn(fabsf(tt.x) < 1024.0f ? qq.x : tt.x);   // NaN -> 0
+            q[i + 1] = __float2int_rn(fabsf(tt.y) < 1024.0f ? qq.y : tt.y);
         }
     } else {
 #pragma unroll
         for (int i = 0; i < 16; ++i) q[i] = __float2int_rn(__fdiv_rn(y[i], d.s));
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = min(max(q[i], -8), 7);
+    for (int i = 0; i < 16; ++i) q[i] = min(max(q[i], -d.qmax - 1), d.qmax);
 #pragma unroll
     for (int w = 0; w < 4; ++w) out[w] = pack4_codes(q[4 * w], q[4 * w + 1], q[4 * w + 2], q[4 * w + 3]);
 }
@@ -419,9 +494,9 @@ __device__ __forceinline__ unsigned long long fma2_rn(unsigned long long a, unsi
     return z;
 }
 
-// quant16 for a row whose scale came from its own absmax (s = max(amax / 7, FLT_MIN)), with
-// the input as eight fp32 pairs.  There every quotient satisfies |y / s| <= 7, so no code
-// needs the clamp, and adding 1.5 * 2^23 to the quotient rounds it to an integer (half to
+// quant16 for a row whose scale came from its own absmax (s = max(amax / qmax, FLT_MIN)), with
+// the input as eight fp32 pairs.  There every quotient satisfies |y / s| <= qmax <= 127, so no
+// code needs the clamp, and adding 1.5 * 2^23 to the quotient rounds it to an integer (half to
 // even) that sits in the low byte of the sum's bit pattern as a two's-complement code.
 // A row that is not `fast` (NaN, inf, tiny or huge scale) takes quant_code per element.
 __device__ __forceinline__ void quant16_dyn2(const unsigned long long (&y2)[8], const RowDivisor& d,
@@ -443,8 +518,8 @@ __device__ __forceinline__ void quant16_dyn2(const unsigned long long (&y2)[8], 
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const float2 y = f2_unpack(y2[i]);
-            u[2 * i] = (uint32_t)quant_code(y.x, d.s);
-            u[2 * i + 1] = (uint32_t)quant_code(y.y, d.s);
+            u[2 * i] = (uint32_t)quant_code(y.x, d.s, d.qmax);
+            u[2 * i + 1] = (uint32_t)quant_code(y.y, d.s, d.qmax);
         }
     }
 #pragma unroll

@@ -20,6 +20,8 @@
 //   rq_mma_kernel      bf16/fp16, g in {16, 64}, longer rows.  A TMA producer fills a ring of
 //                      row blocks; two groups of compute warps rotate them with mma.sync and
 //                      quantize from shared memory.
+//   rq_f32_g16_kernel  (ck_rq_f32.cu) fp32, g = 16, row-major or column-major: K split over
+//                      a cluster, FP64 tensor-core rotation, absmax over distributed shared memory.
 //   rq_generic_kernel  every dtype, g and stride: one row per CTA step, fp32 FFMA with R
 //                      in shared memory (or read through L1 when it does not fit).
 // The TMA-fed kernels store 16 codes at a time where the code rows are 16-byte aligned; the
@@ -102,8 +104,8 @@ __device__ __forceinline__ void store_codes4(int8_t* dst, float4 v, const RowDiv
     }
 }
 
-__device__ __forceinline__ float row_scale(float amax, const float* scale_in) {
-    float s = scale_in ? *scale_in : __fdiv_rn(amax, 7.0f);
+__device__ __forceinline__ float row_scale(float amax, const float* scale_in, int qmax) {
+    float s = scale_in ? *scale_in : __fdiv_rn(amax, (float)qmax);
     return (s < FLT_MIN) ? FLT_MIN : s;   // lower clamp; NaN stays NaN
 }
 
@@ -112,7 +114,7 @@ __global__ void __launch_bounds__(kGenThreads)
     rq_generic_kernel(const T* __restrict__ x, int64_t M, int64_t K, int64_t sm, int64_t sk,
                       const T* __restrict__ R, int g, int r_in_smem,
                       const float* __restrict__ scale_in, int8_t* __restrict__ codes, int64_t ldq,
-                      float* __restrict__ scales, int vec_codes) {
+                      float* __restrict__ scales, int vec_codes, int qmax) {
     extern __shared__ __align__(16) unsigned char gen_smem[];
     float* xs = reinterpret_cast<float*>(gen_smem);
     T* Rs = reinterpret_cast<T*>(xs + K);
@@ -150,9 +152,9 @@ __global__ void __launch_bounds__(kGenThreads)
         __syncthreads();
         float amax = 0.f;
         for (int w = 0; w < kGenThreads / 32; ++w) amax = fmax_nan(amax, warp_max[w]);
-        const float s = row_scale(amax, scale_in);
+        const float s = row_scale(amax, scale_in, qmax);
         if (tid == 0) scales[m] = s;
-        const RowDivisor dv(s);
+        const RowDivisor dv(s, qmax);
 
         int8_t* qr = codes + m * ldq;
         if (kKeep) {
@@ -272,6 +274,7 @@ struct RqMmaParams {
     uint32_t box_bytes;   // bytes one box copy delivers
     uint32_t stage_bytes; // bytes of one ring stage (NB boxes)
     int vec_codes;
+    int qmax;             // code grid [-qmax - 1, qmax]
 };
 
 constexpr int kRqMaxStages = 8;
@@ -441,8 +444,8 @@ __global__ void __launch_bounds__(kRqThreads, 1)
             // ---- row scales (the group's first warp), published through scale_ready
             if (gw == 0) {
                 if (lane < p.RB) {
-                    const float sc = row_scale(__uint_as_float(amax_bits[s][lane]), scale_in);
-                    const RowDivisor dv(sc);
+                    const float sc = row_scale(__uint_as_float(amax_bits[s][lane]), scale_in, p.qmax);
+                    const RowDivisor dv(sc, p.qmax);
                     row_s[s][lane] = sc;
                     row_r[s][lane] = dv.r;
                     amax_bits[s][lane] = 0u;     // ready for the stage's next block
@@ -456,7 +459,7 @@ __global__ void __launch_bounds__(kRqThreads, 1)
             // ---- quantize: 16 consecutive channels per thread step, 16-byte code stores
             for (int r = 0; r < p.RB; ++r) {
                 if (m0 + r >= p.M) break;
-                RowDivisor dv(row_s[s][r]);
+                RowDivisor dv(row_s[s][r], p.qmax);
                 dv.r = row_r[s][r];
                 int8_t* dst_row = codes + (m0 + r) * p.ldq;
                 for (int c = gtid; c < chunks_per_row; c += kRqGroupWarps * 32) {
@@ -520,6 +523,7 @@ struct RqRowParams {
     uint32_t buf_bytes;   // one row buffer (a multiple of 1024 bytes)
     uint32_t box_bytes;   // bytes one box delivers
     int vec_codes;
+    int qmax;             // code grid [-qmax - 1, qmax]
 };
 
 template <typename T, int G, bool DYN>
@@ -665,9 +669,9 @@ __global__ void __launch_bounds__(kRowMaxWarps * 32, 1)
             float mx = fmax_nan(mf.x, mf.y);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            const float sc = row_scale(mx, DYN ? nullptr : scale_in);
+            const float sc = row_scale(mx, DYN ? nullptr : scale_in, p.qmax);
             if (lane == 0) scales[row] = sc;
-            const RowDivisor dv(sc);
+            const RowDivisor dv(sc, p.qmax);
             __syncwarp();   // the warp's stmatrix results are visible to all its lanes
 
             // ---- quantize: 16 consecutive channels per lane step, 16-byte code stores
@@ -725,7 +729,8 @@ __global__ void __launch_bounds__(kRowMaxWarps * 32, 1)
 template <typename T, int G>
 static ck_status launch_row(const void* x, int64_t M, int64_t K, int64_t sm, const void* R,
                             const float* scale_in, int8_t* codes, int64_t ldq, float* scales,
-                            int* dev_status, cudaStream_t stream, CUtensorMapDataType tdt) {
+                            int qmax, int* dev_status, cudaStream_t stream,
+                            CUtensorMapDataType tdt) {
     RqRowParams p;
     p.M = M;
     p.K = K;
@@ -747,6 +752,7 @@ static ck_status launch_row(const void* x, int64_t M, int64_t K, int64_t sm, con
     p.buf_bytes = (uint32_t)buf;
     p.box_bytes = (uint32_t)(G * 2 * p.GB);
     p.vec_codes = (aligned(codes, 16) && ldq % 16 == 0) ? 1 : 0;
+    p.qmax = qmax;
 
     CUtensorMap map;
     const uint64_t dims[3] = {(uint64_t)G, (uint64_t)p.GR, (uint64_t)M};
@@ -816,6 +822,7 @@ struct RqTcParams {
     uint32_t box_bytes;
     uint32_t idesc;
     int vec_codes;
+    int qmax;          // code grid [-qmax - 1, qmax]
 };
 
 template <typename T, bool DYN>
@@ -845,7 +852,9 @@ __device__ __forceinline__ void tc_quant_store(const uint32_t (&yp)[8], const Ro
     }
 }
 
-template <typename T, int G, bool DYN>
+// RG = G: R is the g x g rotation.  RG = 16 < G = 64: the rotation of g = 16 done as one of
+// g = 64 by the block-diagonal diag(R, R, R, R) (its zero blocks add exact zeros to each sum).
+template <typename T, int G, bool DYN, int RG = G>
 __global__ void __launch_bounds__(kTcThreads, 1)
     rq_tc_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ R,
                  const float* __restrict__ scale_in, int8_t* __restrict__ codes,
@@ -897,6 +906,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // loads rows k0 .. k0 + 7 of R at columns n0 .. n0 + 7 (16 bytes each), transposes them in
     // registers and stores the 16-byte chunks of rows n0 .. n0 + 7 of R^T.  Consecutive
     // threads take consecutive k0, so a warp's stores cover distinct swizzled chunks.
+    if constexpr (RG != G) {
+        // block-diagonal R: R^T[n][k] = R[k % RG][n % RG] inside the diagonal blocks, 0 outside
+        for (int i = tid; i < G * G; i += kTcThreads) {
+            const int n = i / G, k = i % G;
+            const T v = (n / RG == k / RG) ? R[(k % RG) * RG + (n % RG)] : Elem<T>::from_f(0.f);
+            *reinterpret_cast<T*>(rt + tc_rt_off<G>(n, k)) = v;
+        }
+    } else
     for (int blk = tid; blk < (G / 8) * (G / 8); blk += kTcThreads) {
         const int k0 = (blk % (G / 8)) * 8, n0 = (blk / (G / 8)) * 8;
         uint32_t a[8][4];
@@ -1035,8 +1052,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 break;
             const unsigned int amax_bits = amax_sh[grp][slot][r];
             slot = slot == 2 ? 0 : slot + 1;
-            const float sc = row_scale(__uint_as_float(amax_bits), DYN ? nullptr : scale_in);
-            const RowDivisor dv(sc);
+            const float sc = row_scale(__uint_as_float(amax_bits), DYN ? nullptr : scale_in, p.qmax);
+            const RowDivisor dv(sc, p.qmax);
             if (row_ok && rho == 0 && h == 0) scales[row] = sc;
             int8_t* dst = codes + row * p.ldq + rho * G + h * kCols;
             if constexpr (kCols == 64) {
@@ -1081,10 +1098,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 // Tensor-core kernel for bf16/fp16, g in {64, 256}, K / g <= 128.  Returns
 // CK_ERR_UNSUPPORTED otherwise.
-template <typename T, int G>
+template <typename T, int G, int RG = G>
 static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, const void* R,
                            const float* scale_in, int8_t* codes, int64_t ldq, float* scales,
-                           int* dev_status, cudaStream_t stream, CUtensorMapDataType tdt) {
+                           int qmax, int* dev_status, cudaStream_t stream,
+                           CUtensorMapDataType tdt) {
     RqTcParams p;
     p.M = M;
     p.K = K;
@@ -1098,6 +1116,7 @@ static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, cons
     p.box_bytes = (uint32_t)(p.RB * p.GR * 128);
     p.idesc = idesc_f16(128, G, std::is_same<T, __nv_bfloat16>::value);
     p.vec_codes = (aligned(codes, 16) && ldq % 16 == 0) ? 1 : 0;
+    p.qmax = qmax;
 
     // x as (channel within group, group, row); each box is 64 channels (128 bytes) of every
     // group of RB rows, fetched at channel offsets 0, 64, .. G - 64
@@ -1118,7 +1137,7 @@ static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, cons
                                                  scales, p, dev_status);
         return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
     };
-    return scale_in ? run(rq_tc_kernel<T, G, false>) : run(rq_tc_kernel<T, G, true>);
+    return scale_in ? run(rq_tc_kernel<T, G, false, RG>) : run(rq_tc_kernel<T, G, true, RG>);
 }
 
 // ===================================================================== host launch
@@ -1126,7 +1145,8 @@ static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, cons
 template <typename T, int G>
 static ck_status launch_mma(const void* x, int64_t M, int64_t K, int64_t sm, const void* R,
                             const float* scale_in, int8_t* codes, int64_t ldq, float* scales,
-                            int* dev_status, cudaStream_t stream, CUtensorMapDataType tdt) {
+                            int qmax, int* dev_status, cudaStream_t stream,
+                            CUtensorMapDataType tdt) {
     RqMmaParams p;
     p.M = M;
     p.K = K;
@@ -1152,6 +1172,7 @@ static ck_status launch_mma(const void* x, int64_t M, int64_t K, int64_t sm, con
     if (p.S > kRqMaxStages) p.S = kRqMaxStages;
     if (p.S < 2) return CK_ERR_UNSUPPORTED;
     p.vec_codes = (aligned(codes, 16) && ldq % 16 == 0) ? 1 : 0;
+    p.qmax = qmax;
 
     CUtensorMap map;
     const uint64_t dims[3] = {(uint64_t)G, (uint64_t)p.Gn, (uint64_t)M};
@@ -1176,7 +1197,7 @@ static ck_status launch_mma(const void* x, int64_t M, int64_t K, int64_t sm, con
 template <typename T>
 static ck_status launch_generic(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
                                 const void* R, int g, const float* scale_in, int8_t* codes,
-                                int64_t ldq, float* scales, cudaStream_t stream) {
+                                int64_t ldq, float* scales, int qmax, cudaStream_t stream) {
     const size_t r_bytes = (size_t)g * g * sizeof(T);
     const size_t xs_bytes = (size_t)K * sizeof(float);
     const int r_in_smem = (xs_bytes + r_bytes <= 200 * 1024) ? 1 : 0;
@@ -1192,7 +1213,7 @@ static ck_status launch_generic(const void* x, int64_t M, int64_t K, int64_t sm,
             return CK_ERR_CUDA;
         kern<<<grid, kGenThreads, smem, stream>>>(static_cast<const T*>(x), M, K, sm, sk,
                                                   static_cast<const T*>(R), g, r_in_smem,
-                                                  scale_in, codes, ldq, scales, vec);
+                                                  scale_in, codes, ldq, scales, vec, qmax);
     } else {
         auto kern = rq_generic_kernel<T, false>;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -1200,73 +1221,65 @@ static ck_status launch_generic(const void* x, int64_t M, int64_t K, int64_t sm,
             return CK_ERR_CUDA;
         kern<<<grid, kGenThreads, smem, stream>>>(static_cast<const T*>(x), M, K, sm, sk,
                                                   static_cast<const T*>(R), g, r_in_smem,
-                                                  scale_in, codes, ldq, scales, vec);
+                                                  scale_in, codes, ldq, scales, vec, qmax);
     }
     return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 
 ck_status launch_rotate_quant(const void* x, ck_dtype dt, int64_t M, int64_t K, int64_t sm,
                               int64_t sk, const void* R, int g, const float* scale_in,
-                              int8_t* codes, int64_t ldq, float* scales, int* dev_status,
-                              cudaStream_t stream) {
+                              int8_t* codes, int64_t ldq, float* scales, int qmax,
+                              int* dev_status, cudaStream_t stream) {
     if (M == 0) return CK_OK;
-    const bool mma_ok = (dt == CK_BF16 || dt == CK_F16) && (g == 16 || g == 64) && sk == 1 &&
-                        aligned(x, 16) && sm % 8 == 0 && sm > 0 && M < (1LL << 31) &&
-                        K / g <= (1LL << 31);
-    const bool tc_ok = (dt == CK_BF16 || dt == CK_F16) && (g == 64 || g == 256) && sk == 1 &&
-                       aligned(x, 16) && aligned(R, 16) && sm % 8 == 0 && sm > 0 &&
-                       M < (1LL << 31);
+    const bool half16 = dt == CK_BF16 || dt == CK_F16;
+    const bool mma_ok = half16 && (g == 16 || g == 64) && sk == 1 && aligned(x, 16) && sm % 8 == 0 &&
+                        sm > 0 && M < (1LL << 31) && K / g <= (1LL << 31);
+    const bool tc_ok = half16 && (g == 64 || g == 256) && sk == 1 && aligned(x, 16) &&
+                       aligned(R, 16) && sm % 8 == 0 && sm > 0 && M < (1LL << 31);
+    const bool bf = dt == CK_BF16;
+    const CUtensorMapDataType tdt = bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+#define CK_RQ_ARGS x, M, K, sm, R, scale_in, codes, ldq, scales, qmax, dev_status, stream, tdt
     if (tc_ok) {
         ck_status st;
-        if (dt == CK_BF16)
-            st = g == 64 ? launch_tc<__nv_bfloat16, 64>(x, M, K, sm, R, scale_in, codes, ldq, scales,
-                                                         dev_status, stream,
-                                                         CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
-                         : launch_tc<__nv_bfloat16, 256>(x, M, K, sm, R, scale_in, codes, ldq, scales,
-                                                          dev_status, stream,
-                                                          CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+        if (bf)
+            st = g == 64 ? launch_tc<__nv_bfloat16, 64>(CK_RQ_ARGS) : launch_tc<__nv_bfloat16, 256>(CK_RQ_ARGS);
         else
-            st = g == 64 ? launch_tc<__half, 64>(x, M, K, sm, R, scale_in, codes, ldq, scales,
-                                                  dev_status, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)
-                         : launch_tc<__half, 256>(x, M, K, sm, R, scale_in, codes, ldq, scales,
-                                                   dev_status, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+            st = g == 64 ? launch_tc<__half, 64>(CK_RQ_ARGS) : launch_tc<__half, 256>(CK_RQ_ARGS);
+        if (st != CK_ERR_UNSUPPORTED) return st;
+    }
+    // g = 16 rows of whole 64-channel groups: the tensor-core kernel with a block-diagonal R
+    const bool tc16_ok = half16 && g == 16 && K % 64 == 0 && sk == 1 && aligned(x, 16) &&
+                         sm % 8 == 0 && sm > 0 && M < (1LL << 31);
+    if (tc16_ok) {
+        const ck_status st = bf ? launch_tc<__nv_bfloat16, 64, 16>(CK_RQ_ARGS)
+                                : launch_tc<__half, 64, 16>(CK_RQ_ARGS);
         if (st != CK_ERR_UNSUPPORTED) return st;
     }
     if (mma_ok) {
-        ck_status st = CK_ERR_UNSUPPORTED;
-        if (dt == CK_BF16)
-            st = g == 64 ? launch_row<__nv_bfloat16, 64>(x, M, K, sm, R, scale_in, codes, ldq, scales,
-                                                          dev_status, stream,
-                                                          CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
-                         : launch_row<__nv_bfloat16, 16>(x, M, K, sm, R, scale_in, codes, ldq, scales,
-                                                          dev_status, stream,
-                                                          CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+        ck_status st;
+        if (bf)
+            st = g == 64 ? launch_row<__nv_bfloat16, 64>(CK_RQ_ARGS) : launch_row<__nv_bfloat16, 16>(CK_RQ_ARGS);
         else
-            st = g == 64 ? launch_row<__half, 64>(x, M, K, sm, R, scale_in, codes, ldq, scales,
-                                                   dev_status, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)
-                         : launch_row<__half, 16>(x, M, K, sm, R, scale_in, codes, ldq, scales,
-                                                   dev_status, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+            st = g == 64 ? launch_row<__half, 64>(CK_RQ_ARGS) : launch_row<__half, 16>(CK_RQ_ARGS);
         if (st != CK_ERR_UNSUPPORTED) return st;
-        if (dt == CK_BF16)
-            return g == 64 ? launch_mma<__nv_bfloat16, 64>(x, M, K, sm, R, scale_in, codes, ldq,
-                                                           scales, dev_status, stream,
-                                                           CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
-                           : launch_mma<__nv_bfloat16, 16>(x, M, K, sm, R, scale_in, codes, ldq,
-                                                           scales, dev_status, stream,
-                                                           CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
-        return g == 64 ? launch_mma<__half, 64>(x, M, K, sm, R, scale_in, codes, ldq, scales,
-                                                dev_status, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)
-                       : launch_mma<__half, 16>(x, M, K, sm, R, scale_in, codes, ldq, scales,
-                                                dev_status, stream, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+        if (bf)
+            return g == 64 ? launch_mma<__nv_bfloat16, 64>(CK_RQ_ARGS) : launch_mma<__nv_bfloat16, 16>(CK_RQ_ARGS);
+        return g == 64 ? launch_mma<__half, 64>(CK_RQ_ARGS) : launch_mma<__half, 16>(CK_RQ_ARGS);
+    }
+#undef CK_RQ_ARGS
+    if (dt == CK_F32 && g == 16) {
+        const ck_status st = launch_rq_f32_g16(x, M, K, sm, sk, R, scale_in, codes, ldq, scales,
+                                               qmax, dev_status, stream);
+        if (st != CK_ERR_UNSUPPORTED) return st;
     }
     switch (dt) {
         case CK_F32:
-            return launch_generic<float>(x, M, K, sm, sk, R, g, scale_in, codes, ldq, scales, stream);
+            return launch_generic<float>(x, M, K, sm, sk, R, g, scale_in, codes, ldq, scales, qmax, stream);
         case CK_F16:
-            return launch_generic<__half>(x, M, K, sm, sk, R, g, scale_in, codes, ldq, scales, stream);
+            return launch_generic<__half>(x, M, K, sm, sk, R, g, scale_in, codes, ldq, scales, qmax, stream);
         case CK_BF16:
             return launch_generic<__nv_bfloat16>(x, M, K, sm, sk, R, g, scale_in, codes, ldq, scales,
-                                                 stream);
+                                                 qmax, stream);
         default:
             return CK_ERR_INVALID_ARG;
     }

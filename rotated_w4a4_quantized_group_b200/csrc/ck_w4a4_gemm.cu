@@ -45,6 +45,7 @@
 #include <stdint.h>
 
 #include "ck_device.cuh"
+#include "ck_gemm_common.cuh"
 #include "ck_internal.h"
 
 namespace ck {
@@ -56,7 +57,7 @@ constexpr int BNA_MAX = 192;             // activation rows per tile: MMA N
 constexpr int XS_MAX = 8;                // code super-stages in shared memory
 constexpr int G_MAX = 4;                 // k-blocks per super-stage
 constexpr int NB_MAX = 4;                // TMEM weight buffers (one super-stage each)
-constexpr int W_ST_MAX = 2 * G_MAX;      // packed-weight stages (one k-block each): 2G
+constexpr int W_ST_MAX = 2 * G_MAX;      // packed-weight k-block buffers: G per unpack set
 constexpr int ND = 16;                   // super-stage completion barriers (> XS_MAX + 1)
 constexpr uint32_t W_BYTES = BW * BK / 2;    // 8 KB
 constexpr uint32_t A_STAGE_COLS = BK / 4;    // 32 TMEM columns of 4 bytes per stage
@@ -78,8 +79,10 @@ static_assert(ND == 16 && ND > XS_MAX + 1, "completion barrier index and parity 
 }  // namespace gemm
 
 struct GemmParams {
-    int64_t M, N, ldo;
+    int64_t M, N;
     int num_kb;        // K blocks of BK
+    int nss;           // super-stages per tile: ceil(num_kb / G)
+    int box3d;         // 1: one TMA box per super-stage (K % BK == 0), 0: one per k-block
     int BNA;           // activation rows per tile (multiple of 16, <= BNA_MAX)
     int tiles_n;       // tiles along N (channels)
     int tiles;         // total tiles
@@ -90,95 +93,15 @@ struct GemmParams {
     const float* a_scale;
     const void* w_scale;
     const void* bias;
-    void* out;
+    OutSegs segs;      // where each channel's outputs go
     int* dev_status;
 };
 
-// Eight signed 4-bit codes of one packed word -> eight sign-extended bytes in k order (the
-// low nibble of byte i is k = 2i).  Per byte, a nibble x in [0, 15] becomes
-// ((x + 0x78) ^ 0x78): x for x < 8 and x + 240 (x - 16 as a signed byte) for x >= 8; the sum
-// stays below 0x100, so no carry crosses a byte.
-__device__ __forceinline__ void unpack_word_s(uint32_t w, uint32_t& o0, uint32_t& o1) {
-    const uint32_t lo = ((w & 0x0F0F0F0Fu) + 0x78787878u) ^ 0x78787878u;          // k even
-    const uint32_t hi = (((w >> 4) & 0x0F0F0F0Fu) + 0x78787878u) ^ 0x78787878u;   // k odd
-    o0 = __byte_perm(lo, hi, 0x5140);                                             // k0 k1 k2 k3
-    o1 = __byte_perm(lo, hi, 0x7362);                                             // k4 k5 k6 k7
-}
-
-// The same eight codes as the bytes 16 w: a signed nibble placed in the high half of a byte
-// reads as 16 times its value.
-__device__ __forceinline__ void unpack_word_x16(uint32_t w, uint32_t& o0, uint32_t& o1) {
-    const uint32_t lo = (w << 4) & 0xF0F0F0F0u;   // k even
-    const uint32_t hi = w & 0xF0F0F0F0u;          // k odd
-    o0 = __byte_perm(lo, hi, 0x5140);
-    o1 = __byte_perm(lo, hi, 0x7362);
-}
-
-// A ring position: slot index and the parity of the slot's current fill.
-struct RingPos {
-    uint32_t idx = 0, phase = 0;
-    __device__ __forceinline__ void step(uint32_t n) {
-        if (++idx == n) {
-            idx = 0;
-            phase ^= 1u;
-        }
-    }
-};
-
-template <typename T> __device__ __forceinline__ float load_scale(const void* p, int64_t i);
-template <> __device__ __forceinline__ float load_scale<float>(const void* p, int64_t i) {
-    return __ldg(static_cast<const float*>(p) + i);
-}
-template <> __device__ __forceinline__ float load_scale<__half>(const void* p, int64_t i) {
-    return __half2float(__ldg(static_cast<const __half*>(p) + i));
-}
-template <> __device__ __forceinline__ float load_scale<__nv_bfloat16>(const void* p, int64_t i) {
-    return __bfloat162float(__ldg(static_cast<const __nv_bfloat16*>(p) + i));
-}
-
-template <typename OutT> struct OutStore;
-template <> struct OutStore<float> {
-    __device__ static __forceinline__ void vec16(float* dst, const float* v) {
-#pragma unroll
-        for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-    }
-    __device__ static __forceinline__ void one(float* dst, float v) { *dst = v; }
-};
-template <> struct OutStore<__nv_bfloat16> {
-    __device__ static __forceinline__ void vec16(__nv_bfloat16* dst, const float* v) {
-#pragma unroll
-        for (int i = 0; i < 16; i += 8) {
-            uint32_t u[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                __nv_bfloat162 h = __floats2bfloat162_rn(v[i + 2 * j], v[i + 2 * j + 1]);
-                u[j] = *reinterpret_cast<uint32_t*>(&h);
-            }
-            *reinterpret_cast<uint4*>(dst + i) = make_uint4(u[0], u[1], u[2], u[3]);
-        }
-    }
-    __device__ static __forceinline__ void one(__nv_bfloat16* dst, float v) {
-        *dst = __float2bfloat16_rn(v);
-    }
-};
-template <> struct OutStore<__half> {
-    __device__ static __forceinline__ void vec16(__half* dst, const float* v) {
-#pragma unroll
-        for (int i = 0; i < 16; i += 8) {
-            uint32_t u[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                __half2 h = __floats2half2_rn(v[i + 2 * j], v[i + 2 * j + 1]);
-                u[j] = *reinterpret_cast<uint32_t*>(&h);
-            }
-            *reinterpret_cast<uint4*>(dst + i) = make_uint4(u[0], u[1], u[2], u[3]);
-        }
-    }
-    __device__ static __forceinline__ void one(__half* dst, float v) { *dst = __float2half_rn(v); }
-};
-
-template <typename OutT, typename ScaleT, bool X16>
+// W8: the W8A8 variant.  The weights are INT8 codes (N, K): TMA brings 128 rows x 128 bytes per
+// k-block (128-byte swizzle) into a ring slot next to the codes' slot of the same super-stage,
+// and the MMA reads them from shared memory as its A operand; no expansion, no tensor-memory
+// weight buffers, and both producers arrive on the slot's barrier.
+template <typename OutT, typename ScaleT, bool X16, bool W8>
 __global__ void __launch_bounds__(gemm::THREADS, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap xmap,
                      const __grid_constant__ CUtensorMap wmap, GemmParams p) {
@@ -188,29 +111,35 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         (reinterpret_cast<uintptr_t>(gemm_smem) + 1023) & ~uintptr_t(1023));
     // packed-weight stage of k-block it: it % 2G, so each unpack set has its own G stages and
     // waits for their fills in order
-    const uint32_t G = (uint32_t)p.G, XS = (uint32_t)p.xs, W_ST = 2u * G, NB = (uint32_t)p.nb;
+    const uint32_t G = (uint32_t)p.G, XS = (uint32_t)p.xs, NB = (uint32_t)p.nb;
     const uint32_t x_bytes = (uint32_t)p.BNA * BK;          // one k-block of codes
     const uint32_t xss_bytes = G * x_bytes;                  // one super-stage
     unsigned char* x_ring = smem;
-    unsigned char* w_ring = x_ring + (size_t)XS * xss_bytes;
+    unsigned char* w_ring = x_ring + (size_t)XS * xss_bytes;   // W8: XS slots of G k-blocks
+    constexpr uint32_t W8_BYTES = BW * BK;                      // one INT8 weight k-block, 16 KB
 
-    __shared__ __align__(8) uint64_t x_full[XS_MAX], w_full[W_ST_MAX], w_empty[W_ST_MAX];
+    __shared__ __align__(8) uint64_t x_full[XS_MAX], w_full[UNP_SETS], w_empty[UNP_SETS];
     __shared__ __align__(8) uint64_t a_full[NB_MAX], done[ND];
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // k-blocks this CTA runs (its tiles blockIdx.x, + gridDim.x, ... times num_kb), numbered
-    // 0.. across tiles; super-stage s holds k-blocks [s G, s G + G)
+    // super-stages this CTA runs: nss per tile (its tiles blockIdx.x, + gridDim.x, ...),
+    // numbered 0.. across tiles; super-stage ss is k-blocks [s G, s G + n_k) of local tile
+    // ss / nss, s = ss % nss, n_k = min(G, num_kb - s G)
     const uint32_t my_tiles =
         (uint32_t)((p.tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x);
-    const uint32_t my_kb = my_tiles * (uint32_t)p.num_kb;
-    const uint32_t my_ss = (my_kb + G - 1) / G;
+    const uint32_t nss = (uint32_t)p.nss;
+    const uint32_t my_ss = my_tiles * nss;
+    auto ss_nk = [&](uint32_t ss) -> uint32_t {
+        const uint32_t kb0 = (ss % nss) * G;
+        return ((uint32_t)p.num_kb - kb0) < G ? ((uint32_t)p.num_kb - kb0) : G;
+    };
 
     if (tid == 0) {
-        for (int s = 0; s < XS_MAX; ++s) mbar_init(&x_full[s], 1);
-        for (int s = 0; s < W_ST_MAX; ++s) {
+        for (int s = 0; s < XS_MAX; ++s) mbar_init(&x_full[s], W8 ? 2 : 1);
+        for (int s = 0; s < UNP_SETS; ++s) {
             mbar_init(&w_full[s], 1);
             mbar_init(&w_empty[s], UNP_SET_WARPS);
         }
@@ -244,25 +173,27 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
     if (warp == WARP_TMA_X) {
         // ---------------------------------------------------------------- codes producer
         if (lane == 0) {
-            uint32_t issued = 0;
-            uint32_t slot = 0, kb = 0;
-            int t = blockIdx.x;
+            uint32_t issued = 0, slot = 0;
             bool ok = true;
             for (uint32_t ss = 0; ok && ss < my_ss; ++ss) {
                 if (ss >= XS && !wait_done(ss - XS)) {
                     ok = false;
                     break;
                 }
-                const uint32_t n_k = (my_kb - ss * G) < G ? (my_kb - ss * G) : G;
+                const int t = (int)blockIdx.x + (int)(ss / nss) * (int)gridDim.x;
+                const int32_t m0 = (t / p.tiles_n) * p.BNA;
+                const int32_t kb0 = (int32_t)((ss % nss) * G);
+                const uint32_t n_k = ss_nk(ss);
                 unsigned char* dst = x_ring + (size_t)slot * xss_bytes;
-                mbar_arrive_expect_tx(&x_full[slot], n_k * x_bytes);
-                for (uint32_t j = 0; j < n_k; ++j) {
-                    const int32_t m0 = (t / p.tiles_n) * p.BNA;
-                    tma_load_2d(dst + (size_t)j * x_bytes, &xmap, &x_full[slot], (int)kb * BK, m0);
-                    if (++kb == (uint32_t)p.num_kb) {
-                        kb = 0;
-                        t += gridDim.x;
-                    }
+                if (p.box3d) {
+                    // one box of G k-blocks (those past K arrive as zeros and are not used)
+                    mbar_arrive_expect_tx(&x_full[slot], G * x_bytes);
+                    tma_load_3d(dst, &xmap, &x_full[slot], 0, m0, kb0);
+                } else {
+                    mbar_arrive_expect_tx(&x_full[slot], n_k * x_bytes);
+                    for (uint32_t j = 0; j < n_k; ++j)
+                        tma_load_2d(dst + (size_t)j * x_bytes, &xmap, &x_full[slot],
+                                    (kb0 + (int32_t)j) * BK, m0);
                 }
                 ++issued;
                 if (++slot == XS) slot = 0;
@@ -271,29 +202,70 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                 for (uint32_t j = issued > XS ? issued - XS : 0; j < issued; ++j)
                     mbar_wait(&x_full[j % XS], (j / XS) & 1u, nullptr, nullptr);
         }
-    } else if (warp == WARP_TMA_W) {
-        // ---------------------------------------------------------------- packed W producer
+    } else if (warp == WARP_TMA_W && W8) {
+        // ---------------------------------------------------------------- INT8 W producer
+        // super-stage ss fills weight slot ss % XS, on the codes' barrier of that slot
         if (lane == 0) {
-            uint32_t it = 0, issued = 0;
-            RingPos rw;
+            uint32_t issued = 0, slot = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x) {
-                const int32_t n0 = (t % p.tiles_n) * BW;
-                for (int kb = 0; kb < p.num_kb; ++kb, ++it, rw.step(W_ST)) {
-                    if (it >= W_ST && !mbar_wait(&w_empty[rw.idx], rw.phase ^ 1u, &abort_flag,
-                                                 p.dev_status)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&w_full[rw.idx], W_BYTES);
-                    tma_load_2d(w_ring + (size_t)rw.idx * W_BYTES, &wmap, &w_full[rw.idx],
-                                kb * (BK / 2), n0);
-                    ++issued;
+            for (uint32_t ss = 0; ok && ss < my_ss; ++ss) {
+                if (ss >= XS && !wait_done(ss - XS)) {
+                    ok = false;
+                    break;
                 }
+                const int t = (int)blockIdx.x + (int)(ss / nss) * (int)gridDim.x;
+                const int32_t n0 = (t % p.tiles_n) * BW;
+                const int32_t kb0 = (int32_t)((ss % nss) * G);
+                const uint32_t n_k = ss_nk(ss);
+                unsigned char* dst = w_ring + (size_t)slot * G * W8_BYTES;
+                if (p.box3d) {
+                    mbar_arrive_expect_tx(&x_full[slot], G * W8_BYTES);
+                    tma_load_3d(dst, &wmap, &x_full[slot], 0, n0, kb0);
+                } else {
+                    mbar_arrive_expect_tx(&x_full[slot], n_k * W8_BYTES);
+                    for (uint32_t j = 0; j < n_k; ++j)
+                        tma_load_2d(dst + (size_t)j * W8_BYTES, &wmap, &x_full[slot],
+                                    (kb0 + (int32_t)j) * BK, n0);
+                }
+                ++issued;
+                if (++slot == XS) slot = 0;
             }
             if (!ok)
-                for (uint32_t j = issued > W_ST ? issued - W_ST : 0; j < issued; ++j)
-                    mbar_wait(&w_full[j % W_ST], (j / W_ST) & 1u, nullptr, nullptr);
+                for (uint32_t j = issued > XS ? issued - XS : 0; j < issued; ++j)
+                    mbar_wait(&x_full[j % XS], (j / XS) & 1u, nullptr, nullptr);
+        }
+    } else if (warp == WARP_TMA_W) {
+        // ---------------------------------------------------------------- packed W producer
+        // super-stage ss fills the G k-block buffers of unpack set ss % 2 (fill ss / 2)
+        if (lane == 0) {
+            uint32_t issued = 0;
+            bool ok = true;
+            for (uint32_t ss = 0; ok && ss < my_ss; ++ss) {
+                const uint32_t set = ss & 1u;
+                if (ss >= UNP_SETS &&
+                    !mbar_wait(&w_empty[set], ((ss >> 1) - 1) & 1u, &abort_flag, p.dev_status)) {
+                    ok = false;
+                    break;
+                }
+                const int t = (int)blockIdx.x + (int)(ss / nss) * (int)gridDim.x;
+                const int32_t n0 = (t % p.tiles_n) * BW;
+                const int32_t kb0 = (int32_t)((ss % nss) * G);
+                const uint32_t n_k = ss_nk(ss);
+                unsigned char* dst = w_ring + (size_t)set * G * W_BYTES;
+                if (p.box3d) {
+                    mbar_arrive_expect_tx(&w_full[set], G * W_BYTES);
+                    tma_load_3d(dst, &wmap, &w_full[set], 0, n0, kb0);
+                } else {
+                    mbar_arrive_expect_tx(&w_full[set], n_k * W_BYTES);
+                    for (uint32_t j = 0; j < n_k; ++j)
+                        tma_load_2d(dst + (size_t)j * W_BYTES, &wmap, &w_full[set],
+                                    (kb0 + (int32_t)j) * (BK / 2), n0);
+                }
+                ++issued;
+            }
+            if (!ok)
+                for (uint32_t j = issued > UNP_SETS ? issued - UNP_SETS : 0; j < issued; ++j)
+                    mbar_wait(&w_full[j & 1u], (j >> 1) & 1u, nullptr, nullptr);
         }
     } else if (warp == WARP_MMA) {
         // ---------------------------------------------------------------- MMA issuer
@@ -302,47 +274,53 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
             // (s G + j) x_bytes later (start-address field counts 16-byte units)
             const uint64_t bdesc0 = smem_desc_k_sw128(smem_u32(x_ring));
             const uint32_t kstep = x_bytes >> 4;
-            uint32_t slot = 0, xphase = 0, kb = 0, lt = 0;
+            const uint64_t adesc0 = smem_desc_k_sw128(smem_u32(w_ring));   // W8 weights
+            uint32_t slot = 0, xphase = 0, lt = 0;
             RingPos rb;   // TMEM weight buffer of the super-stage
             bool ok = true;
             uint32_t d_tmem = tmem_base;
             for (uint32_t ss = 0; ok && ss < my_ss; ++ss, rb.step(NB)) {
                 if (!mbar_wait(&x_full[slot], xphase, &abort_flag, p.dev_status) ||
-                    !mbar_wait(&a_full[rb.idx], rb.phase, &abort_flag, p.dev_status)) {
+                    (!W8 && !mbar_wait(&a_full[rb.idx], rb.phase, &abort_flag, p.dev_status))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t n_k = (my_kb - ss * G) < G ? (my_kb - ss * G) : G;
+                const uint32_t kb0 = (ss % nss) * G;
+                const uint32_t n_k = ss_nk(ss);
                 const uint32_t a_ss = tmem_base + a_col0 + rb.idx * G * A_STAGE_COLS;
-                for (uint32_t j = 0; j < n_k; ++j) {
-                    if (kb == 0) {
-                        // a new tile: its accumulator must have been drained by the epilogue
-                        const uint32_t acc = lt & 1u;
-                        if (lt >= 2 && !mbar_wait(&acc_empty[acc], ((lt >> 1) - 1) & 1u, &abort_flag,
-                                                  p.dev_status)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        d_tmem = tmem_base + acc * (uint32_t)p.BNA;
+                if (kb0 == 0) {
+                    // a new tile: its accumulator must have been drained by the epilogue
+                    const uint32_t acc = lt & 1u;
+                    if (lt >= 2 && !mbar_wait(&acc_empty[acc], ((lt >> 1) - 1) & 1u, &abort_flag,
+                                              p.dev_status)) {
+                        ok = false;
+                        break;
                     }
+                    tc_fence_after();
+                    d_tmem = tmem_base + acc * (uint32_t)p.BNA;
+                }
+                for (uint32_t j = 0; j < n_k; ++j) {
                     const uint64_t bdesc = bdesc0 + (uint64_t)((slot * G + j) * kstep);
                     const uint32_t a_tmem = a_ss + j * A_STAGE_COLS;
+                    const uint64_t adesc = adesc0 + (uint64_t)((slot * G + j) * (W8_BYTES >> 4));
 #pragma unroll
                     for (int kk = 0; kk < BK / 32; ++kk) {
-                        // one MMA K step: 32 bytes = 8 TMEM columns of A, 32 bytes of the
-                        // 128-byte swizzled B row
-                        tc_mma_i8_ts(d_tmem, a_tmem + (uint32_t)(kk * 8), bdesc + (uint64_t)(kk * 2),
-                                     p.idesc, (kb | (uint32_t)kk) != 0 ? 1u : 0u);
-                    }
-                    if (++kb == (uint32_t)p.num_kb) {
-                        tc_commit(&acc_full[lt & 1u]);
-                        kb = 0;
-                        ++lt;
+                        // one MMA K step: 32 bytes of K = 8 TMEM columns of A (or 32 bytes of
+                        // the 128-byte swizzled A row for W8), 32 bytes of the swizzled B row
+                        const uint32_t acc_flag = ((kb0 + j) | (uint32_t)kk) != 0 ? 1u : 0u;
+                        if (W8)
+                            tc_mma_i8(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2),
+                                      p.idesc, acc_flag);
+                        else
+                            tc_mma_i8_ts(d_tmem, a_tmem + (uint32_t)(kk * 8),
+                                         bdesc + (uint64_t)(kk * 2), p.idesc, acc_flag);
                     }
                 }
-                if (!ok) break;
+                if (kb0 + n_k == (uint32_t)p.num_kb) {
+                    tc_commit(&acc_full[lt & 1u]);
+                    ++lt;
+                }
                 tc_commit(&done[ss & (ND - 1)]);
                 if (++slot == XS) {
                     slot = 0;
@@ -353,7 +331,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
             tc_commit(&drain_bar);
             mbar_wait(&drain_bar, 0, nullptr, p.dev_status);
         }
-    } else if (warp >= UNP_WARP0 && warp < UNP_WARP0 + UNP_WARPS) {
+    } else if (!W8 && warp >= UNP_WARP0 && warp < UNP_WARP0 + UNP_WARPS) {
         // ---------------------------------------------------------------- unpack into TMEM
         const int u = warp - UNP_WARP0;
         const int q = warp & 3;                        // TMEM lanes 32q .. 32q + 31
@@ -368,37 +346,44 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + a_col0 + (uint32_t)(h * 16);
         bool ok = true;
         uint32_t buf = set;   // TMEM weight buffer of super-stage ss: ss % NB
+        const unsigned char* wset = w_ring + (size_t)set * G * W_BYTES;
         for (uint32_t ss = set; ok && ss < my_ss; ss += UNP_SETS) {
             // the buffer is free once the MMAs of its previous super-stage (ss - NB) completed
             if (ss >= NB && !__all_sync(0xffffffffu, wait_done(ss - NB))) break;
             tc_fence_after();
             const uint32_t t_buf = t_row + buf * G * A_STAGE_COLS;
-            const uint32_t it0 = ss * G;
-            const uint32_t n_k = (my_kb - it0) < G ? (my_kb - it0) : G;
-            for (uint32_t j = 0; j < n_k; ++j) {
-                // k-block it0 + j: W stage (it0 + j) % 2G = set G + j, fill (it0 + j) / 2G = ss / 2
-                const uint32_t sw = set * G + j;
-                // every lane waits; the warp leaves together (tcgen05.st below is .aligned)
-                if (!__all_sync(0xffffffffu, mbar_wait(&w_full[sw], (ss >> 1) & 1u, &abort_flag,
-                                                       p.dev_status))) {
-                    ok = false;
-                    break;
-                }
-                const unsigned char* wst = w_ring + (size_t)sw * W_BYTES;
-                const uint4 c0 = *reinterpret_cast<const uint4*>(wst + off0);
-                const uint4 c1 = *reinterpret_cast<const uint4*>(wst + off1);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&w_empty[sw]);
-                uint32_t v[16];
-                const uint32_t c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    if (X16) unpack_word_x16(c[i], v[2 * i], v[2 * i + 1]);
-                    else unpack_word_s(c[i], v[2 * i], v[2 * i + 1]);
-                }
-                tc_st_32x32b_x16(t_buf + j * A_STAGE_COLS, v);
+            const uint32_t n_k = ss_nk(ss);
+            // every lane waits; the warp leaves together (tcgen05.st below is .aligned)
+            if (!__all_sync(0xffffffffu, mbar_wait(&w_full[set], (ss >> 1) & 1u, &abort_flag,
+                                                   p.dev_status))) {
+                ok = false;
+                break;
             }
-            if (!ok) break;
+            uint4 c0[G_MAX], c1[G_MAX];
+#pragma unroll
+            for (uint32_t j = 0; j < (uint32_t)G_MAX; ++j) {
+                if (j < n_k) {
+                    const unsigned char* wst = wset + (size_t)j * W_BYTES;
+                    c0[j] = *reinterpret_cast<const uint4*>(wst + off0);
+                    c1[j] = *reinterpret_cast<const uint4*>(wst + off1);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&w_empty[set]);
+#pragma unroll
+            for (uint32_t j = 0; j < (uint32_t)G_MAX; ++j) {
+                if (j < n_k) {
+                    uint32_t v[16];
+                    const uint32_t c[8] = {c0[j].x, c0[j].y, c0[j].z, c0[j].w,
+                                           c1[j].x, c1[j].y, c1[j].z, c1[j].w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        if (X16) unpack_word_x16(c[i], v[2 * i], v[2 * i + 1]);
+                        else unpack_word_s(c[i], v[2 * i], v[2 * i + 1]);
+                    }
+                    tc_st_32x32b_x16(t_buf + j * A_STAGE_COLS, v);
+                }
+            }
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -406,6 +391,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
             buf += UNP_SETS;
             if (buf >= NB) buf -= NB;
         }
+        tc_wait_st();   // no tensor-memory store is pending when the CTA frees its columns
     } else if ((warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) || warp >= EPI_WARP1) {
         // ---------------------------------------------------------------- epilogue
         const int q = warp & 3;                        // TMEM lanes 32q .. 32q + 31
@@ -430,7 +416,11 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                 break;
             tc_fence_after();
             const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + acc * (uint32_t)p.BNA;
-            OutT* ocol = static_cast<OutT*>(p.out) + (n_ok ? n : 0);
+            // the lane's channel's output segment
+            int sg = 0;
+            while (n_ok && sg + 1 < p.segs.n && n >= p.segs.start[sg + 1]) ++sg;
+            OutT* ocol = static_cast<OutT*>(p.segs.ptr[sg]) + (n_ok ? n - p.segs.start[sg] : 0);
+            const int64_t ldo = p.segs.ldo[sg];
 #pragma unroll
             for (int k = 0; k < BNA_MAX / 32; ++k) {
                 const int c0 = 32 * k + 16 * eh;       // first row of this warp's chunk
@@ -447,7 +437,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                             o = __fmul_rn(o, a_s);
                             o = __fmul_rn(o, ws);
                             if (p.bias) o = __fadd_rn(o, bs);
-                            if (n_ok) OutStore<OutT>::one(ocol + (m0 + c0 + j) * p.ldo, o);
+                            if (n_ok) OutStore<OutT>::one(ocol + (m0 + c0 + j) * ldo, o);
                         }
                     }
                 }
@@ -468,9 +458,11 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
 
 template <typename OutT, typename ScaleT>
 static ck_status launch_typed(const CUtensorMap& xmap, const CUtensorMap& wmap,
-                              const GemmParams& p, size_t smem, int grid, bool x16,
+                              const GemmParams& p, size_t smem, int grid, bool x16, bool w8,
                               cudaStream_t stream) {
-    auto kern = x16 ? w4a4_gemm_kernel<OutT, ScaleT, true> : w4a4_gemm_kernel<OutT, ScaleT, false>;
+    auto kern = w8 ? w4a4_gemm_kernel<OutT, ScaleT, false, true>
+                   : x16 ? w4a4_gemm_kernel<OutT, ScaleT, true, false>
+                         : w4a4_gemm_kernel<OutT, ScaleT, false, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return CK_ERR_CUDA;
@@ -480,13 +472,13 @@ static ck_status launch_typed(const CUtensorMap& xmap, const CUtensorMap& wmap,
 
 template <typename OutT>
 static ck_status launch_out(const CUtensorMap& xmap, const CUtensorMap& wmap, const GemmParams& p,
-                            size_t smem, int grid, bool x16, ck_dtype scale_dt,
+                            size_t smem, int grid, bool x16, bool w8, ck_dtype scale_dt,
                             cudaStream_t stream) {
     switch (scale_dt) {
-        case CK_F32: return launch_typed<OutT, float>(xmap, wmap, p, smem, grid, x16, stream);
-        case CK_F16: return launch_typed<OutT, __half>(xmap, wmap, p, smem, grid, x16, stream);
+        case CK_F32: return launch_typed<OutT, float>(xmap, wmap, p, smem, grid, x16, w8, stream);
+        case CK_F16: return launch_typed<OutT, __half>(xmap, wmap, p, smem, grid, x16, w8, stream);
         case CK_BF16:
-            return launch_typed<OutT, __nv_bfloat16>(xmap, wmap, p, smem, grid, x16, stream);
+            return launch_typed<OutT, __nv_bfloat16>(xmap, wmap, p, smem, grid, x16, w8, stream);
         default: return CK_ERR_INVALID_ARG;
     }
 }
@@ -510,71 +502,123 @@ static int choose_bna(int64_t M, int64_t N, int sms) {
     return best;
 }
 
-ck_status launch_w4a4_gemm(const int8_t* codes, int64_t ldq, const float* a_scale, int64_t M,
-                           int64_t K, const int8_t* w_packed, int64_t w_ld, int64_t N,
-                           const void* w_scale, ck_dtype scale_dt, const void* bias, void* out,
-                           ck_dtype out_dt, int64_t ldo, int* dev_status, cudaStream_t stream) {
+// The persistent GEMM for packed INT4 weights (w8 false, (N, K/2) bytes) or INT8 weights
+// (w8 true, (N, K) bytes); codes and weights with 16-byte-aligned rows.
+static ck_status launch_persistent(const int8_t* codes, int64_t ldq, const float* a_scale,
+                                   int64_t M, int64_t K, const int8_t* w, int64_t w_ld, int64_t N,
+                                   const void* w_scale, ck_dtype scale_dt, const void* bias,
+                                   const OutSegs& segs, ck_dtype out_dt, bool w8, int* dev_status,
+                                   cudaStream_t stream) {
     using namespace gemm;
-    if (M == 0 || N == 0) return CK_OK;
     const int sms = num_sms();
     GemmParams p;
     p.BNA = choose_bna(M, N, sms);
+    const bool box3d = K % BK == 0;
+    const int num_kb = (int)((K + BK - 1) / BK);
+    // weight bytes per row of one k-block: 64 packed (two codes a byte) or 128
+    const uint32_t wkb = w8 ? BK : BK / 2;
+    const CUtensorMapSwizzle wsw = w8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap xmap, wmap;
-    {
+    // with whole 128-byte k-blocks, one 3-D box fetches the G k-blocks of a super-stage:
+    // (byte of the k-block, row, k-block); otherwise one 2-D box per k-block, zero past K
+    const uint32_t G_box = 2;
+    if (box3d) {
+        const uint64_t dims[3] = {(uint64_t)BK, (uint64_t)M, (uint64_t)num_kb};
+        const uint64_t strides[2] = {(uint64_t)ldq, (uint64_t)BK};
+        const uint32_t box[3] = {BK, (uint32_t)p.BNA, G_box};
+        ck_status st = encode_tma(&xmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, codes, dims, strides,
+                                  box, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != CK_OK) return st;
+        const uint64_t wdims[3] = {(uint64_t)wkb, (uint64_t)N, (uint64_t)num_kb};
+        const uint64_t wstrides[2] = {(uint64_t)w_ld, (uint64_t)wkb};
+        const uint32_t wbox[3] = {wkb, BW, G_box};
+        st = encode_tma(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w, wdims, wstrides, wbox, wsw);
+        if (st != CK_OK) return st;
+    } else {
         const uint64_t dims[2] = {(uint64_t)K, (uint64_t)M};
         const uint64_t strides[1] = {(uint64_t)ldq};
         const uint32_t box[2] = {BK, (uint32_t)p.BNA};
         ck_status st = encode_tma(&xmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, dims, strides,
                                   box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (st != CK_OK) return st;
-    }
-    {
-        const uint64_t dims[2] = {(uint64_t)(K / 2), (uint64_t)N};
-        const uint64_t strides[1] = {(uint64_t)w_ld};
-        const uint32_t box[2] = {BK / 2, BW};
-        ck_status st = encode_tma(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w_packed, dims, strides,
-                                  box, CU_TENSOR_MAP_SWIZZLE_64B);
+        const uint64_t wdims[2] = {(uint64_t)(w8 ? K : K / 2), (uint64_t)N};
+        const uint64_t wstrides[1] = {(uint64_t)w_ld};
+        const uint32_t wbox[2] = {wkb, BW};
+        st = encode_tma(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w, wdims, wstrides, wbox, wsw);
         if (st != CK_OK) return st;
     }
     p.M = M;
     p.N = N;
-    p.ldo = ldo;
-    p.num_kb = (int)((K + BK - 1) / BK);
+    p.num_kb = num_kb;
+    p.box3d = box3d ? 1 : 0;
     p.tiles_n = (int)((N + BW - 1) / BW);
     const int64_t tiles = (int64_t)p.tiles_n * ((M + p.BNA - 1) / p.BNA);
     if (tiles >= (1LL << 31)) return CK_ERR_UNSUPPORTED;
     p.tiles = (int)tiles;
-    // TMEM: two accumulators of BNA columns; the rest holds the two weight buffers of G
-    // k-blocks (32 columns each)
-    // two k-blocks per super-stage and as many weight buffers as fit (2..4): the unpack of a
+    // TMEM: two accumulators of BNA columns; for packed weights the rest holds the weight
+    // buffers of G k-blocks (32 columns each), as many as fit (2..4): the unpack of a
     // super-stage may start once the MMAs of the super-stage nb before it completed
-    p.G = 2;
-    p.nb = (int)((TMEM_COLS - 2u * (uint32_t)p.BNA) / ((uint32_t)p.G * A_STAGE_COLS));
+    p.G = (int)G_box;   // the 3-D boxes above hold exactly one super-stage
+    p.nb = w8 ? 2 : (int)((TMEM_COLS - 2u * (uint32_t)p.BNA) / ((uint32_t)p.G * A_STAGE_COLS));
     if (p.nb > NB_MAX) p.nb = NB_MAX;
     if (p.nb < 2) return CK_ERR_UNSUPPORTED;
     const size_t xss_bytes = (size_t)p.G * p.BNA * BK;
-    const size_t w_ring_bytes = (size_t)2 * p.G * W_BYTES;
-    p.xs = (int)((SMEM_BUDGET - w_ring_bytes) / xss_bytes);
-    if (p.xs > XS_MAX) p.xs = XS_MAX;
+    size_t w_ring_bytes;
+    if (w8) {
+        // one INT8 weight super-stage per codes slot
+        const size_t wss = (size_t)p.G * BW * BK;
+        p.xs = (int)(SMEM_BUDGET / (xss_bytes + wss));
+        if (p.xs > XS_MAX) p.xs = XS_MAX;
+        w_ring_bytes = (size_t)p.xs * wss;
+    } else {
+        w_ring_bytes = (size_t)2 * p.G * W_BYTES;
+        p.xs = (int)((SMEM_BUDGET - w_ring_bytes) / xss_bytes);
+        if (p.xs > XS_MAX) p.xs = XS_MAX;
+    }
     if (p.G < 1 || p.xs < 2) return CK_ERR_UNSUPPORTED;
+    p.nss = (p.num_kb + p.G - 1) / p.G;
     const size_t smem = (size_t)p.xs * xss_bytes + w_ring_bytes + 1024;
-    // signed 8-bit A and B, s32 accumulator, 128 x BNA
-    p.idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(p.BNA >> 3) << 17) |
-              ((uint32_t)(BW >> 4) << 24);
+    p.idesc = idesc_i8(BW, p.BNA);   // signed 8-bit A and B, s32 accumulator, 128 x BNA
     p.a_scale = a_scale;
     p.w_scale = w_scale;
     p.bias = bias;
-    p.out = out;
+    p.segs = segs;
     p.dev_status = dev_status;
     const int grid = (int)(p.tiles < sms ? p.tiles : sms);
-    const bool x16 = K <= SCALED16_MAX_K;
+    const bool x16 = !w8 && K <= SCALED16_MAX_K;
     switch (out_dt) {
-        case CK_F32: return launch_out<float>(xmap, wmap, p, smem, grid, x16, scale_dt, stream);
-        case CK_F16: return launch_out<__half>(xmap, wmap, p, smem, grid, x16, scale_dt, stream);
+        case CK_F32: return launch_out<float>(xmap, wmap, p, smem, grid, x16, w8, scale_dt, stream);
+        case CK_F16: return launch_out<__half>(xmap, wmap, p, smem, grid, x16, w8, scale_dt, stream);
         case CK_BF16:
-            return launch_out<__nv_bfloat16>(xmap, wmap, p, smem, grid, x16, scale_dt, stream);
+            return launch_out<__nv_bfloat16>(xmap, wmap, p, smem, grid, x16, w8, scale_dt, stream);
         default: return CK_ERR_INVALID_ARG;
     }
+}
+
+ck_status launch_w4a4_gemm(const int8_t* codes, int64_t ldq, const float* a_scale, int64_t M,
+                           int64_t K, const int8_t* w_packed, int64_t w_ld, int64_t N,
+                           const void* w_scale, ck_dtype scale_dt, const void* bias,
+                           const OutSegs& segs, ck_dtype out_dt, int* dev_status,
+                           cudaStream_t stream) {
+    if (M == 0 || N == 0) return CK_OK;
+    if (M <= 64) {   // few rows: split K over clusters so the weights stream on every SM
+        const ck_status st = launch_w4a4_splitk(codes, ldq, a_scale, M, K, w_packed, w_ld, N,
+                                                w_scale, scale_dt, bias, segs, out_dt,
+                                                dev_status, stream);
+        if (st != CK_ERR_UNSUPPORTED) return st;
+    }
+    return launch_persistent(codes, ldq, a_scale, M, K, w_packed, w_ld, N, w_scale, scale_dt,
+                             bias, segs, out_dt, false, dev_status, stream);
+}
+
+ck_status launch_w8a8_gemm(const int8_t* codes, int64_t ldq, const float* a_scale, int64_t M,
+                           int64_t K, const int8_t* w, int64_t w_ld, int64_t N,
+                           const void* w_scale, ck_dtype scale_dt, const void* bias,
+                           const OutSegs& segs, ck_dtype out_dt, int* dev_status,
+                           cudaStream_t stream) {
+    if (M == 0 || N == 0) return CK_OK;
+    return launch_persistent(codes, ldq, a_scale, M, K, w, w_ld, N, w_scale, scale_dt, bias, segs,
+                             out_dt, true, dev_status, stream);
 }
 
 }  // namespace ck

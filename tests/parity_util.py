@@ -122,8 +122,13 @@ def _abs_terms(x_rows: np.ndarray, R: np.ndarray, g: int, ks: np.ndarray, r_idx:
 
 def compare_stage1(gc: np.ndarray, gs: np.ndarray, oc: np.ndarray, os_: np.ndarray, dtype,
                    what: str = "", g: int = 256, *, x: torch.Tensor | None = None,
-                   R: torch.Tensor | None = None, rows=None, scale_in: float | None = None):
+                   R: torch.Tensor | None = None, rows=None, scale_in: float | None = None,
+                   qmax: int = 7, max_rate: float = CODE_MISMATCH_MAX):
     """GPU vs oracle codes/scales for the same rows; returns the code mismatch count.
+
+    qmax 127 (the W8A8 variant's INT8 grid) keeps every bound; only the mismatch rate limit,
+    max_rate, is the caller's: with 16-bit inputs one dtype ulp of y moves the INT8 quotient
+    by up to 127 * 2^-7 ~ 1, so the rate follows the rotation's rounding flips.
 
     Every mismatched code must sit at a rounding tie: x and R (the inputs, CPU) and rows
     (which rows of x the arrays hold; all rows when None) let the check recompute the
@@ -133,7 +138,7 @@ def compare_stage1(gc: np.ndarray, gs: np.ndarray, oc: np.ndarray, os_: np.ndarr
     diff = gc - oc
     assert np.abs(diff).max(initial=0) <= 1, f"{what}: a code differs by more than 1"
     rate = float((diff != 0).mean()) if diff.size else 0.0
-    assert rate <= CODE_MISMATCH_MAX, f"{what}: code mismatch rate {rate:.3g}"
+    assert rate <= max_rate, f"{what}: code mismatch rate {rate:.3g}"
     finite = np.isfinite(os_)
     np.testing.assert_array_equal(np.isfinite(gs), finite, err_msg=what)
     rel = np.abs(gs[finite].astype(np.float64) - os_[finite]) / os_[finite]
@@ -174,6 +179,12 @@ def oracle_on_codes(codes: np.ndarray, scales: np.ndarray, w_packed_cpu: torch.T
 
 def output_widening(gc: np.ndarray, oc: np.ndarray, gs: np.ndarray, os_: np.ndarray,
                     w_packed_cpu: torch.Tensor, K: int, cols, w_scale_cpu) -> np.ndarray:
+    w = oracle.unpack_w4(w_packed_cpu[cols], K).astype(np.int64)
+    return widening_for_weights(gc, oc, gs, os_, w, w_scale_cpu[torch.as_tensor(cols)])
+
+
+def widening_for_weights(gc: np.ndarray, oc: np.ndarray, gs: np.ndarray, os_: np.ndarray,
+                         w: np.ndarray, w_scale_cols) -> np.ndarray:
     """(rows, cols) bound on |out_gpu - out_oracle| that the stage-1 differences the parity
     rule allows can cause, beyond the output rounding that rtol covers.
 
@@ -185,8 +196,8 @@ def output_widening(gc: np.ndarray, oc: np.ndarray, gs: np.ndarray, os_: np.ndar
     A row whose codes and scale both equal the oracle's gives an identical output (0)."""
     g32 = gc.astype(np.int32)
     o32 = oc.astype(np.int32)
-    mis = (g32 != o32).astype(np.int64)
-    w = oracle.unpack_w4(w_packed_cpu[cols], K).astype(np.int64)
+    mis = (g32 != o32).astype(np.int64) * np.abs(g32 - o32)
+    w = np.asarray(w, dtype=np.int64)
     dacc = (mis @ np.abs(w).T).astype(np.float64)
     acc = np.abs((o32.astype(np.int64) @ w.T).astype(np.float64))
     ag = np.abs(gs.astype(np.float64))
@@ -194,7 +205,7 @@ def output_widening(gc: np.ndarray, oc: np.ndarray, gs: np.ndarray, os_: np.ndar
     amax = np.maximum(ag, ao)[:, None]
     da = np.abs(gs.astype(np.float64) - os_.astype(np.float64))[:, None]
     differs = (mis.any(axis=1) | (gs != os_))[:, None]
-    ws = np.abs(w_scale_cpu[torch.as_tensor(cols)].to(torch.float64).numpy())[None, :]
+    ws = np.abs(torch.as_tensor(w_scale_cols).to(torch.float64).numpy())[None, :]
     extra = ws * (dacc * amax + acc * da + differs * 4.0 * 2.0 ** -24 * (acc + dacc) * amax)
     return extra * 1.01
 

@@ -151,3 +151,85 @@ def test_binding_refuses_host_tensors(L):
         ck.ck_rotate_quant(x, R, 64)
     with pytest.raises(ValueError, match="CUDA device"):
         ck.ck_unpack_w4(torch.zeros(4, 32, dtype=torch.int8), 64)
+
+
+def grouped(L, **kw):
+    a = dict(x=1 << 20, dt=ck.CK_BF16, M=4, K=64, sm=64, sk=1, R=1 << 20, g=16, a_scale=NULL,
+             w=1 << 20, w_ld=32, w_scale=1 << 20, sdt=ck.CK_BF16, bias=NULL, G=2,
+             gn=[8, 8], outs=[1 << 20, 1 << 21], ldos=[8, 8], odt=ck.CK_BF16, ws=1 << 20,
+             ws_bytes=1 << 20)
+    a.update(kw)
+    G = len(a["gn"])
+    gn = (ctypes.c_int64 * max(G, 1))(*a["gn"])
+    outs = (ctypes.c_void_p * max(G, 1))(*a["outs"])
+    ldos = (ctypes.c_int64 * max(G, 1))(*a["ldos"])
+    return L.ck_w4a4_grouped_linear(a["x"], a["dt"], a["M"], a["K"], a["sm"], a["sk"], a["R"],
+                                    a["g"], a["a_scale"], a["w"], a["w_ld"], a["w_scale"], a["sdt"],
+                                    a["bias"], a["G"], gn, outs, ldos, a["odt"], a["ws"],
+                                    a["ws_bytes"], None, None)
+
+
+@pytest.mark.parametrize("bad", [dict(G=0), dict(G=9, gn=[1] * 9, outs=[1 << 20] * 9, ldos=[1] * 9),
+                                 dict(gn=[8, -1]), dict(ldos=[8, 7]), dict(outs=[1 << 20, None]),
+                                 dict(K=63), dict(g=8), dict(w_ld=31), dict(sdt=ck.CK_I8)])
+def test_grouped_linear_rejects_on_host(L, bad):
+    assert grouped(L, **bad) == ck.CK_ERR_INVALID_ARG
+
+
+def test_grouped_linear_empty_group_and_empty_rows(L):
+    # an empty group needs no output pointer; M = 0 is a no-op
+    assert grouped(L, M=0, x=NULL, outs=[None, None], ws=NULL, ws_bytes=0) == ck.CK_OK
+    assert grouped(L, gn=[0, 0], outs=[None, None], ldos=[0, 0], ws=NULL, ws_bytes=0) == ck.CK_OK
+
+
+def test_grouped_linear_missing_workspace(L):
+    assert grouped(L, ws=NULL, ws_bytes=0) == ck.CK_ERR_WORKSPACE
+
+
+def w8(L, **kw):
+    a = dict(x=1 << 20, dt=ck.CK_BF16, M=4, K=64, sm=64, sk=1, R=1 << 20, g=16, a_scale=NULL,
+             w=1 << 20, N=8, w_ld=64, w_scale=1 << 20, sdt=ck.CK_BF16, bias=NULL, out=1 << 20,
+             odt=ck.CK_BF16, ldo=8, ws=1 << 20, ws_bytes=1 << 20)
+    a.update(kw)
+    return L.ck_w8a8_linear(a["x"], a["dt"], a["M"], a["K"], a["sm"], a["sk"], a["R"], a["g"],
+                            a["a_scale"], a["w"], a["N"], a["w_ld"], a["w_scale"], a["sdt"],
+                            a["bias"], a["out"], a["odt"], a["ldo"], a["ws"], a["ws_bytes"],
+                            None, None)
+
+
+@pytest.mark.parametrize("bad", [dict(w_ld=63), dict(K=63), dict(g=8), dict(ldo=7), dict(out=NULL),
+                                 dict(dt=ck.CK_I8, a_scale=NULL), dict(sdt=ck.CK_I8)])
+def test_w8a8_linear_rejects_on_host(L, bad):
+    assert w8(L, **bad) == ck.CK_ERR_INVALID_ARG
+
+
+def test_w8a8_overflow_guard_is_the_int8_bound(L):
+    """|acc| <= 128 * 128 * K: K = 131071 passes the guard, 131072 does not."""
+    K = 131072
+    assert w8(L, dt=ck.CK_I8, K=K, sm=K, w_ld=K, a_scale=1 << 20) == ck.CK_ERR_OVERFLOW
+    assert w8(L, dt=ck.CK_I8, K=K - 2, sm=K, w_ld=K, a_scale=1 << 20, ws=NULL,
+              ws_bytes=0) != ck.CK_ERR_OVERFLOW
+
+
+def test_w8a8_workspace_sizes(L):
+    assert L.ck_w8a8_linear_workspace_bytes(8192, 3840, 3840, 3840) == \
+        ck.workspace_bytes(8192, 3840, 3840, 1920)
+    # an unaligned INT8 weight pitch needs room for a 16-byte-pitched (N, K) copy
+    assert L.ck_w8a8_linear_workspace_bytes(7, 5, 48, 50) >= \
+        L.ck_w8a8_linear_workspace_bytes(7, 5, 48, 48) + 5 * 48
+    assert L.ck_w8a8_linear_workspace_bytes(7, 5, 48, 47) == 0
+
+
+def test_rotate_quant_int8_rejects_like_stage_1(L):
+    assert L.ck_rotate_quant_int8(1 << 20, ck.CK_BF16, 4, 64, 64, 1, 1 << 20, 32, None, 1 << 20,
+                                  64, 1 << 20, None, None) == ck.CK_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("bad", [dict(K=62, g=2), dict(K=63), dict(g=32), dict(ldp=31), dict(sr=2),
+                                 dict(x=NULL), dict(p=NULL), dict(s=NULL), dict(dt=ck.CK_I8)])
+def test_packed_quantizer_rejects_on_host(L, bad):
+    a = dict(x=1 << 20, dt=ck.CK_BF16, M=4, K=64, g=16, sr=1, p=1 << 20, ldp=32, s=1 << 20)
+    a.update(bad)
+    assert L.ck_rotate_quant_packed(a["x"], a["dt"], a["M"], a["K"], a["K"], 1, 1 << 20, a["g"],
+                                    None, a["sr"], 7, 0, a["p"], a["ldp"], a["s"], None) == \
+        ck.CK_ERR_INVALID_ARG

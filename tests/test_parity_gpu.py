@@ -14,6 +14,7 @@ import torch
 
 import oracle
 from parity_util import (assert_close, compare_stage1, oracle_on_codes, output_widening,
+                         widening_for_weights,
                          sample_cols, sample_rows, to_device, workspace_stage1)
 from rotated_w4a4_quantized_group_b200 import ck
 from rotated_w4a4_quantized_group_b200 import workloads as W
@@ -466,3 +467,407 @@ def test_quantizer_caller_scale_extremes_with_identity_rotation(dt, g):
         oc, os_ = oracle.rotate_quant(xs, R, g, scale_in=float(scale))
         np.testing.assert_array_equal(scales.cpu().numpy(), os_)
         np.testing.assert_array_equal(codes.cpu().numpy(), oc)
+
+
+# ------------------------------------------------------------------- fp32, g = 16 (fp64 sums)
+
+def _colmajor(x: torch.Tensor, pad: int = 0) -> torch.Tensor:
+    """x (M, K) as the transposed view of a (K, M + pad) row-major buffer."""
+    M, K = x.shape
+    buf = torch.zeros(K, M + pad, dtype=x.dtype)
+    buf[:, :M] = x.t()
+    return buf[:, :M].t()
+
+
+@pytest.mark.parametrize("layout,M,K,pad", [("col", 16, 80, 0), ("col", 200, 464, 0),
+                                            ("col", 1000, 3840, 12), ("col", 300, 16384, 4),
+                                            ("col", 4096, 16384, 0), ("row", 1, 16, 0),
+                                            ("row", 37, 80, 0), ("row", 333, 3840, 0),
+                                            ("row", 129, 10240, 0), ("row", 20, 16384, 0),
+                                            ("row", 50, 32768, 0)])
+def test_rotate_quant_f32_g16_equals_the_oracle_bit_for_bit(layout, M, K, pad):
+    """fp32 input with g = 16 forms each rotated value as the in-order fp64 sum of its sixteen
+    exact products, rounded once to fp32, as the oracle does: codes and scales must equal the
+    oracle's exactly.  Column-major views (unit M stride, 16-byte column pitch, some padded)
+    and row-major rows from one group to 32768 channels, K split over a cluster where a block
+    does not fit one CTA; a non-symmetric R, outlier channels and zero rows."""
+    g = torch.Generator().manual_seed(M * 7 + K)
+    x = torch.randn(M, K, generator=g)
+    x[:, torch.randperm(K, generator=g)[: max(1, K // 100)]] *= 20.0
+    x[M // 3] = 0.0
+    if layout == "col":
+        x = _colmajor(x, pad)
+    elif pad:
+        x = torch.zeros(M, K + pad)[:, :K].copy_(x)
+    R = W.haar_orthogonal(16, torch.Generator().manual_seed(K)).float().contiguous()
+    codes, scales = ck.ck_rotate_quant(to_device(x), R.cuda(), 16)
+    torch.cuda.synchronize()
+    rows = sample_rows(M, 96) if M * K > 4_000_000 else np.arange(M)
+    oc, os_ = oracle.rotate_quant(x, R, 16, rows=rows)
+    idx = torch.from_numpy(rows).cuda()
+    np.testing.assert_array_equal(scales[idx].cpu().numpy(), os_)
+    np.testing.assert_array_equal(codes[idx].cpu().numpy(), oc)
+
+
+@pytest.mark.parametrize("layout", ["col", "row"])
+def test_rotate_quant_f32_g16_caller_scale_and_non_finite(layout):
+    M, K = 48, 256
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(M, K, generator=g)
+    x[2, 5] = float("nan")
+    x[7, 9] = float("inf")
+    xv = _colmajor(x) if layout == "col" else x
+    R = W.haar_orthogonal(16, torch.Generator().manual_seed(6)).float().contiguous()
+    codes, scales = ck.ck_rotate_quant(to_device(xv), R.cuda(), 16)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.rotate_quant(xv, R, 16)
+    np.testing.assert_array_equal(scales.cpu().numpy(), os_)
+    np.testing.assert_array_equal(codes.cpu().numpy(), oc)
+    s = torch.tensor([0.05], dtype=torch.float32)
+    codes, scales = ck.ck_rotate_quant(to_device(xv), R.cuda(), 16, scale_in=s.cuda())
+    torch.cuda.synchronize()
+    oc, os_ = oracle.rotate_quant(xv, R, 16, scale_in=0.05)
+    np.testing.assert_array_equal(scales.cpu().numpy(), os_)
+    np.testing.assert_array_equal(codes.cpu().numpy(), oc)
+
+
+def test_linear_f32_g16_colmajor_outputs_equal_the_oracle():
+    """The column-major fp32 workload at a size with 16-byte column pitch: stage 1 equals the
+    oracle exactly, so every output equals the whole oracle path bit for bit."""
+    case = W.LINEAR_CASES["krea_m4096_k16384_n6144_g16_f32_colmajor"].replace(M=400, N=300,
+                                                                            K=16 * 61)
+    inp = W.make_linear_inputs(case)
+    assert inp["x"].stride(0) == 1 and inp["x"].stride(1) % 4 == 0
+    out, ws = _run_linear(inp, case)
+    ref, oc, os_ = oracle.linear(inp["x"], inp["R"], case.g, inp["w_packed"], inp["w_scale"],
+                                 inp["bias"])
+    gcodes, gscales = workspace_stage1(ws, case.M, case.K)
+    np.testing.assert_array_equal(gcodes.cpu().numpy(), oc)
+    np.testing.assert_array_equal(gscales.cpu().numpy(), os_)
+    assert torch.equal(out.cpu().view(torch.int32), ref.view(torch.int32))
+
+
+# ------------------------------------------------------------------- few rows (split K)
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 128), (1, 3840, 3840), (7, 200, 448), (16, 6144, 16384),
+                                   (32, 3840, 3840), (33, 129, 10240), (64, 3840, 3840),
+                                   (64, 300, 48), (5, 1000, 1152)])
+def test_few_rows_gemm_accumulators_bit_exact(M, N, K):
+    """M <= 64 takes the split-K kernel (K split over a cluster, partial INT32 accumulators
+    summed through distributed shared memory): unit scales, fp32 out give the accumulator
+    exactly; then scales, bias and a 16-bit output against the oracle's epilogue."""
+    g = torch.Generator().manual_seed(M * 31 + N + K)
+    q = torch.randint(-8, 8, (M, K), generator=g, dtype=torch.int8)
+    q[0, : min(K, 64)] = -8
+    wp = torch.randint(-128, 128, (N, K // 2), generator=g, dtype=torch.int8)
+    wp[0] = -120                                          # every code of channel 0 is -8
+    out = ck.ck_w4a4_linear(q.cuda(), None, 0, wp.cuda(), torch.ones(N, device="cuda"),
+                            a_scale=torch.ones(M, device="cuda"), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    cols = sample_cols(N, 160)
+    acc = oracle.gemm_s32(q.numpy(), oracle.unpack_w4(wp[cols], K))
+    np.testing.assert_array_equal(out.cpu().numpy()[:, cols], acc.astype(np.float32))
+    a = torch.rand(M, generator=g) + 0.1
+    ws = (torch.rand(N, generator=g) * 0.015 + 0.005).to(torch.bfloat16)
+    b = torch.randn(N, generator=g).to(torch.bfloat16)
+    out2 = ck.ck_w4a4_linear(q.cuda(), None, 0, wp.cuda(), ws.cuda(), b.cuda(), a_scale=a.cuda(),
+                             out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    ref = oracle.epilogue(acc, a.numpy(), ws[cols], b[cols], torch.bfloat16)
+    assert torch.equal(out2.cpu()[:, torch.from_numpy(cols)], ref)
+
+
+@pytest.mark.parametrize("M", [1, 8, 16, 32])
+def test_few_rows_linear_every_output(M):
+    """The decode-sized linear (M = 1 to 32 rows of the Z-Image recipe, K = N = 3840) through
+    both stages, every output compared with the oracle."""
+    case = W.LINEAR_CASES["zimage_m32_k3840_n3840_g64_bf16"].replace(M=M, seed=100 + M)
+    _check_linear(case, np.arange(case.M), sample_cols(case.N, 512))
+
+
+# ------------------------------------------------------------------- grouped linear
+
+@pytest.mark.parametrize("M,groups,dt,bias", [(197, [128, 96, 200], "bf16", True),
+                                             (8192, [3840, 1024, 1024], "bf16", True),
+                                             (32, [3840, 3840, 3840], "bf16", True),
+                                             (300, [64, 1, 130, 7, 256], "f16", False),
+                                             (5, [200, 56], "f32", True)])
+def test_grouped_linear_equals_each_linear_and_the_oracle(M, groups, dt, bias):
+    """Q/K/V-style projections of one input: one stage 1, one GEMM over the stacked weights.
+    Each group's output must equal ck_w4a4_linear with that group's weights alone, bit for
+    bit, and the oracle applied to that group within the parity rule."""
+    K, g = 448 if M < 8192 else 3840, 64
+    base = W.LINEAR_CASES[W.HEADLINE]
+    case = base.replace(M=M, K=K, N=sum(groups), dtype=dt, has_bias=bias, seed=M + len(groups))
+    inp = W.make_linear_inputs(case)
+    x, R = inp["x"].cuda(), inp["R"].cuda()
+    parts, o = [], 0
+    for n in groups:
+        b = None if inp["bias"] is None else inp["bias"][o:o + n].cuda()
+        parts.append((inp["w_packed"][o:o + n].cuda(), inp["w_scale"][o:o + n].cuda(), b))
+        o += n
+    wp, wsc, bs, gn = ck.fuse_linear_weights(parts)
+    outs = ck.ck_w4a4_grouped_linear(x, R, g, wp, wsc, bs, gn)
+    singles = [ck.ck_w4a4_linear(x, R, g, p[0], p[1], p[2]) for p in parts]
+    torch.cuda.synchronize()
+    itype = torch.int32 if dt == "f32" else torch.int16
+    rows = sample_rows(M, 64)
+    o = 0
+    for i, n in enumerate(groups):
+        assert torch.equal(outs[i].view(itype), singles[i].view(itype)), f"group {i}"
+        cols = sample_cols(n, 96)
+        bi = None if inp["bias"] is None else inp["bias"][o:o + n]
+        ref, oc, os_ = oracle.linear(inp["x"], inp["R"], g, inp["w_packed"][o:o + n],
+                                     inp["w_scale"][o:o + n], bi, rows=rows, cols=cols)
+        got = outs[i].cpu()[torch.from_numpy(rows)][:, torch.from_numpy(cols)]
+        # the GPU's own codes for these rows: from a stage-1 call on the same input
+        gc, gs = ck.ck_rotate_quant(x, R, g)
+        gc = gc[torch.from_numpy(rows).cuda()].cpu().numpy()
+        gs = gs[torch.from_numpy(rows).cuda()].cpu().numpy()
+        compare_stage1(gc, gs, oc, os_, DT[dt], f"group {i}", g, x=inp["x"], R=inp["R"], rows=rows)
+        extra = output_widening(gc, oc, gs, os_, inp["w_packed"][o:o + n], K, cols,
+                                inp["w_scale"][o:o + n])
+        assert_close(got, ref, DT[dt], f"group {i}", extra)
+        o += n
+
+
+def test_grouped_linear_with_codes_in_and_pitched_outputs():
+    """The GEMM-only path (int8 codes with row scales) into outputs that are views of wider
+    buffers: guard columns stay untouched."""
+    M, K, groups = 150, 384, [100, 28, 300]
+    g = torch.Generator().manual_seed(4)
+    q = torch.randint(-8, 8, (M, K), generator=g, dtype=torch.int8).cuda()
+    a = (torch.rand(M, generator=g) + 0.1).cuda()
+    N = sum(groups)
+    wp = torch.randint(-128, 128, (N, K // 2), generator=g, dtype=torch.int8).cuda()
+    wsc = (torch.rand(N, generator=g) + 0.5).cuda()
+    bufs = [torch.full((M, n + 5), 7.0, device="cuda") for n in groups]
+    outs = [b[:, 2:2 + n] for b, n in zip(bufs, groups)]
+    ck.ck_w4a4_grouped_linear(q, None, 0, wp, wsc, None, groups, outs=outs, a_scale=a)
+    full = ck.ck_w4a4_linear(q, None, 0, wp, wsc, a_scale=a, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    o = 0
+    for b, out, n in zip(bufs, outs, groups):
+        assert torch.equal(out, full[:, o:o + n])
+        assert (b[:, :2] == 7.0).all() and (b[:, 2 + n:] == 7.0).all()
+        o += n
+
+
+# ------------------------------------------------------------------- W8A8 variant
+
+W8_RATE = 5e-3   # INT8 codes of 16-bit inputs: ~ the rate at which the dtype rounding of y flips
+
+
+@pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("g", [16, 64, 256])
+def test_int8_stage1_identity_rotation_bit_exact(dt, g):
+    """R = I makes y exact in every kernel: the INT8 codes and scales equal the oracle's."""
+    rng = np.random.default_rng(500 + g)
+    M, K = 200, 3840
+    x = rng.standard_normal((M, K)) * 3
+    x[:, rng.choice(K, K // 100, replace=False)] *= 20.0
+    x[7] = 0
+    xt = torch.from_numpy(x).to(DT[dt])
+    R = torch.eye(g, dtype=DT[dt])
+    codes, scales = ck.ck_rotate_quant_int8(xt.cuda(), R.cuda(), g)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.rotate_quant_int8(xt, R, g)
+    np.testing.assert_array_equal(scales.cpu().numpy(), os_)
+    np.testing.assert_array_equal(codes.cpu().numpy(), oc)
+
+
+@pytest.mark.parametrize("layout", ["row", "col"])
+def test_int8_stage1_f32_g16_bit_exact(layout):
+    g = torch.Generator().manual_seed(61)
+    x = torch.randn(256, 1024, generator=g) * 4
+    xv = _colmajor(x) if layout == "col" else x
+    R = W.haar_orthogonal(16, torch.Generator().manual_seed(62)).float().contiguous()
+    codes, scales = ck.ck_rotate_quant_int8(to_device(xv), R.cuda(), 16)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.rotate_quant_int8(xv, R, 16)
+    np.testing.assert_array_equal(scales.cpu().numpy(), os_)
+    np.testing.assert_array_equal(codes.cpu().numpy(), oc)
+
+
+@pytest.mark.parametrize("dt,g,M,K", [("bf16", 64, 8192, 3840), ("f16", 256, 8192, 10240),
+                                      ("bf16", 16, 300, 3840), ("f16", 64, 50, 16384)])
+def test_int8_stage1_general_rotation(dt, g, M, K):
+    case = W.RotateCase(f"int8_{dt}_{g}", M=M, K=K, g=g, dtype=dt, seed=g + K)
+    inp = W.make_rotate_inputs(case)
+    R = W.haar_orthogonal(g, torch.Generator().manual_seed(K)).to(DT[dt]).contiguous()
+    codes, scales = ck.ck_rotate_quant_int8(to_device(inp["x"]), R.cuda(), g)
+    torch.cuda.synchronize()
+    rows = sample_rows(M, 48)
+    oc, os_ = oracle.rotate_quant_int8(inp["x"], R, g, rows=rows)
+    idx = torch.from_numpy(rows).cuda()
+    compare_stage1(codes[idx].cpu().numpy(), scales[idx].cpu().numpy(), oc, os_, DT[dt], case.name,
+                   g, x=inp["x"], R=R, rows=rows, qmax=127, max_rate=W8_RATE)
+
+
+@pytest.mark.parametrize("M,N,K,out_dt", [(1, 1, 128, torch.float32), (200, 300, 448, torch.float32),
+                                          (4000, 2000, 384, torch.bfloat16),
+                                          (8192, 3840, 3840, torch.bfloat16),
+                                          (77, 513, 4096, torch.float16)])
+def test_w8a8_gemm_accumulators_bit_exact(M, N, K, out_dt):
+    g = torch.Generator().manual_seed(M + N + K + 8)
+    q = torch.randint(-128, 128, (M, K), generator=g, dtype=torch.int8)
+    w = torch.randint(-128, 128, (N, K), generator=g, dtype=torch.int8)
+    q[0] = -128
+    w[0] = -128                                  # acc[0, 0] = 16384 K, the bound
+    out = ck.ck_w8a8_linear(q.cuda(), None, 0, w.cuda(), torch.ones(N, device="cuda"),
+                            a_scale=torch.ones(M, device="cuda"), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    rows, cols = sample_rows(M, 64), sample_cols(N, 96)
+    acc = oracle.gemm_s32(q.numpy()[rows], w.numpy()[cols])
+    got = out.cpu().numpy()[rows][:, cols]
+    # exact in fp32 while |acc| < 2^24; beyond, the fp32 cast of the exact INT32 value
+    np.testing.assert_array_equal(got, acc.astype(np.float32))
+    assert got[0, 0] == 16384 * K
+    a = torch.rand(M, generator=g) * 0.01 + 0.001
+    ws = (torch.rand(N, generator=g) * 0.015 + 0.005).to(out_dt)
+    b = torch.randn(N, generator=g).to(out_dt)
+    out2 = ck.ck_w8a8_linear(q.cuda(), None, 0, w.cuda(), ws.cuda(), b.cuda(), a_scale=a.cuda(),
+                             out_dtype=out_dt)
+    torch.cuda.synchronize()
+    ref = oracle.epilogue(acc, a.numpy()[rows], ws[cols], b[cols], out_dt)
+    assert torch.equal(out2.cpu()[torch.from_numpy(rows)][:, torch.from_numpy(cols)], ref)
+
+
+@pytest.mark.parametrize("dt,M,N,K,g", [("bf16", 197, 301, 448, 64), ("f16", 300, 130, 768, 256),
+                                        ("f32", 129, 260, 464, 16), ("bf16", 8192, 3840, 3840, 64)])
+def test_w8a8_linear_against_the_oracle(dt, M, N, K, g):
+    """The whole W8A8 path: bit-exact against the oracle's GEMM + epilogue on the GPU's own INT8
+    codes, and within the parity rule against the whole oracle path (tie flips widened)."""
+    gen = torch.Generator().manual_seed(M + N)
+    case = W.LinearCase("w8", M=M, K=K, N=N, g=g, dtype=dt, rotation="haar", seed=M * 3 + g)
+    inp = W.make_linear_inputs(case)
+    w8 = torch.randint(-128, 128, (N, K), generator=gen, dtype=torch.int8)
+    x, R = to_device(inp["x"]), inp["R"].cuda()
+    ws = torch.empty(int(ck.lib().ck_w8a8_linear_workspace_bytes(M, N, K, K)), dtype=torch.uint8,
+                     device="cuda")
+    out = ck.ck_w8a8_linear(x, R, g, w8.cuda(), inp["w_scale"].cuda(), inp["bias"].cuda(),
+                            workspace=ws)
+    torch.cuda.synchronize()
+    rows, cols = sample_rows(M, 48), sample_cols(N, 64)
+    gcodes, gscales = workspace_stage1(ws, M, K)
+    gc = gcodes[torch.from_numpy(rows).cuda()].cpu().numpy()
+    gs = gscales[torch.from_numpy(rows).cuda()].cpu().numpy()
+    ref, oc, os_ = oracle.linear_w8a8(inp["x"], inp["R"], g, w8, inp["w_scale"], inp["bias"],
+                                      rows=rows, cols=cols)
+    compare_stage1(gc, gs, oc, os_, DT[dt], "w8a8", g, x=inp["x"], R=inp["R"], rows=rows,
+                   qmax=127, max_rate=W8_RATE)
+    got = out.cpu()[torch.from_numpy(rows)][:, torch.from_numpy(cols)]
+    acc = oracle.gemm_s32(gc, w8.numpy()[cols])
+    exact = oracle.epilogue(acc, gs, inp["w_scale"][cols], inp["bias"][cols], DT[dt])
+    itype = torch.int32 if dt == "f32" else torch.int16
+    assert torch.equal(got.view(itype), exact.view(itype))
+    extra = widening_for_weights(gc, oc, gs, os_, w8.numpy()[cols], inp["w_scale"][cols])
+    assert_close(got, ref, DT[dt], "w8a8", extra)
+
+
+# ------------------------------------------------------------------- packed quantizer
+
+def _unpack_codes(packed: np.ndarray) -> np.ndarray:
+    lo = (packed & 0xF).astype(np.int64)
+    hi = (packed >> 4).astype(np.int64)
+    out = np.empty((packed.shape[0], 2 * packed.shape[1]), dtype=np.int64)
+    out[:, 0::2] = np.where(lo >= 8, lo - 16, lo)
+    out[:, 1::2] = np.where(hi >= 8, hi - 16, hi)
+    return out
+
+
+@pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("stochastic", [False, True])
+def test_packed_quantizer_identity_rotation_bit_exact(dt, stochastic):
+    """R = I: y is exact on both sides, so nearest and stochastic codes (the same Philox draws,
+    the same fp32 operations) and the packed bytes equal the oracle's."""
+    rng = np.random.default_rng(70)
+    M, K, g = 96, 1024, 64
+    x = rng.standard_normal((M, K)) * 2
+    x[:, rng.choice(K, 10, replace=False)] *= 20
+    x[3] = 0
+    xt = torch.from_numpy(x).to(DT[dt])
+    R = torch.eye(g, dtype=DT[dt])
+    packed, scales = ck.ck_rotate_quant_packed(xt.cuda(), R.cuda(), g, stochastic=stochastic,
+                                               seed=0x1234ABCD5678, offset=99)
+    torch.cuda.synchronize()
+    y = oracle.rotate(xt, R, g)
+    op, os_ = oracle.quantize_packed(y, np.arange(M), K, stochastic=stochastic,
+                                     seed=0x1234ABCD5678, offset=99)
+    np.testing.assert_array_equal(scales.cpu().numpy(), os_)
+    np.testing.assert_array_equal(packed.cpu().numpy(), op)
+
+
+def test_packed_quantizer_nearest_matches_stage1_codes():
+    """Nearest rounding gives ck_rotate_quant's codes, packed (identity rotation: y exact)."""
+    x = torch.randn(50, 512, generator=torch.Generator().manual_seed(71)).to(torch.bfloat16).cuda()
+    R = torch.eye(16, dtype=torch.bfloat16).cuda()
+    packed, s1 = ck.ck_rotate_quant_packed(x, R, 16)
+    codes, s2 = ck.ck_rotate_quant(x, R, 16)
+    torch.cuda.synchronize()
+    assert torch.equal(s1, s2)
+    np.testing.assert_array_equal(_unpack_codes(packed.cpu().numpy()), codes.cpu().numpy())
+
+
+@pytest.mark.parametrize("dt,g", [("bf16", 64), ("f16", 256), ("f32", 16)])
+def test_packed_quantizer_stochastic_general_rotation(dt, g):
+    """A general R: y may differ from the oracle's by its accumulation's rounding, so a code may
+    differ only where t + u lies within that difference of an integer (the stochastic analog
+    of a tie), by one step; scales follow the stage-1 rule."""
+    M, K = 64, 2048
+    x = torch.randn(M, K, generator=torch.Generator().manual_seed(72)).to(DT[dt])
+    R = W.haar_orthogonal(g, torch.Generator().manual_seed(73)).to(DT[dt]).contiguous()
+    seed, off = 2024, 5
+    packed, scales = ck.ck_rotate_quant_packed(x.cuda(), R.cuda(), g, stochastic=True, seed=seed,
+                                               offset=off)
+    torch.cuda.synchronize()
+    y = oracle.rotate(x, R, g)
+    op, os_ = oracle.quantize_packed(y, np.arange(M), K, stochastic=True, seed=seed, offset=off)
+    gs = scales.cpu().numpy()
+    rel = np.abs(gs.astype(np.float64) - os_) / os_
+    from parity_util import scale_rtol, tie_distance_bound
+    assert (rel <= scale_rtol(DT[dt], g)).all()
+    gq, oq = _unpack_codes(packed.cpu().numpy()), _unpack_codes(op)
+    diff = gq - oq
+    assert np.abs(diff).max() <= 1 and (diff != 0).mean() <= 1e-3
+    for r, k in zip(*np.nonzero(diff)):
+        e = r * K + k
+        word = oracle.philox4x32_10([e & 0xFFFFFFFF, e >> 32, off, 0], [seed, 0])[0]
+        u = float(np.float32(word >> 8) * np.float32(2.0 ** -24))
+        t = y[r, k] / float(os_[r])
+        xr = oracle.decode(x[r].contiguous())
+        j, c = divmod(int(k), g)
+        terms = np.abs(xr[j * g:(j + 1) * g]) @ np.abs(oracle.decode(R.contiguous())[:, c])
+        bound = tie_distance_bound(np.array([y[r, k]]), np.array([float(os_[r])]), np.array([terms]),
+                                   DT[dt], g, dynamic=True)[0] + 2.0 ** -23 * (abs(t) + 1)
+        dist = abs((t + u) - round(t + u))
+        assert dist <= bound, (r, k, t, u, dist, bound)
+
+
+def test_packed_quantizer_seed_and_offset_change_the_draws():
+    x = torch.randn(32, 1024, generator=torch.Generator().manual_seed(74)).cuda()
+    R = torch.eye(16).cuda()
+    a, _ = ck.ck_rotate_quant_packed(x, R, 16, stochastic=True, seed=1)
+    b, _ = ck.ck_rotate_quant_packed(x, R, 16, stochastic=True, seed=1)
+    c, _ = ck.ck_rotate_quant_packed(x, R, 16, stochastic=True, seed=2)
+    d, _ = ck.ck_rotate_quant_packed(x, R, 16, stochastic=True, seed=1, offset=1)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and not torch.equal(a, c) and not torch.equal(a, d)
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+@pytest.mark.parametrize("M,K", [(300, 64), (1000, 448), (8192, 3840), (77, 8192)])
+def test_rotate_quant_g16_on_tensor_cores(dt, M, K):
+    """g = 16 rows of whole 64-channel groups run as a g = 64 rotation by diag(R, R, R, R) on
+    the tensor-core kernel.  A non-symmetric R, so a transposed or misplaced block shows; every
+    output of the sampled rows is compared."""
+    case = W.RotateCase(f"g16tc_{dt}_{K}", M=M, K=K, g=16, dtype=dt, seed=K + M)
+    x = W.make_rotate_inputs(case)["x"]
+    R = W.haar_orthogonal(16, torch.Generator().manual_seed(K)).to(DT[dt]).contiguous()
+    codes, scales = ck.ck_rotate_quant(to_device(x), R.cuda(), 16)
+    torch.cuda.synchronize()
+    rows = sample_rows(M, 64)
+    oc, os_ = oracle.rotate_quant(x, R, 16, rows=rows)
+    idx = torch.from_numpy(rows).cuda()
+    compare_stage1(codes[idx].cpu().numpy(), scales[idx].cpu().numpy(), oc, os_, DT[dt], case.name,
+                   16, x=x, R=R, rows=rows)
