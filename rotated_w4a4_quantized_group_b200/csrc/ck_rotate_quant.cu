@@ -852,8 +852,10 @@ __device__ __forceinline__ void tc_quant_store(const uint32_t (&yp)[8], const Ro
     }
 }
 
-// RG = G: R is the g x g rotation.  RG = 16 < G = 64: the rotation of g = 16 done as one of
-// g = 64 by the block-diagonal diag(R, R, R, R) (its zero blocks add exact zeros to each sum).
+// RG = G: R is the g x g rotation.  RG = 16 < G = 64: rows of g = 16 groups viewed as 64-channel
+// group-rows; each of the four 16-channel groups is its own MMA (M = 128, N = 16, K = 16) of
+// the group's 16 channels against R^T, into its own 16 accumulator columns, so no group sees
+// another group's values (an Inf stays within its group, as in the per-group rotation).
 template <typename T, int G, bool DYN, int RG = G>
 __global__ void __launch_bounds__(kTcThreads, 1)
     rq_tc_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ R,
@@ -907,7 +909,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // registers and stores the 16-byte chunks of rows n0 .. n0 + 7 of R^T.  Consecutive
     // threads take consecutive k0, so a warp's stores cover distinct swizzled chunks.
     if constexpr (RG != G) {
-        // block-diagonal R: R^T[n][k] = R[k % RG][n % RG] inside the diagonal blocks, 0 outside
+        // R^T in the diagonal blocks (the only ones the MMAs read), zeros elsewhere
         for (int i = tid; i < G * G; i += kTcThreads) {
             const int n = i / G, k = i % G;
             const T v = (n / RG == k / RG) ? R[(k % RG) * RG + (n % RG)] : Elem<T>::from_f(0.f);
@@ -979,10 +981,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tc_fence_after();
                     const uint64_t adesc = adesc0 + (uint64_t)(s * (kTcStageBytes >> 4));
                     const uint64_t bdesc = bdesc0 + (uint64_t)(a * ((G * 128) >> 4));
+                    if constexpr (RG != G) {
+                        // group gi: A channels 16 gi .. (32 bytes in), B = R^T rows 16 gi ..
+                        // (16 rows of 128 bytes = 128 units in) at the same channels, N = 16
+                        constexpr uint32_t idesc16 = idesc_f16(128, RG, std::is_same<T, __nv_bfloat16>::value);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)   // K = 16 (32 bytes) per instruction
-                        tc_mma_f16(tmem_base + (uint32_t)(b * G), adesc + (uint64_t)(kk * 2),
-                                   bdesc + (uint64_t)(kk * 2), p.idesc, (a > 0 || kk > 0) ? 1u : 0u);
+                        for (int gi = 0; gi < G / RG; ++gi)
+                            tc_mma_f16(tmem_base + (uint32_t)(b * G + RG * gi), adesc + (uint64_t)(gi * 2),
+                                       bdesc + (uint64_t)(gi * ((RG * 128) >> 4) + gi * 2), idesc16, 0u);
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)   // K = 16 (32 bytes) per instruction
+                            tc_mma_f16(tmem_base + (uint32_t)(b * G), adesc + (uint64_t)(kk * 2),
+                                       bdesc + (uint64_t)(kk * 2), p.idesc, (a > 0 || kk > 0) ? 1u : 0u);
+                    }
                     tc_commit(&x_empty[s]);
                 }
                 if (ok) tc_commit(&d_full[b]);

@@ -80,6 +80,19 @@ __device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, dou
                  : "d"(a), "d"(b));
 }
 
+// Sixteen codes of a row: the dynamic-scale path (no clamp needed) or the general one.
+__device__ __forceinline__ void quant16_any(const float (&y)[16], const RowDivisor& dv, bool dyn,
+                                            uint32_t (&out)[4]) {
+    if (dyn) {
+        unsigned long long y2[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y2[i] = f2_pack(y[2 * i], y[2 * i + 1]);
+        quant16_dyn2(y2, dv, out);
+    } else {
+        quant16(y, dv, out);
+    }
+}
+
 __device__ __forceinline__ float f32_row_scale(float amax, const float* scale_in, int qmax) {
     const float s = scale_in ? *scale_in : __fdiv_rn(amax, (float)qmax);
     return (s < FLT_MIN) ? FLT_MIN : s;   // lower clamp; NaN stays NaN
@@ -97,6 +110,7 @@ __global__ void __launch_bounds__(rqf32::kThreads, 2)
     __shared__ __align__(8) uint64_t full[kMaxBoxes];
     __shared__ unsigned int amax_sh[2][kMaxRB];   // this CTA's partial row maxima (|y| bits)
     __shared__ float row_s[kMaxRB], row_r[kMaxRB];
+    __shared__ unsigned int peer_sh[kMaxCluster][kMaxRB];   // every CTA's partial maxima
     __shared__ int abort_flag;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -216,89 +230,85 @@ __global__ void __launch_bounds__(rqf32::kThreads, 2)
             if (fc == 0) atomicMax(&amax_sh[par][m], __float_as_uint(mx));
         } else {
             // task = (row m, groups 16 o .. 16 o + 15 of the slice) as two fragment sets of 8
-            // group-rows.  Group j of box b = j / GBb is 64-byte row (m GBb + j - b GBb) of the box
+            // group-rows.  Warps own rows: wpr warps share a row (taking every wpr-th 16 groups),
+            // a warp takes every (8 / wpr)-th row.  Group j of box b = j / GBb is 64-byte row
+            // (m GBb + j - b GBb) of the box
             const int o16 = (ngroups + 15) / 16;
-            float mx = 0.f;
-            int cur = -1;
-            for (int t = warp; ok && t < p.RB * o16; t += kWarps) {
-                const int mrow = t / o16, o = t - mrow * o16;
-                if (mrow != cur) {   // warp-uniform: flush the previous row's maximum
-                    if (cur >= 0) {
-#pragma unroll
-                        for (int dd = 16; dd > 0; dd >>= 1) mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, dd));
-                        if (lane == 0) atomicMax(&amax_sh[par][cur], __float_as_uint(mx));
+            const int wpr = p.RB >= kWarps ? 1 : kWarps / p.RB;
+            for (int mrow = warp / wpr; ok && mrow < p.RB; mrow += kWarps / wpr) {
+                float mx = 0.f;
+                for (int o = warp % wpr; ok && o < o16; o += wpr) {
+                    const int jlast = (16 * o + 15) < ngroups ? (16 * o + 15) : (ngroups - 1);
+                    if (!wait_box(jlast / p.GBb)) {
+                        ok = false;
+                        break;
                     }
-                    cur = mrow;
-                    mx = 0.f;
-                }
-                const int jlast = (16 * o + 15) < ngroups ? (16 * o + 15) : (ngroups - 1);
-                if (!wait_box(jlast / p.GBb)) {
-                    ok = false;
-                    break;
-                }
-                double a[2][4];
-                float* bxs[2];
-                uint32_t rows_[2];
-                bool jv[2];
+                    double a[2][4];
+                    float* bxs[2];
+                    uint32_t rows_[2];
+                    bool jv[2];
 #pragma unroll
-                for (int t2 = 0; t2 < 2; ++t2) {
-                    const int j = 16 * o + 8 * t2 + fr;
-                    jv[t2] = j < ngroups;
-                    const int b = jv[t2] ? j / p.GBb : 0;
-                    bxs[t2] = tile + (size_t)b * box_floats;
-                    rows_[t2] = jv[t2] ? (uint32_t)(mrow * p.GBb + (j - b * p.GBb)) : 0u;
-                    const uint32_t ph = (rows_[t2] >> 1) & 3u;
+                    for (int t2 = 0; t2 < 2; ++t2) {
+                        const int j = 16 * o + 8 * t2 + fr;
+                        jv[t2] = j < ngroups;
+                        const int b = jv[t2] ? j / p.GBb : 0;
+                        bxs[t2] = tile + (size_t)b * box_floats;
+                        rows_[t2] = jv[t2] ? (uint32_t)(mrow * p.GBb + (j - b * p.GBb)) : 0u;
+                        const uint32_t ph = (rows_[t2] >> 1) & 3u;
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            a[t2][ks] = jv[t2] ? (double)bxs[t2][rows_[t2] * 16u + (((uint32_t)ks ^ ph) << 2) + fc] : 0.0;
+                    }
+                    __syncwarp();
+                    double d[2][2][2];
+#pragma unroll
+                    for (int nh = 0; nh < 2; ++nh)
+#pragma unroll
+                        for (int t2 = 0; t2 < 2; ++t2) d[t2][nh][0] = d[t2][nh][1] = 0.0;
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        a[t2][ks] = jv[t2] ? (double)bxs[t2][rows_[t2] * 16u + (((uint32_t)ks ^ ph) << 2) + fc] : 0.0;
-                }
-                __syncwarp();
-                double d[2][2][2];
 #pragma unroll
-                for (int nh = 0; nh < 2; ++nh)
+                        for (int nh = 0; nh < 2; ++nh) {
+                            dmma_8x8x4(d[0][nh][0], d[0][nh][1], a[0][ks], rb[ks][nh]);
+                            dmma_8x8x4(d[1][nh][0], d[1][nh][1], a[1][ks], rb[ks][nh]);
+                        }
 #pragma unroll
-                    for (int t2 = 0; t2 < 2; ++t2) d[t2][nh][0] = d[t2][nh][1] = 0.0;
+                    for (int t2 = 0; t2 < 2; ++t2) {
+                        if (!jv[t2]) continue;
+                        const uint32_t ph = (rows_[t2] >> 1) & 3u;
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-                    for (int nh = 0; nh < 2; ++nh) {
-                        dmma_8x8x4(d[0][nh][0], d[0][nh][1], a[0][ks], rb[ks][nh]);
-                        dmma_8x8x4(d[1][nh][0], d[1][nh][1], a[1][ks], rb[ks][nh]);
-                    }
-#pragma unroll
-                for (int t2 = 0; t2 < 2; ++t2) {
-                    if (!jv[t2]) continue;
-                    const uint32_t ph = (rows_[t2] >> 1) & 3u;
-#pragma unroll
-                    for (int nh = 0; nh < 2; ++nh) {
-                        const float y0 = __double2float_rn(d[t2][nh][0]);
-                        const float y1 = __double2float_rn(d[t2][nh][1]);
-                        mx = fmax_nan(mx, fmax_nan(fabsf(y0), fabsf(y1)));
-                        // words 8 nh + 2 fc, + 1: chunk 2 nh + fc / 2
-                        const uint32_t off = rows_[t2] * 16u +
-                                             ((((uint32_t)(2 * nh) + (fc >> 1)) ^ ph) << 2) +
-                                             2u * (fc & 1);
-                        *reinterpret_cast<float2*>(bxs[t2] + off) = make_float2(y0, y1);
+                        for (int nh = 0; nh < 2; ++nh) {
+                            const float y0 = __double2float_rn(d[t2][nh][0]);
+                            const float y1 = __double2float_rn(d[t2][nh][1]);
+                            mx = fmax_nan(mx, fmax_nan(fabsf(y0), fabsf(y1)));
+                            // words 8 nh + 2 fc, + 1: chunk 2 nh + fc / 2
+                            const uint32_t off = rows_[t2] * 16u +
+                                                 ((((uint32_t)(2 * nh) + (fc >> 1)) ^ ph) << 2) +
+                                                 2u * (fc & 1);
+                            *reinterpret_cast<float2*>(bxs[t2] + off) = make_float2(y0, y1);
+                        }
                     }
                 }
-            }
-            if (cur >= 0) {
 #pragma unroll
                 for (int dd = 16; dd > 0; dd >>= 1) mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, dd));
-                if (lane == 0) atomicMax(&amax_sh[par][cur], __float_as_uint(mx));
+                if (lane == 0) atomicMax(&amax_sh[par][mrow], __float_as_uint(mx));
             }
         }
         __syncthreads();
         // ---------------------------------------------------------------- row scales
         // every CTA of the cluster takes this barrier once per block, whatever happened above
         if (ncta > 1) cluster_sync_all();
+        // peer maxima: thread (row m, CTA q) reads one word, then each row's thread takes the
+        // maximum of the CTA's slots (one distributed read per thread, all in parallel)
+        for (int i = tid; i < p.RB * (int)ncta; i += kThreads) {
+            const int m = i % p.RB;
+            const uint32_t q = (uint32_t)(i / p.RB);
+            peer_sh[q][m] = q == rank ? amax_sh[par][m] : dsmem_load_u32(&amax_sh[par][m], q);
+        }
+        __syncthreads();
         if (tid < p.RB) {
-            unsigned int bits = amax_sh[par][tid];
-            for (uint32_t q = 0; q < ncta; ++q)
-                if (q != rank) {
-                    const unsigned int v = dsmem_load_u32(&amax_sh[par][tid], q);
-                    bits = v > bits ? v : bits;   // |y| bits order like the values; NaN is largest
-                }
+            unsigned int bits = 0u;
+            for (uint32_t q = 0; q < ncta; ++q) bits = peer_sh[q][tid] > bits ? peer_sh[q][tid] : bits;
             const float s = f32_row_scale(__uint_as_float(bits), scale_in, p.qmax);
             const RowDivisor dv(s, p.qmax);
             row_s[tid] = s;
@@ -320,7 +330,7 @@ __global__ void __launch_bounds__(rqf32::kThreads, 2)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) y[i] = tile[sw64(16u * j + i, (uint32_t)m)];
                     uint32_t out[4];
-                    quant16(y, dv, out);
+                    quant16_any(y, dv, scale_in == nullptr, out);
                     int8_t* dst = codes + (m0 + m) * p.ldq + k0 + 16 * j;
                     if (p.vec_codes) {
                         *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
@@ -349,7 +359,7 @@ __global__ void __launch_bounds__(rqf32::kThreads, 2)
                         y[4 * q + 3] = v.w;
                     }
                     uint32_t out[4];
-                    quant16(y, dv, out);
+                    quant16_any(y, dv, scale_in == nullptr, out);
                     int8_t* dst = codes + (m0 + m) * p.ldq + k0 + 16 * j;
                     if (p.vec_codes) {
                         *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);

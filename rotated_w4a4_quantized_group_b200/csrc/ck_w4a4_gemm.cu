@@ -13,7 +13,8 @@
 // operand and live in tensor memory; the activation codes are its B operand, staged in
 // shared memory by TMA.  A tile is 128 output channels x BNA activation rows (BNA <= 192)
 // and is accumulated transposed, D[n, m] (TMEM lane = channel n, column = row m):
-//   warp 0      TMA producer of the codes: BNA rows x 128 bytes per stage, 128-byte swizzle
+//   warps 0, 3  TMA producers of the codes, BNA rows x 128 bytes per k-block, 128-byte swizzle:
+//               warp 0 the even k-blocks of each super-stage, warp 3 the odd ones
 //   warp 2      TMA producer of the packed weights: 128 rows x 64 bytes, 64-byte swizzle
 //   warps 8-23  unpack, in two sets of eight that take alternate super-stages: each thread
 //               owns one weight row (a TMEM lane) and one half of each k-block's K; it expands
@@ -62,7 +63,7 @@ constexpr int ND = 16;                   // super-stage completion barriers (> X
 constexpr uint32_t W_BYTES = BW * BK / 2;    // 8 KB
 constexpr uint32_t A_STAGE_COLS = BK / 4;    // 32 TMEM columns of 4 bytes per stage
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int WARP_TMA_X = 0, WARP_MMA = 1, WARP_TMA_W = 2;
+constexpr int WARP_TMA_X = 0, WARP_MMA = 1, WARP_TMA_W = 2, WARP_TMA_X2 = 3;
 // epilogue: warps 4..7 and 24..27, two per TMEM lane quarter, taking alternate 16-row chunks
 constexpr int EPI_WARP0 = 4, EPI_WARP1 = 24, EPI_WARPS = 8;
 constexpr int UNP_WARP0 = 8, UNP_SET_WARPS = 8, UNP_SETS = 2;   // warps 8..23
@@ -70,6 +71,9 @@ constexpr int UNP_WARPS = UNP_SET_WARPS * UNP_SETS;
 constexpr int THREADS = (EPI_WARP1 + 4) * 32;
 constexpr int64_t SCALED16_MAX_K = (1LL << 21) - 1;   // 16 * 64 * K < 2^31
 constexpr size_t SMEM_BUDGET = 220 * 1024;
+// per epilogue warp: one 16-row x 32-channel chunk of outputs (fp32 at most) staged for
+// 16-byte stores
+constexpr uint32_t EPI_STAGE_BYTES = 16 * 32 * 4;
 static_assert(UNP_WARP0 % 4 == 0 && EPI_WARP0 % 4 == 0 && EPI_WARP1 % 4 == 0,
               "TMEM lane quarters follow warp % 4");
 static_assert(UNP_WARP0 + UNP_WARPS == EPI_WARP1, "warp roles tile the CTA");
@@ -117,6 +121,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
     unsigned char* x_ring = smem;
     unsigned char* w_ring = x_ring + (size_t)XS * xss_bytes;   // W8: XS slots of G k-blocks
     constexpr uint32_t W8_BYTES = BW * BK;                      // one INT8 weight k-block, 16 KB
+    unsigned char* epi_stage = w_ring + (W8 ? (size_t)XS * G * W8_BYTES : (size_t)2 * G * W_BYTES);
 
     __shared__ __align__(8) uint64_t x_full[XS_MAX], w_full[UNP_SETS], w_empty[UNP_SETS];
     __shared__ __align__(8) uint64_t a_full[NB_MAX], done[ND];
@@ -138,7 +143,8 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
     };
 
     if (tid == 0) {
-        for (int s = 0; s < XS_MAX; ++s) mbar_init(&x_full[s], W8 ? 2 : 1);
+        // the two codes producers, and the INT8 weights producer (W8)
+        for (int s = 0; s < XS_MAX; ++s) mbar_init(&x_full[s], W8 ? 3 : 2);
         for (int s = 0; s < UNP_SETS; ++s) {
             mbar_init(&w_full[s], 1);
             mbar_init(&w_empty[s], UNP_SET_WARPS);
@@ -170,9 +176,12 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         return mbar_wait(&done[s & (ND - 1)], (s >> 4) & 1u, &abort_flag, p.dev_status);
     };
 
-    if (warp == WARP_TMA_X) {
-        // ---------------------------------------------------------------- codes producer
+    if (warp == WARP_TMA_X || warp == WARP_TMA_X2) {
+        // ---------------------------------------------------------------- codes producers
+        // warp WARP_TMA_X brings the even k-blocks of each super-stage, warp WARP_TMA_X2 the
+        // odd ones: one box per issuing thread and k-block, so two boxes load at once
         if (lane == 0) {
+            const uint32_t par = warp == WARP_TMA_X2 ? 1u : 0u;
             uint32_t issued = 0, slot = 0;
             bool ok = true;
             for (uint32_t ss = 0; ok && ss < my_ss; ++ss) {
@@ -185,15 +194,14 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                 const int32_t kb0 = (int32_t)((ss % nss) * G);
                 const uint32_t n_k = ss_nk(ss);
                 unsigned char* dst = x_ring + (size_t)slot * xss_bytes;
-                if (p.box3d) {
-                    // one box of G k-blocks (those past K arrive as zeros and are not used)
-                    mbar_arrive_expect_tx(&x_full[slot], G * x_bytes);
-                    tma_load_3d(dst, &xmap, &x_full[slot], 0, m0, kb0);
-                } else {
-                    mbar_arrive_expect_tx(&x_full[slot], n_k * x_bytes);
-                    for (uint32_t j = 0; j < n_k; ++j)
+                const uint32_t mine = n_k > par ? (n_k - par + 1) / 2 : 0;   // k-blocks par, par + 2, ..
+                if (mine) {
+                    mbar_arrive_expect_tx(&x_full[slot], mine * x_bytes);
+                    for (uint32_t j = par; j < n_k; j += 2)
                         tma_load_2d(dst + (size_t)j * x_bytes, &xmap, &x_full[slot],
                                     (kb0 + (int32_t)j) * BK, m0);
+                } else {
+                    mbar_arrive(&x_full[slot]);
                 }
                 ++issued;
                 if (++slot == XS) slot = 0;
@@ -421,6 +429,17 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
             while (n_ok && sg + 1 < p.segs.n && n >= p.segs.start[sg + 1]) ++sg;
             OutT* ocol = static_cast<OutT*>(p.segs.ptr[sg]) + (n_ok ? n - p.segs.start[sg] : 0);
             const int64_t ldo = p.segs.ldo[sg];
+            // 16-byte stores from a staged chunk when the warp's 32 channels are all present, in
+            // one segment, and every 16-byte piece of every row is aligned
+            constexpr int PER16 = 16 / (int)sizeof(OutT);          // outputs per 16 bytes
+            const int sg0 = __shfl_sync(0xffffffffu, sg, 0);
+            // lane 0's column address: the warp's first channel
+            const unsigned long long obits =
+                __shfl_sync(0xffffffffu, (unsigned long long)reinterpret_cast<uintptr_t>(ocol), 0);
+            const bool vec = __all_sync(0xffffffffu, n_ok && sg == sg0) && (obits % 16 == 0) &&
+                             (ldo % PER16 == 0);
+            OutT* stage = reinterpret_cast<OutT*>(epi_stage + (size_t)(q + 4 * eh) * EPI_STAGE_BYTES);
+            OutT* obase = reinterpret_cast<OutT*>(static_cast<uintptr_t>(obits));
 #pragma unroll
             for (int k = 0; k < BNA_MAX / 32; ++k) {
                 const int c0 = 32 * k + 16 * eh;       // first row of this warp's chunk
@@ -431,14 +450,28 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const float a_s = __shfl_sync(0xffffffffu, as_r[k], 16 * eh + j);
-                        if (c0 + j < rows) {
-                            const int accv = X16 ? ((int)r[j] >> 4) : (int)r[j];   // exact: 16 | acc
-                            float o = __int2float_rn(accv);
-                            o = __fmul_rn(o, a_s);
-                            o = __fmul_rn(o, ws);
-                            if (p.bias) o = __fadd_rn(o, bs);
-                            if (n_ok) OutStore<OutT>::one(ocol + (m0 + c0 + j) * ldo, o);
+                        const int accv = X16 ? ((int)r[j] >> 4) : (int)r[j];   // exact: 16 | acc
+                        float o = __int2float_rn(accv);
+                        o = __fmul_rn(o, a_s);
+                        o = __fmul_rn(o, ws);
+                        if (p.bias) o = __fadd_rn(o, bs);
+                        if (vec) {
+                            OutStore<OutT>::one(stage + j * 32 + lane, o);   // row j, channel lane
+                        } else if (c0 + j < rows && n_ok) {
+                            OutStore<OutT>::one(ocol + (m0 + c0 + j) * ldo, o);
                         }
+                    }
+                    if (vec) {
+                        __syncwarp();
+                        // 16 rows x 32 channels: 32 / PER16 pieces of 16 bytes a row
+                        constexpr int PIECES = 32 / PER16;
+                        for (int i = lane; i < 16 * PIECES; i += 32) {
+                            const int row = i / PIECES, pc = i % PIECES;
+                            if (c0 + row < rows)
+                                *reinterpret_cast<uint4*>(obase + (m0 + c0 + row) * ldo + pc * PER16) =
+                                    *reinterpret_cast<const uint4*>(stage + row * 32 + pc * PER16);
+                        }
+                        __syncwarp();
                     }
                 }
             }
@@ -522,29 +555,28 @@ static ck_status launch_persistent(const int8_t* codes, int64_t ldq, const float
     // with whole 128-byte k-blocks, one 3-D box fetches the G k-blocks of a super-stage:
     // (byte of the k-block, row, k-block); otherwise one 2-D box per k-block, zero past K
     const uint32_t G_box = 2;
-    if (box3d) {
-        const uint64_t dims[3] = {(uint64_t)BK, (uint64_t)M, (uint64_t)num_kb};
-        const uint64_t strides[2] = {(uint64_t)ldq, (uint64_t)BK};
-        const uint32_t box[3] = {BK, (uint32_t)p.BNA, G_box};
-        ck_status st = encode_tma(&xmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, codes, dims, strides,
-                                  box, CU_TENSOR_MAP_SWIZZLE_128B);
-        if (st != CK_OK) return st;
-        const uint64_t wdims[3] = {(uint64_t)wkb, (uint64_t)N, (uint64_t)num_kb};
-        const uint64_t wstrides[2] = {(uint64_t)w_ld, (uint64_t)wkb};
-        const uint32_t wbox[3] = {wkb, BW, G_box};
-        st = encode_tma(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w, wdims, wstrides, wbox, wsw);
-        if (st != CK_OK) return st;
-    } else {
+    {
+        // codes: one 2-D box (128 bytes x BNA rows) per k-block, zero past K and M
         const uint64_t dims[2] = {(uint64_t)K, (uint64_t)M};
         const uint64_t strides[1] = {(uint64_t)ldq};
         const uint32_t box[2] = {BK, (uint32_t)p.BNA};
         ck_status st = encode_tma(&xmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, dims, strides,
                                   box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (st != CK_OK) return st;
+    }
+    if (box3d) {
+        const uint64_t wdims[3] = {(uint64_t)wkb, (uint64_t)N, (uint64_t)num_kb};
+        const uint64_t wstrides[2] = {(uint64_t)w_ld, (uint64_t)wkb};
+        const uint32_t wbox[3] = {wkb, BW, G_box};
+        const ck_status st = encode_tma(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w, wdims, wstrides,
+                                        wbox, wsw);
+        if (st != CK_OK) return st;
+    } else {
         const uint64_t wdims[2] = {(uint64_t)(w8 ? K : K / 2), (uint64_t)N};
         const uint64_t wstrides[1] = {(uint64_t)w_ld};
         const uint32_t wbox[2] = {wkb, BW};
-        st = encode_tma(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w, wdims, wstrides, wbox, wsw);
+        const ck_status st = encode_tma(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w, wdims,
+                                        wstrides, wbox, wsw);
         if (st != CK_OK) return st;
     }
     p.M = M;
@@ -567,17 +599,17 @@ static ck_status launch_persistent(const int8_t* codes, int64_t ldq, const float
     if (w8) {
         // one INT8 weight super-stage per codes slot
         const size_t wss = (size_t)p.G * BW * BK;
-        p.xs = (int)(SMEM_BUDGET / (xss_bytes + wss));
+        p.xs = (int)((SMEM_BUDGET - EPI_WARPS * EPI_STAGE_BYTES) / (xss_bytes + wss));
         if (p.xs > XS_MAX) p.xs = XS_MAX;
         w_ring_bytes = (size_t)p.xs * wss;
     } else {
         w_ring_bytes = (size_t)2 * p.G * W_BYTES;
-        p.xs = (int)((SMEM_BUDGET - w_ring_bytes) / xss_bytes);
+        p.xs = (int)((SMEM_BUDGET - w_ring_bytes - EPI_WARPS * EPI_STAGE_BYTES) / xss_bytes);
         if (p.xs > XS_MAX) p.xs = XS_MAX;
     }
     if (p.G < 1 || p.xs < 2) return CK_ERR_UNSUPPORTED;
     p.nss = (p.num_kb + p.G - 1) / p.G;
-    const size_t smem = (size_t)p.xs * xss_bytes + w_ring_bytes + 1024;
+    const size_t smem = (size_t)p.xs * xss_bytes + w_ring_bytes + EPI_WARPS * EPI_STAGE_BYTES + 1024;
     p.idesc = idesc_i8(BW, p.BNA);   // signed 8-bit A and B, s32 accumulator, 128 x BNA
     p.a_scale = a_scale;
     p.w_scale = w_scale;

@@ -11,9 +11,10 @@
 // With few rows the work is a weight read: 128-channel tiles give only N / 128 CTAs (30 for
 // N = 3840).  Here each tile's K is split over a cluster of S CTAs (S * N / 128 ~ one CTA per
 // SM), and each CTA:
-//   warp 0      issues TMA copies of its whole K range at once: packed weights (128 rows x
-//               64 bytes per k-block, 64-byte swizzle) and codes (BNA rows x 128 bytes,
-//               128-byte swizzle), two k-blocks per box, one mbarrier per box pair;
+//   warps 0, 2  issue TMA copies of the CTA's whole K range at once, one box per lane: packed
+//               weights (warp 0; 128 rows x 64 bytes per k-block, 64-byte swizzle) and codes
+//               (warp 2; BNA rows x 128 bytes, 128-byte swizzle), two k-blocks per box, one
+//               mbarrier per box pair;
 //   warps 4-7   expand the weight nibbles (one weight row per thread) into tensor memory in
 //               chunks of up to six k-blocks, the MMA's A operand, then read the accumulator;
 //   warp 1      allocates tensor memory and issues tcgen05.mma kind::i8 (128 x BNA x 32, A from
@@ -38,7 +39,7 @@ namespace splitk {
 constexpr int BW = 128;                      // weight rows (channels) per tile: MMA M
 constexpr int BK = 128;                      // K elements per k-block
 constexpr int THREADS = 256;
-constexpr int WARP_TMA = 0, WARP_MMA = 1, UNP_WARP0 = 4;
+constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_TMA2 = 2, UNP_WARP0 = 4;
 constexpr int KB_MAX = 32;                   // k-blocks of one CTA held in shared memory
 constexpr int CHUNK_KB = 6;                  // k-blocks expanded into tensor memory at a time
 constexpr uint32_t TMEM_COLS = 256;
@@ -110,23 +111,34 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_sh;
 
-    if (warp == WARP_TMA) {
+    if (warp == WARP_TMA || warp == WARP_TMA2) {
         // ---------------------------------------------------------------- TMA: the whole range
-        if (lane == 0) {
-            for (int i = 0; i < npairs; ++i) {
-                const int kb = kb_lo + 2 * i;
+        // lane i of warp WARP_TMA brings pair i's weights, lane i of warp WARP_TMA2 its codes:
+        // one box per issuing thread, so the copies do not queue behind one another.  The pair's
+        // byte count is registered on its barrier before either warp issues (named barrier).
+        if (warp == WARP_TMA) {
+            for (int i = lane; i < npairs; i += 32) {
                 const uint32_t nk = p.box3d ? 2u : (uint32_t)((n_kb - 2 * i) < 2 ? (n_kb - 2 * i) : 2);
                 mbar_arrive_expect_tx(&ld_full[i], nk * (W_BYTES + p.x_bytes));
-                if (p.box3d) {
+            }
+        }
+        asm volatile("bar.sync 1, 64;" ::: "memory");
+        for (int i = lane; i < npairs; i += 32) {
+            const int kb = kb_lo + 2 * i;
+            const uint32_t nk = p.box3d ? 2u : (uint32_t)((n_kb - 2 * i) < 2 ? (n_kb - 2 * i) : 2);
+            if (p.box3d) {
+                if (warp == WARP_TMA)
                     tma_load_3d(wbuf + (size_t)(2 * i) * W_BYTES, &wmap, &ld_full[i], 0, n0, kb);
+                else
                     tma_load_3d(xbuf + (size_t)(2 * i) * p.x_bytes, &xmap, &ld_full[i], 0, 0, kb);
-                } else {
-                    for (uint32_t j = 0; j < nk; ++j) {
+            } else {
+                for (uint32_t j = 0; j < nk; ++j) {
+                    if (warp == WARP_TMA)
                         tma_load_2d(wbuf + (size_t)(2 * i + j) * W_BYTES, &wmap, &ld_full[i],
                                     (kb + (int)j) * (BK / 2), n0);
+                    else
                         tma_load_2d(xbuf + (size_t)(2 * i + j) * p.x_bytes, &xmap, &ld_full[i],
                                     (kb + (int)j) * BK, 0);
-                    }
                 }
             }
         }
