@@ -119,6 +119,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// ------------------------------------------------------------------ warps
+
+// True in exactly one lane of the (fully converged) warp, false in the others.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t chosen;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(chosen));
+    return chosen != 0;
+}
+
 // ------------------------------------------------------------------ thread-block clusters
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -277,37 +277,39 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         }
     } else if (warp == WARP_MMA) {
         // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            // descriptor of code k-block 0 of slot 0; k-block j of slot s starts
-            // (s G + j) x_bytes later (start-address field counts 16-byte units)
-            const uint64_t bdesc0 = smem_desc_k_sw128(smem_u32(x_ring));
-            const uint32_t kstep = x_bytes >> 4;
-            const uint64_t adesc0 = smem_desc_k_sw128(smem_u32(w_ring));   // W8 weights
-            uint32_t slot = 0, xphase = 0, lt = 0;
-            RingPos rb;   // TMEM weight buffer of the super-stage
-            bool ok = true;
-            uint32_t d_tmem = tmem_base;
-            for (uint32_t ss = 0; ok && ss < my_ss; ++ss, rb.step(NB)) {
-                if (!mbar_wait(&x_full[slot], xphase, &abort_flag, p.dev_status) ||
-                    (!W8 && !mbar_wait(&a_full[rb.idx], rb.phase, &abort_flag, p.dev_status))) {
-                    ok = false;
+        // The whole warp walks the ring and takes every wait (a vote makes each decision
+        // uniform), so every value an MMA takes is computed uniformly across the warp; one lane,
+        // elected once, issues all MMAs and commits (a commit tracks its own thread's MMAs).
+        const bool leader = elect_one();
+        // descriptor of code k-block 0 of slot 0; k-block j of slot s starts
+        // (s G + j) x_bytes later (start-address field counts 16-byte units)
+        const uint64_t bdesc0 = smem_desc_k_sw128(smem_u32(x_ring));
+        const uint32_t kstep = x_bytes >> 4;
+        const uint64_t adesc0 = smem_desc_k_sw128(smem_u32(w_ring));   // W8 weights
+        uint32_t slot = 0, xphase = 0, lt = 0;
+        RingPos rb;   // TMEM weight buffer of the super-stage
+        uint32_t d_tmem = tmem_base;
+        for (uint32_t ss = 0; ss < my_ss; ++ss, rb.step(NB)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&x_full[slot], xphase, &abort_flag, p.dev_status)))
+                break;
+            if (!W8 && !__all_sync(0xffffffffu, mbar_wait(&a_full[rb.idx], rb.phase, &abort_flag,
+                                                          p.dev_status)))
+                break;
+            tc_fence_after();
+            const uint32_t kb0 = (ss % nss) * G;
+            const uint32_t n_k = ss_nk(ss);
+            const uint32_t a_ss = tmem_base + a_col0 + rb.idx * G * A_STAGE_COLS;
+            if (kb0 == 0) {
+                // a new tile: its accumulator must have been drained by the epilogue
+                const uint32_t acc = lt & 1u;
+                if (lt >= 2 && !__all_sync(0xffffffffu, mbar_wait(&acc_empty[acc], ((lt >> 1) - 1) & 1u,
+                                                                  &abort_flag, p.dev_status)))
                     break;
-                }
                 tc_fence_after();
-                const uint32_t kb0 = (ss % nss) * G;
-                const uint32_t n_k = ss_nk(ss);
-                const uint32_t a_ss = tmem_base + a_col0 + rb.idx * G * A_STAGE_COLS;
-                if (kb0 == 0) {
-                    // a new tile: its accumulator must have been drained by the epilogue
-                    const uint32_t acc = lt & 1u;
-                    if (lt >= 2 && !mbar_wait(&acc_empty[acc], ((lt >> 1) - 1) & 1u, &abort_flag,
-                                              p.dev_status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    d_tmem = tmem_base + acc * (uint32_t)p.BNA;
-                }
+                d_tmem = tmem_base + acc * (uint32_t)p.BNA;
+            }
+            const bool last = kb0 + n_k == (uint32_t)p.num_kb;
+            if (leader) {
                 for (uint32_t j = 0; j < n_k; ++j) {
                     const uint64_t bdesc = bdesc0 + (uint64_t)((slot * G + j) * kstep);
                     const uint32_t a_tmem = a_ss + j * A_STAGE_COLS;
@@ -325,20 +327,22 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                                          bdesc + (uint64_t)(kk * 2), p.idesc, acc_flag);
                     }
                 }
-                if (kb0 + n_k == (uint32_t)p.num_kb) {
-                    tc_commit(&acc_full[lt & 1u]);
-                    ++lt;
-                }
+                if (last) tc_commit(&acc_full[lt & 1u]);
                 tc_commit(&done[ss & (ND - 1)]);
-                if (++slot == XS) {
-                    slot = 0;
-                    xphase ^= 1u;
-                }
             }
-            // every MMA issued above has completed once drain_bar flips
+            __syncwarp();
+            if (last) ++lt;
+            if (++slot == XS) {
+                slot = 0;
+                xphase ^= 1u;
+            }
+        }
+        // every MMA issued above has completed once drain_bar flips
+        if (leader) {
             tc_commit(&drain_bar);
             mbar_wait(&drain_bar, 0, nullptr, p.dev_status);
         }
+        __syncwarp();
     } else if (!W8 && warp >= UNP_WARP0 && warp < UNP_WARP0 + UNP_WARPS) {
         // ---------------------------------------------------------------- unpack into TMEM
         const int u = warp - UNP_WARP0;
