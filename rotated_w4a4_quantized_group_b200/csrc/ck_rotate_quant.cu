@@ -950,37 +950,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
-        if (lane == 0) {
-            int issued = my_boxes < kStages ? my_boxes : kStages;
-            for (; issued < my_boxes; ++issued) {
-                const int s = issued % kStages, f = issued / kStages;
-                if (!mbar_wait(&x_empty[s], (uint32_t)(f - 1) & 1u, &abort_flag, dev_status)) break;
-                issue(issued);
-            }
-            if (abort_flag)
-                for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
-                    mbar_wait(&x_full[j % kStages], (uint32_t)(j / kStages) & 1u, nullptr, nullptr);
+        // The warp walks the ring together (a vote makes each wait's outcome uniform) and one
+        // elected lane issues, so the copy operands are computed uniformly across the warp.
+        const bool leader = elect_one();
+        int issued = my_boxes < kStages ? my_boxes : kStages;
+        for (; issued < my_boxes; ++issued) {
+            const int s = issued % kStages, f = issued / kStages;
+            if (!__all_sync(0xffffffffu, mbar_wait(&x_empty[s], (uint32_t)(f - 1) & 1u, &abort_flag,
+                                                   dev_status)))
+                break;
+            if (leader) issue(issued);
+            __syncwarp();
         }
+        if (leader && abort_flag)
+            for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
+                mbar_wait(&x_full[j % kStages], (uint32_t)(j / kStages) & 1u, nullptr, nullptr);
+        __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            const uint64_t adesc0 = smem_desc_k_sw128(smem_u32(xring));
-            const uint64_t bdesc0 = smem_desc_k_sw128(smem_u32(rt));
-            bool ok = true;
-            for (int i = 0; i < my_tiles && ok; ++i) {
-                const int b = i % kAcc;
-                if (i >= kAcc &&
-                    !mbar_wait(&d_empty[b], (uint32_t)((i / kAcc) - 1) & 1u, &abort_flag, dev_status))
+        // the same warp-wide walk; the elected lane issues every MMA and commit (a commit
+        // tracks the MMAs of its own thread)
+        const bool leader = elect_one();
+        const uint64_t adesc0 = smem_desc_k_sw128(smem_u32(xring));
+        const uint64_t bdesc0 = smem_desc_k_sw128(smem_u32(rt));
+        bool ok = true;
+        for (int i = 0; i < my_tiles && ok; ++i) {
+            const int b = i % kAcc;
+            if (i >= kAcc &&
+                !__all_sync(0xffffffffu, mbar_wait(&d_empty[b], (uint32_t)((i / kAcc) - 1) & 1u,
+                                                   &abort_flag, dev_status)))
+                break;
+            for (int a = 0; a < kAtoms; ++a) {
+                const int n = i * kAtoms + a, s = n % kStages;
+                if (!__all_sync(0xffffffffu, mbar_wait(&x_full[s], (uint32_t)(n / kStages) & 1u,
+                                                       &abort_flag, dev_status))) {
+                    ok = false;
                     break;
-                for (int a = 0; a < kAtoms; ++a) {
-                    const int n = i * kAtoms + a, s = n % kStages;
-                    if (!mbar_wait(&x_full[s], (uint32_t)(n / kStages) & 1u, &abort_flag, dev_status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t adesc = adesc0 + (uint64_t)(s * (kTcStageBytes >> 4));
-                    const uint64_t bdesc = bdesc0 + (uint64_t)(a * ((G * 128) >> 4));
+                }
+                tc_fence_after();
+                const uint64_t adesc = adesc0 + (uint64_t)(s * (kTcStageBytes >> 4));
+                const uint64_t bdesc = bdesc0 + (uint64_t)(a * ((G * 128) >> 4));
+                if (leader) {
                     if constexpr (RG != G) {
                         // group gi: A channels 16 gi .. (32 bytes in), B = R^T rows 16 gi ..
                         // (16 rows of 128 bytes = 128 units in) at the same channels, N = 16
@@ -997,11 +1007,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                     tc_commit(&x_empty[s]);
                 }
-                if (ok) tc_commit(&d_full[b]);
+                __syncwarp();
             }
+            if (ok && leader) tc_commit(&d_full[b]);
+            __syncwarp();
+        }
+        if (leader) {
             tc_commit(&drain_bar);
             mbar_wait(&drain_bar, 0, nullptr, dev_status);
         }
+        __syncwarp();
     } else {
         // ---------------------------------------------------------------- epilogue warps
         const int q = warp & 3;                          // TMEM lanes 32q .. 32q + 31

@@ -144,22 +144,25 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
         }
     } else if (warp == WARP_MMA) {
         // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            const uint64_t bdesc0 = smem_desc_k_sw128(smem_u32(xbuf));
-            const uint32_t kstep = p.x_bytes >> 4;
-            bool ok = true;
-            for (int c = 0; ok && c < nchunks; ++c) {
-                if (!mbar_wait(&a_full, (uint32_t)c & 1u, &abort_flag, p.dev_status)) {
-                    ok = false;
-                    break;
-                }
-                const int kb0 = c * CHUNK_KB;
-                const int nc = (n_kb - kb0) < CHUNK_KB ? (n_kb - kb0) : CHUNK_KB;
-                // the codes of the chunk landed (the expansion waited for the same barriers)
-                for (int i = kb0 / 2; i <= (kb0 + nc - 1) / 2; ++i)
-                    if (!mbar_wait(&ld_full[i], 0, &abort_flag, p.dev_status)) ok = false;
-                if (!ok) break;
-                tc_fence_after();
+        // the warp walks the chunks together (votes make each wait's outcome uniform, so the
+        // MMA operands are computed uniformly); one elected lane issues every MMA and commit
+        const bool leader = elect_one();
+        const uint64_t bdesc0 = smem_desc_k_sw128(smem_u32(xbuf));
+        const uint32_t kstep = p.x_bytes >> 4;
+        bool ok = true;
+        for (int c = 0; ok && c < nchunks; ++c) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&a_full, (uint32_t)c & 1u, &abort_flag, p.dev_status))) {
+                ok = false;
+                break;
+            }
+            const int kb0 = c * CHUNK_KB;
+            const int nc = (n_kb - kb0) < CHUNK_KB ? (n_kb - kb0) : CHUNK_KB;
+            // the codes of the chunk landed (the expansion waited for the same barriers)
+            for (int i = kb0 / 2; i <= (kb0 + nc - 1) / 2; ++i)
+                if (!__all_sync(0xffffffffu, mbar_wait(&ld_full[i], 0, &abort_flag, p.dev_status))) ok = false;
+            if (!ok) break;
+            tc_fence_after();
+            if (leader) {
                 for (int j = 0; j < nc; ++j) {
                     const int kb = kb0 + j;
                     const uint64_t bdesc = bdesc0 + (uint64_t)((uint32_t)kb * kstep);
@@ -171,11 +174,15 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
                 }
                 tc_commit(&chunk_done);
             }
+            __syncwarp();
+        }
+        if (leader) {
             if (ok) tc_commit(&acc_full);
             // every MMA issued above has completed once drain_bar flips
             tc_commit(&drain_bar);
             mbar_wait(&drain_bar, 0, nullptr, p.dev_status);
         }
+        __syncwarp();
     } else if (warp >= UNP_WARP0) {
         // ---------------------------------------------------------------- expand, accumulate
         const int q = warp & 3;                    // TMEM lanes 32 q .. 32 q + 31
