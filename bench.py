@@ -4,10 +4,14 @@
 
 One step is one pass of the whole hot path over one batch of synthetic input already
 resident in HBM: stage 1 (group-wise rotation + signed-INT4 row quantization, INT8
-codes) then stage 2 (W4A4 GEMM with in-shared-memory weight unpack, exact INT32
+codes) then stage 2 (W4A4 GEMM with the weight unpack into tensor memory, exact INT32
 accumulation and the scale/bias epilogue), through the C ABI.  The two stages are issued
 as ck_rotate_quant then ck_w4a4_linear on the codes (the same kernels ck_w4a4_linear
-launches from activations) so each kernel's duration is measured with CUDA events.
+launches from activations).  Each step is captured once in a CUDA graph and the timed steps
+are graph replays, back to back, with CUDA events around all of them; every step uses its own
+copy of the activations, weights, codes and outputs, and the copies together take at least
+three times the L2, so no step finds its data in the L2.  Each kernel's own duration (for the
+roofline) comes the same way from replays of that kernel alone over its copies.
 
 Rank 0 prints one JSON line.  With N > 1 (torchrun) every rank runs its own replica of
 the workload (the path has no exchange step): weak scaling, max device time over ranks.
@@ -40,7 +44,9 @@ UNIT = "TOPS"
 # INT8 dense tensor throughput relative to BF16 dense on B200 (4.5 vs 2.25 PFLOP/s nominal)
 INT8_OVER_BF16 = 2.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-L2_FLUSH_BYTES = 512 << 20
+# the B200's L2 holds 126 MB: launches cycle through copies of their data totalling at least
+# three times that, so no launch finds its own data still in the L2
+L2_COLD_FOOTPRINT = 3 * (128 << 20)
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -301,7 +307,9 @@ def config_of(case, world: int) -> dict:
     """The workload description both arms print (identical for the same case)."""
     return {"workload": case.name, "M": case.M, "K": case.K, "N": case.N, "g": case.g,
             "x_dtype": case.dtype, "rotation": case.rotation, "layout": case.layout,
-            "l2": "GPU arm: flushed (512 MiB write) before every step, outside the timed events",
+            "l2": "GPU arm: inputs larger than L2 (every launch cycles through copies of its "
+                  "activations, weights, codes and outputs totalling >= 3 x the 126 MB L2; no "
+                  "flush)",
             "parallelism": f"replicas x{world}"}
 
 
@@ -364,79 +372,135 @@ def gemm_roofline(M, N, K, case, gemm_ms, pk, pk_kind, sm_mhz, traffic):
             "tops": ops / (gemm_ms * 1e-3) / 1e12, "peak_source": f"{pk_kind} HBM copy"}
 
 
+def sets_for(per_set_bytes: int, cap: int) -> int:
+    """How many independent copies of a launch's data to cycle through so that their
+    combined footprint is at least three times the L2 (each launch's data has then been
+    evicted since its last use), at least 3 and at most `cap`."""
+    need = -(-L2_COLD_FOOTPRINT // max(1, per_set_bytes))
+    return int(max(3, min(cap, need)))
+
+
+def capture(fn) -> "torch.cuda.CUDAGraph":
+    """A CUDA graph of the kernels fn launches on the current stream (run once before)."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def timed_replays(graphs, n: int, stream) -> float:
+    """Milliseconds for n graph replays cycling through `graphs`, events around them all."""
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        graphs[i % len(graphs)].replay()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1)
+
+
 def run_ck(args, case, world, rank, local):
     from rotated_w4a4_quantized_group_b200 import ck
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     inp = W.make_linear_inputs(case)
-    if case.layout == "colmajor":       # keep the column-major layout on the device
-        x = inp["x"].t().contiguous().to(dev).t()
-    else:
-        x = inp["x"].contiguous().to(dev)
-    R = inp["R"].to(dev)
-    wp = inp["w_packed"].to(dev)
-    wsc = inp["w_scale"].to(dev)
-    bias = None if inp["bias"] is None else inp["bias"].to(dev)
     M, N, K, g = case.M, case.N, case.K, case.g
-    out = torch.empty(M, N, dtype=W.DTYPES[case.dtype], device=dev)
-    ws = torch.empty(ck.workspace_bytes(M, N, K, wp.stride(0)), dtype=torch.uint8, device=dev)
-    P = ck.workspace_codes_pitch(K)
-    off = ck.workspace_scales_offset(M, K)
-    codes = ws[: M * P].view(torch.int8).view(M, P)[:, :K]
-    scales = ws[off: off + 4 * M].view(torch.float32)
+    if case.layout == "colmajor":       # keep the column-major layout on the device
+        x_host = inp["x"].t().contiguous()
+        place = lambda t: t.to(dev).t()
+    else:
+        x_host = inp["x"].contiguous()
+        place = lambda t: t.to(dev)
+    R = inp["R"].to(dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    odt = W.DTYPES[case.dtype]
+    wsz = ck.workspace_bytes(M, N, K, inp["w_packed"].stride(0))
+    x_bytes = x_host.numel() * x_host.element_size()
+    w_bytes = inp["w_packed"].numel() + 2 * N * 4
+    out_bytes = M * N * torch.tensor([], dtype=odt).element_size()
+    # Every step reads its own copy of the activations and weights and writes its own codes and
+    # outputs: S copies whose footprint is at least three times the L2, cycled, so each step's
+    # data has left the L2 since its last use (no flush needed; events only around the steps).
+    S = sets_for(x_bytes + wsz + out_bytes + w_bytes, 64)
 
-    def step():
-        ck.ck_rotate_quant(x, R, g, codes=codes, scales=scales, dev_status=status, stream=stream)
-        ev_mid = torch.cuda.Event(enable_timing=True)
-        ev_mid.record(stream)
-        ck.ck_w4a4_linear(codes, None, 0, wp, wsc, bias, a_scale=scales, out=out,
-                          dev_status=status, stream=stream, workspace=ws)
-        return ev_mid
+    class Set:
+        pass
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
+    sets = []
+    for _ in range(S):
+        st = Set()
+        st.x = place(x_host)
+        st.wp = inp["w_packed"].to(dev)
+        st.wsc = inp["w_scale"].to(dev)
+        st.bias = None if inp["bias"] is None else inp["bias"].to(dev)
+        st.out = torch.empty(M, N, dtype=odt, device=dev)
+        st.ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+        P, off = ck.workspace_codes_pitch(K), ck.workspace_scales_offset(M, K)
+        st.codes = st.ws[: M * P].view(torch.int8).view(M, P)[:, :K]
+        st.scales = st.ws[off: off + 4 * M].view(torch.float32)
+        sets.append(st)
+
+    def stage1(st):
+        ck.ck_rotate_quant(st.x, R, g, codes=st.codes, scales=st.scales, dev_status=status)
+
+    def gemm(st):
+        ck.ck_w4a4_linear(st.codes, None, 0, st.wp, st.wsc, st.bias, a_scale=st.scales,
+                          out=st.out, dev_status=status, workspace=st.ws)
+
+    # one graph per set for the step (stage 1 then the GEMM on its codes), and one graph per
+    # kernel over all sets for the per-launch durations of the roofline
+    step_graphs = [capture(lambda st=st: (stage1(st), gemm(st))) for st in sets]
+    gemm_graph = capture(lambda: [gemm(st) for st in sets])
+    # stage 1 alone reads and writes less per launch: more activation/code copies if needed
+    s1_bytes_set = x_bytes + M * ck.workspace_codes_pitch(K) + 4 * M
+    S1 = sets_for(s1_bytes_set, 4096)
+    s1_sets = list(sets)
+    for _ in range(S1 - S):
+        st = Set()
+        st.x = place(x_host)
+        st.codes = torch.empty(M, K, dtype=torch.int8, device=dev)
+        st.scales = torch.empty(M, dtype=torch.float32, device=dev)
+        s1_sets.append(st)
+    s1_graph = capture(lambda: [stage1(st) for st in s1_sets])
+
+    for i in range(args.warmup):
+        step_graphs[i % S].replay()
+    torch.cuda.synchronize()
     barrier(world)
 
-    evs = []
     with ClockSampler(local) as clk:
         # clock soak: back-to-back steps for about a second under the sampler, so the clock
         # record covers the same load the timed steps see (untimed, before them)
         t_soak = time.perf_counter()
         while time.perf_counter() - t_soak < args.clock_soak_s:
-            for _ in range(20):
-                flush.zero_()
-                step()
+            for i in range(20):
+                step_graphs[i % S].replay()
             torch.cuda.synchronize()
         barrier(world)
         t_wall = time.perf_counter()
-        for _ in range(args.steps):
-            flush.zero_()                                    # L2 flush outside the events
-            e0 = torch.cuda.Event(enable_timing=True)
-            e2 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            e1 = step()
-            e2.record(stream)
-            evs.append((e0, e1, e2))
+        total_ms = timed_replays(step_graphs, args.steps, stream)
         barrier(world)
         t_wall = time.perf_counter() - t_wall
+        reps = max(1, -(-args.steps // S))
+        gemm_ms = timed_replays([gemm_graph], reps, stream) / (reps * S)
+        reps1 = max(1, -(-args.steps // S1))
+        s1_ms = timed_replays([s1_graph], reps1, stream) / (reps1 * S1)
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()}")
-    stage1 = [a.elapsed_time(b) for a, b, _ in evs]
-    gemm = [b.elapsed_time(c) for _, b, c in evs]
-    total_ms = sum(s + t for s, t in zip(stage1, gemm))
     total_ms = max_over_ranks(total_ms, world)
+    gemm_ms = max_over_ranks(gemm_ms, world)
+    s1_ms = max_over_ranks(s1_ms, world)
     ms_per_step = total_ms / args.steps
     flops = 2.0 * M * N * K
     value = flops * world / (ms_per_step * 1e-3) / 1e12
 
     pk, pk_kind = peaks()
-    gemm_ms = statistics.mean(gemm)
-    s1_ms = statistics.mean(stage1)
     s1_bytes = W.algorithmic_bytes_rotate_quant(M, K, g, case.dtype)
     s1_gbs = s1_bytes / (s1_ms * 1e-3) / 1e9
     gemm_file = os.path.join(ROOT, "rotated_w4a4_quantized_group_b200", "csrc", "ck_w4a4_gemm.cu")
@@ -444,6 +508,8 @@ def run_ck(args, case, world, rank, local):
     clocks = clk.summary()
     roof = gemm_roofline(M, N, K, case, gemm_ms, pk, pk_kind, clocks.get("sm_mhz"),
                          recorded_traffic(gemm_file, case.name))
+    x, out, ws, wp, wsc, bias = sets[0].x, sets[0].out, sets[0].ws, sets[0].wp, sets[0].wsc, sets[0].bias
+    footprint = S * (x_bytes + wsz + out_bytes + w_bytes)
 
     # ---- end to end through the public call with host buffers (pinned), copies timed
     xh = inp["x"].contiguous().pin_memory() if case.layout != "colmajor" else \
@@ -484,6 +550,10 @@ def run_ck(args, case, world, rank, local):
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "wall_s_timed_region": t_wall,
+        "timing": {"method": "CUDA graphs replayed back to back, CUDA events around the timed "
+                             "replays only", "sets": S, "footprint_bytes": footprint,
+                   "stage1_sets": S1, "per_kernel": "gemm_ms and stage1 ms from replays of each "
+                   "kernel alone over its sets"},
     }
     if not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(case, inp, args.cpu_budget)
@@ -491,14 +561,14 @@ def run_ck(args, case, world, rank, local):
 
 
 def run_sweep(args, local):
-    """Stage 1 alone on the 72 rotate+quantize cases: median event time over the timed
-    iterations (L2 flushed before each, outside the events), GB/s of the algorithmic bytes."""
+    """Stage 1 alone on the 72 rotate+quantize cases: each case's launches cycle through
+    copies of its activations and codes totalling at least three times the L2 (captured in one
+    CUDA graph), events around the timed replays; GB/s of the algorithmic bytes."""
     from rotated_w4a4_quantized_group_b200 import ck
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     pk, pk_kind = peaks()
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     out = []
@@ -507,39 +577,38 @@ def run_sweep(args, local):
             continue
         inp = W.make_rotate_inputs(case)
         xc = inp["x"]
-        if case.layout == "pitch2k":
-            buf = torch.zeros(case.M, 2 * case.K, dtype=xc.dtype, device=dev)
-            buf[:, :case.K] = xc.to(dev)
-            x = buf[:, :case.K]
-        else:
-            x = xc.to(dev)
         R = inp["R"].to(dev)
-        codes = torch.empty(case.M, case.K, dtype=torch.int8, device=dev)
-        scales = torch.empty(case.M, dtype=torch.float32, device=dev)
-        for _ in range(3):
-            ck.ck_rotate_quant(x, R, case.g, codes=codes, scales=scales, dev_status=status)
-        ts = []
-        for _ in range(args.steps):
-            flush.zero_()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            ck.ck_rotate_quant(x, R, case.g, codes=codes, scales=scales, dev_status=status,
-                               stream=stream)
-            e1.record(stream)
-            ts.append((e0, e1))
-        torch.cuda.synchronize()
-        ms = statistics.median(a.elapsed_time(b) for a, b in ts)
+        per_set = case.M * case.K * (xc.element_size() * (2 if case.layout == "pitch2k" else 1) + 1)
+        S = sets_for(per_set, 4096)
+        views = []
+        for _ in range(S):
+            if case.layout == "pitch2k":
+                buf = torch.zeros(case.M, 2 * case.K, dtype=xc.dtype, device=dev)
+                buf[:, :case.K] = xc.to(dev)
+                x = buf[:, :case.K]
+            else:
+                x = xc.to(dev)
+            views.append((x, torch.empty(case.M, case.K, dtype=torch.int8, device=dev),
+                          torch.empty(case.M, dtype=torch.float32, device=dev)))
+        graph = capture(lambda: [ck.ck_rotate_quant(x, R, case.g, codes=c, scales=sc,
+                                                    dev_status=status) for x, c, sc in views])
+        for _ in range(2):
+            graph.replay()
+        reps = max(1, -(-args.steps // S))
+        ms = timed_replays([graph], reps, stream) / (reps * S)
         nbytes = W.algorithmic_bytes_rotate_quant(case.M, case.K, case.g, case.dtype)
         gbs = nbytes / (ms * 1e-3) / 1e9
         out.append({"case": case.name, "us": ms * 1e3, "algorithmic_bytes": nbytes, "gbs": gbs,
-                    "frac_hbm": gbs / pk["hbm_gbs"]})
-        del x, codes, scales
+                    "frac_hbm": gbs / pk["hbm_gbs"], "launches": reps * S, "sets": S})
+        del views, graph
+        torch.cuda.synchronize()
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()}")
     return {"sweep": "rotate+quantize, stage 1 alone", "unit": "GB/s", "steps": args.steps,
             "hbm_peak_gbs": pk["hbm_gbs"], "peak_source": f"{pk_kind} HBM copy",
-            "l2": "flushed (512 MiB write) before every timed launch, outside the events",
+            "l2": "inputs larger than L2: launches cycle through copies of the activations and "
+                  "codes totalling >= 3 x the 126 MB L2, replayed from a CUDA graph; events "
+                  "around the timed replays only",
             "cases": out}
 
 
