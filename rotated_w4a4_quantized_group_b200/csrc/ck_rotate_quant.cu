@@ -1294,6 +1294,11 @@ ck_status launch_rotate_quant(const void* x, ck_dtype dt, int64_t M, int64_t K, 
         return g == 64 ? launch_mma<__half, 64>(CK_RQ_ARGS) : launch_mma<__half, 16>(CK_RQ_ARGS);
     }
 #undef CK_RQ_ARGS
+    if (dt == CK_F32 && g == 64) {
+        const ck_status st = launch_rq_f32_ffma64(x, M, K, sm, sk, R, scale_in, codes, ldq, scales,
+                                                  qmax, dev_status, stream);
+        if (st != CK_ERR_UNSUPPORTED) return st;
+    }
     if (dt == CK_F32 && g == 16) {
         const ck_status st = launch_rq_f32_g16(x, M, K, sm, sk, R, scale_in, codes, ldq, scales,
                                                qmax, dev_status, stream);

@@ -175,6 +175,29 @@ def test_rotate_quant_long_rows(dt, g, K):
                    x=x, R=R)
 
 
+@pytest.mark.parametrize("M,groups,pitch", [(77, 5, 0), (33, 1, 0), (5, 255, 0), (3, 256, 0),
+                                            (130, 60, 64), (9, 160, 0)])
+def test_rotate_quant_f32_g64_blocks(M, groups, pitch):
+    """fp32 rows at g = 64 (the FFMA kernel): blocks of whole rows, a ragged last block
+    (77 rows of 5 groups in blocks of 32), one-group rows, the longest rows one box holds (255
+    and 256 groups), a row pitch past K, and rows of 60 and 160 groups whose warp tiles of 16
+    group-rows straddle rows.  R is a non-symmetric orthogonal matrix.  Every output is
+    compared."""
+    g, K = 64, 64 * groups
+    case = W.RotateCase(f"f32_g64_{M}_{groups}", M=M, K=K, g=g, dtype="f32", seed=M + groups)
+    x = W.make_rotate_inputs(case)["x"]
+    if pitch:
+        buf = torch.zeros(M, K + pitch, dtype=x.dtype)
+        buf[:, :K] = x
+        x = buf[:, :K]
+    R = W.haar_orthogonal(g, torch.Generator().manual_seed(M * groups)).float().contiguous()
+    codes, scales = ck.ck_rotate_quant(to_device(x), R.cuda(), g)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.rotate_quant(x, R, g)
+    compare_stage1(codes.cpu().numpy(), scales.cpu().numpy(), oc, os_, torch.float32, case.name,
+                   g, x=x, R=R)
+
+
 @pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
 def test_rotate_quant_zero_rows_and_caller_zero_scale(dt):
     x = torch.randn(20, 128, generator=torch.Generator().manual_seed(5)).to(DT[dt])
