@@ -74,13 +74,14 @@ typedef enum { CK_F32 = 0, CK_F16 = 1, CK_BF16 = 2, CK_I8 = 3 } ck_dtype;
  *   codes    (M, K) int8 output, row pitch ldq >= K bytes; values in [-8, 7].
  *   scales   (M,) fp32 output, the scale each row was divided by (always written).
  *
- * Accumulation is fp32 and the rotated value is rounded to x_dtype before the
- * absmax, so a code may differ by one from an exact-arithmetic evaluation where
- * y / s lies within rounding of a half-integer.
+ * The rotated value is the sum rounded once to x_dtype before the absmax.  For fp32 input
+ * at g = 16 the sum is formed exactly (fp64 products and sums) and matches an exact
+ * evaluation bit for bit; otherwise it accumulates in fp32, so a code may differ by one
+ * from an exact-arithmetic evaluation where y / s lies within rounding of a half-integer.
  * Errors: CK_ERR_INVALID_ARG (null x/R/codes/scales, M < 0, K <= 0, K % g != 0,
  * bad g or dtype, ldq < K, R not 16-byte aligned), CK_ERR_UNSUPPORTED (a shape no kernel of
- * this build takes: an fp32 row above 56,000 channels that is neither row-major nor
- * column-major with a 16-byte pitch), CK_ERR_CUDA (launch failure).
+ * this build takes: an fp32 row of more than about 56,000 channels, unless g = 16 and x is
+ * row-major or column-major with a 16-byte-aligned pitch), CK_ERR_CUDA (launch failure).
  */
 ck_status ck_rotate_quant(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
                           int64_t stride_m, int64_t stride_k, const void* R, int g,
