@@ -817,7 +817,8 @@ __device__ __forceinline__ uint32_t tc_rt_off(int n, int k) {
 struct RqTcParams {
     int64_t M, K, ldq;
     int GR;            // group-rows per row (K / g), at most 128
-    int RB;            // rows per tile, RB * GR <= 128
+    int RB;            // rows per tile, RB * GR <= 128 (1 for split rows)
+    int L;             // split rows: group-rows per part
     int tiles;
     uint32_t box_bytes;
     uint32_t idesc;
@@ -856,12 +857,20 @@ __device__ __forceinline__ void tc_quant_store(const uint32_t (&yp)[8], const Ro
 // group-rows; each of the four 16-channel groups is its own MMA (M = 128, N = 16, K = 16) of
 // the group's 16 channels against R^T, into its own 16 accumulator columns, so no group sees
 // another group's values (an Inf stays within its group, as in the per-group rotation).
-template <typename T, int G, bool DYN, int RG = G>
+//
+// P = 2 (G = 64 only): rows of 129 to 256 group-rows, one row per tile in two parts of L <= 128
+// group-rows.  Part a is its own TMA box (64 channels x L groups of the row) and its own
+// 64-column block a of the tile's accumulator (D[l, 64 a + c] for group-row a L + l), so a
+// group's accumulator has 128 columns; the epilogue reads both blocks twice (row absmax, then
+// the codes).
+template <typename T, int G, bool DYN, int RG = G, int P = 1>
 __global__ void __launch_bounds__(kTcThreads, 1)
     rq_tc_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ R,
                  const float* __restrict__ scale_in, int8_t* __restrict__ codes,
                  float* __restrict__ scales, RqTcParams p, int* dev_status) {
-    constexpr int kAcc = kTcAcc<G>, kStages = kTcXStages<G>, kAtoms = G / 64;
+    static_assert(P == 1 || G == 64, "split rows only at G = 64");
+    constexpr int kAcc = kTcAcc<G>, kStages = kTcXStages<G>, kAtoms = P > 1 ? P : G / 64;
+    constexpr int kAccCols = G * P;                 // TMEM columns of one accumulator
     constexpr int kGrpWarps = kTcEpiWarps / kAcc;   // 4 or 8
     constexpr int kCols = G / (kGrpWarps / 4);      // accumulator columns a warp finishes
     extern __shared__ __align__(1024) unsigned char tc_smem[];
@@ -882,6 +891,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     auto issue = [&](int n) {
         const int s = n % kStages, a = n % kAtoms;
         const int t = (int)blockIdx.x + (n / kAtoms) * (int)gridDim.x;
+        if constexpr (P > 1) {   // part a of row t: groups a L .. a L + L - 1
+            mbar_arrive_expect_tx(&x_full[s], p.box_bytes);
+            tma_load_3d(xring + (size_t)s * kTcStageBytes, &xmap, &x_full[s], 0, a * p.L, t);
+            return;
+        }
         mbar_arrive_expect_tx(&x_full[s], p.box_bytes);
         tma_load_3d(xring + (size_t)s * kTcStageBytes, &xmap, &x_full[s], 64 * a, 0, t * p.RB);
     };
@@ -940,7 +954,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     fence_proxy_async_smem();   // R^T, written by threads, is read by the tensor core
     if (warp == 1) {
-        tmem_alloc(&tmem_base_sh, kAcc * G);
+        tmem_alloc(&tmem_base_sh, kAcc * kAccCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -989,7 +1003,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 tc_fence_after();
                 const uint64_t adesc = adesc0 + (uint64_t)(s * (kTcStageBytes >> 4));
-                const uint64_t bdesc = bdesc0 + (uint64_t)(a * ((G * 128) >> 4));
+                const uint64_t bdesc = bdesc0 + (uint64_t)((P > 1 ? 0 : a) * ((G * 128) >> 4));
                 if (leader) {
                     if constexpr (RG != G) {
                         // group gi: A channels 16 gi .. (32 bytes in), B = R^T rows 16 gi ..
@@ -997,13 +1011,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         constexpr uint32_t idesc16 = idesc_f16(128, RG, std::is_same<T, __nv_bfloat16>::value);
 #pragma unroll
                         for (int gi = 0; gi < G / RG; ++gi)
-                            tc_mma_f16(tmem_base + (uint32_t)(b * G + RG * gi), adesc + (uint64_t)(gi * 2),
+                            tc_mma_f16(tmem_base + (uint32_t)(b * kAccCols + (P > 1 ? 64 * a : 0) + RG * gi),
+                                       adesc + (uint64_t)(gi * 2),
                                        bdesc + (uint64_t)(gi * ((RG * 128) >> 4) + gi * 2), idesc16, 0u);
                     } else {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)   // K = 16 (32 bytes) per instruction
-                            tc_mma_f16(tmem_base + (uint32_t)(b * G), adesc + (uint64_t)(kk * 2),
-                                       bdesc + (uint64_t)(kk * 2), p.idesc, (a > 0 || kk > 0) ? 1u : 0u);
+                            tc_mma_f16(tmem_base + (uint32_t)(b * kAccCols + (P > 1 ? 64 * a : 0)),
+                                       adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), p.idesc,
+                                       ((P == 1 && a > 0) || kk > 0) ? 1u : 0u);
                     }
                     tc_commit(&x_empty[s]);
                 }
@@ -1019,6 +1035,83 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- epilogue warps
+      if constexpr (P > 1) {
+        // one row per tile; lane l of the group holds group-rows l (block 0) and L + l (block 1)
+        const int q = warp & 3;
+        const int e = warp - kTcEpiWarp0;
+        const int grp = e / kGrpWarps;
+        const int l = q * 32 + lane;
+        const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(grp * kAccCols);
+        const bool zeroer = q == 0;
+        int slot = 0;
+        for (int i = grp, j = 0; i < my_tiles; i += kAcc, ++j) {
+            const int64_t row = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
+            const bool row_ok = row < p.M;
+            if (!__all_sync(0xffffffffu, mbar_wait(&d_full[grp], (uint32_t)j & 1u, &abort_flag,
+                                                   dev_status)))
+                break;
+            tc_fence_after();
+            // pass 1: round to T, fold |y| of the lane's valid group-rows into the row absmax
+            uint32_t m2 = 0u;
+#pragma unroll 1
+            for (int a = 0; a < P; ++a) {
+                const bool gr_ok = l < p.L && a * p.L + l < p.GR;
+#pragma unroll 1
+                for (int c = 0; c < 64; c += 32) {
+                    uint32_t v[32];
+                    tc_ld_32x32b_x32(tacc + (uint32_t)(64 * a + c), v);
+                    tc_wait_ld();
+                    if (gr_ok) {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k)
+                            m2 = MmaOp<T>::absmax2(
+                                m2, MmaOp<T>::pack(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1])));
+                    }
+                }
+            }
+            if (zeroer && lane == 0) amax_sh[grp][slot == 2 ? 0 : slot + 1][0] = 0u;
+            const float2 mf = MmaOp<T>::unpack(m2);
+            if (row_ok && l < p.L) atomicMax(&amax_sh[grp][slot][0], __float_as_uint(fmax_nan(mf.x, mf.y)));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&amax_bar[grp]);
+            if (!__all_sync(0xffffffffu, mbar_wait(&amax_bar[grp], (uint32_t)j & 1u, &abort_flag,
+                                                   dev_status)))
+                break;
+            const unsigned int amax_bits = amax_sh[grp][slot][0];
+            slot = slot == 2 ? 0 : slot + 1;
+            const float sc = row_scale(__uint_as_float(amax_bits), DYN ? nullptr : scale_in, p.qmax);
+            const RowDivisor dv(sc, p.qmax);
+            if (row_ok && l == 0) scales[row] = sc;
+            // pass 2: the codes, 64 per valid group-row
+#pragma unroll 1
+            for (int a = 0; a < P; ++a) {
+                const int gr = a * p.L + l;
+                const bool gr_ok = row_ok && l < p.L && gr < p.GR;
+                int8_t* dst = codes + row * p.ldq + (int64_t)gr * G;
+#pragma unroll 1
+                for (int c = 0; c < 64; c += 32) {
+                    uint32_t v[32];
+                    tc_ld_32x32b_x32(tacc + (uint32_t)(64 * a + c), v);
+                    tc_wait_ld();
+                    if (gr_ok) {
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            uint32_t y8[8];
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                y8[k] = MmaOp<T>::pack(__uint_as_float(v[16 * u + 2 * k]),
+                                                       __uint_as_float(v[16 * u + 2 * k + 1]));
+                            tc_quant_store<T, DYN>(y8, dv, scale_in, dst + c + 16 * u,
+                                                   p.vec_codes != 0);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&d_empty[grp]);   // done reading the accumulator
+        }
+      } else {
         const int q = warp & 3;                          // TMEM lanes 32q .. 32q + 31
         const int e = warp - kTcEpiWarp0;
         const int grp = e / kGrpWarps;                   // tiles i = grp (mod kAcc), accumulator grp
@@ -1027,7 +1120,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool valid = L < p.RB * p.GR;
         const int r = valid ? L / p.GR : 0, rho = valid ? L - r * p.GR : 0;
         const uint32_t tacc =
-            tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(grp * G + h * kCols);
+            tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(grp * kAccCols + h * kCols);
         const bool zeroer = q == 0 && h == 0;
         int slot = 0;
         for (int i = grp, j = 0; i < my_tiles; i += kAcc, ++j) {
@@ -1114,18 +1207,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (lane == 0) mbar_arrive(&d_empty[grp]);   // done reading the accumulator
             }
         }
+      }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTcAcc<G> * G);
+        tmem_dealloc(tmem_base, kAcc * kAccCols);
     }
 }
 
-// Tensor-core kernel for bf16/fp16, g in {64, 256}, K / g <= 128.  Returns
-// CK_ERR_UNSUPPORTED otherwise.
-template <typename T, int G, int RG = G>
+// Tensor-core kernel for bf16/fp16, g in {64, 256}, K / g <= 128 (P = 1), or g = 64 rows of
+// 129 .. 128 P groups split in P parts.  Returns CK_ERR_UNSUPPORTED otherwise.
+template <typename T, int G, int RG = G, int P = 1>
 static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, const void* R,
                            const float* scale_in, int8_t* codes, int64_t ldq, float* scales,
                            int qmax, int* dev_status, cudaStream_t stream,
@@ -1134,13 +1228,15 @@ static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, cons
     p.M = M;
     p.K = K;
     p.ldq = ldq;
-    if (K % G != 0 || K / G < 1 || K / G > 128) return CK_ERR_UNSUPPORTED;
+    if (K % G != 0 || K / G < 1 || K / G > 128 * P || (P > 1 && K / G <= 128))
+        return CK_ERR_UNSUPPORTED;
     p.GR = (int)(K / G);
-    p.RB = 128 / p.GR;
+    p.RB = P > 1 ? 1 : 128 / p.GR;
+    p.L = P > 1 ? (p.GR + P - 1) / P : p.GR;
     const int64_t tiles = (M + p.RB - 1) / p.RB;
     if (tiles >= (1LL << 31) / p.RB) return CK_ERR_UNSUPPORTED;
     p.tiles = (int)tiles;
-    p.box_bytes = (uint32_t)(p.RB * p.GR * 128);
+    p.box_bytes = (uint32_t)(p.RB * p.L * 128);
     p.idesc = idesc_f16(128, G, std::is_same<T, __nv_bfloat16>::value);
     p.vec_codes = (aligned(codes, 16) && ldq % 16 == 0) ? 1 : 0;
     p.qmax = qmax;
@@ -1150,7 +1246,7 @@ static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, cons
     CUtensorMap map;
     const uint64_t dims[3] = {(uint64_t)G, (uint64_t)p.GR, (uint64_t)M};
     const uint64_t strides[2] = {(uint64_t)G * 2, (uint64_t)sm * 2};
-    const uint32_t box[3] = {64u, (uint32_t)p.GR, (uint32_t)p.RB};
+    const uint32_t box[3] = {64u, (uint32_t)p.L, (uint32_t)p.RB};
     ck_status st = encode_tma(&map, tdt, 3, x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != CK_OK) return st;
 
@@ -1164,7 +1260,7 @@ static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, cons
                                                  scales, p, dev_status);
         return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
     };
-    return scale_in ? run(rq_tc_kernel<T, G, false, RG>) : run(rq_tc_kernel<T, G, true, RG>);
+    return scale_in ? run(rq_tc_kernel<T, G, false, RG, P>) : run(rq_tc_kernel<T, G, true, RG, P>);
 }
 
 // ===================================================================== host launch
@@ -1273,13 +1369,19 @@ ck_status launch_rotate_quant(const void* x, ck_dtype dt, int64_t M, int64_t K, 
         else
             st = g == 64 ? launch_tc<__half, 64>(CK_RQ_ARGS) : launch_tc<__half, 256>(CK_RQ_ARGS);
         if (st != CK_ERR_UNSUPPORTED) return st;
+        if (g == 64) {   // rows of 129 to 256 groups, in two parts
+            st = bf ? launch_tc<__nv_bfloat16, 64, 64, 2>(CK_RQ_ARGS) : launch_tc<__half, 64, 64, 2>(CK_RQ_ARGS);
+            if (st != CK_ERR_UNSUPPORTED) return st;
+        }
     }
     // g = 16 rows of whole 64-channel groups: the tensor-core kernel with a block-diagonal R
     const bool tc16_ok = half16 && g == 16 && K % 64 == 0 && sk == 1 && aligned(x, 16) &&
                          sm % 8 == 0 && sm > 0 && M < (1LL << 31);
     if (tc16_ok) {
-        const ck_status st = bf ? launch_tc<__nv_bfloat16, 64, 16>(CK_RQ_ARGS)
-                                : launch_tc<__half, 64, 16>(CK_RQ_ARGS);
+        ck_status st = bf ? launch_tc<__nv_bfloat16, 64, 16>(CK_RQ_ARGS)
+                          : launch_tc<__half, 64, 16>(CK_RQ_ARGS);
+        if (st != CK_ERR_UNSUPPORTED) return st;
+        st = bf ? launch_tc<__nv_bfloat16, 64, 16, 2>(CK_RQ_ARGS) : launch_tc<__half, 64, 16, 2>(CK_RQ_ARGS);
         if (st != CK_ERR_UNSUPPORTED) return st;
     }
     if (mma_ok) {

@@ -140,14 +140,18 @@ def test_rotate_quant_small_every_row(dt, g, layout):
 
 @pytest.mark.parametrize("dt", ["f16", "bf16"])
 @pytest.mark.parametrize("g,groups,M", [(64, 1, 1000), (64, 127, 200), (64, 128, 160), (64, 129, 20),
+                                        (64, 131, 9), (64, 160, 301), (64, 255, 7), (64, 256, 150),
+                                        (64, 257, 3), (16, 516, 11), (16, 640, 200), (16, 1024, 5),
                                         (256, 1, 1000), (256, 43, 333), (256, 128, 150),
                                         (256, 129, 3)])
 def test_rotate_quant_tile_shapes(dt, g, groups, M):
-    """Rows of 1 to 129 groups: a tile packs floor(128 / groups) rows, so these cover a tile of
-    128 one-group rows, one row of 127 or 128 groups, a ragged last tile, more tiles than SMs
-    (150 rows of 128 groups), and the first row length past 128 groups, which another kernel
-    takes.  R is a non-symmetric orthogonal matrix, so R and R^T give different results.
-    Every output is compared."""
+    """Rows of 1 to 257 groups: a tile packs floor(128 / groups) rows, so these cover a tile of
+    128 one-group rows, one row of 127 or 128 groups, a ragged last tile and more tiles than SMs
+    (150 rows of 128 groups).  Rows of 129 to 256 64-channel group-rows (g = 64, and g = 16 at
+    K = 64 x 129 .. 64 x 256) are split in two parts of a tile, evenly or not (131 groups: 66 +
+    65), 301 rows give more tiles than SMs, and the first lengths past each kernel's limit (257
+    groups at g = 64, 129 at g = 256) go to other kernels.  R is a non-symmetric orthogonal
+    matrix, so R and R^T give different results.  Every output is compared."""
     case = W.RotateCase(f"tiles_{dt}_{g}_{groups}", M=M, K=g * groups, g=g, dtype=dt,
                         seed=groups + g)
     x = W.make_rotate_inputs(case)["x"]
