@@ -56,7 +56,7 @@ constexpr int BW = 128;                  // weight rows (output channels) per ti
 constexpr int BK = 128;                  // K elements per stage (bytes of codes)
 constexpr int BNA_MAX = 192;             // activation rows per tile: MMA N
 constexpr int XS_MAX = 8;                // code super-stages in shared memory
-constexpr int G_MAX = 4;                 // k-blocks per super-stage
+constexpr int G_MAX = 2;                 // k-blocks per super-stage (one 3-D box of each operand)
 constexpr int NB_MAX = 4;                // TMEM weight buffers (one super-stage each)
 constexpr int W_ST_MAX = 2 * G_MAX;      // packed-weight k-block buffers: G per unpack set
 constexpr int ND = 16;                   // super-stage completion barriers (> XS_MAX + 1)
@@ -360,9 +360,6 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         uint32_t buf = set;   // TMEM weight buffer of super-stage ss: ss % NB
         const unsigned char* wset = w_ring + (size_t)set * G * W_BYTES;
         for (uint32_t ss = set; ok && ss < my_ss; ss += UNP_SETS) {
-            // the buffer is free once the MMAs of its previous super-stage (ss - NB) completed
-            if (ss >= NB && !__all_sync(0xffffffffu, wait_done(ss - NB))) break;
-            tc_fence_after();
             const uint32_t t_buf = t_row + buf * G * A_STAGE_COLS;
             const uint32_t n_k = ss_nk(ss);
             // every lane waits; the warp leaves together (tcgen05.st below is .aligned)
@@ -382,20 +379,27 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&w_empty[set]);
+            // expand into registers before waiting for the tensor-memory buffer, so that only
+            // the stores lie between the MMAs of super-stage ss - NB completing and those of ss
+            uint32_t v[G_MAX][16];
 #pragma unroll
             for (uint32_t j = 0; j < (uint32_t)G_MAX; ++j) {
                 if (j < n_k) {
-                    uint32_t v[16];
                     const uint32_t c[8] = {c0[j].x, c0[j].y, c0[j].z, c0[j].w,
                                            c1[j].x, c1[j].y, c1[j].z, c1[j].w};
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        if (X16) unpack_word_x16(c[i], v[2 * i], v[2 * i + 1]);
-                        else unpack_word_s(c[i], v[2 * i], v[2 * i + 1]);
+                        if (X16) unpack_word_x16(c[i], v[j][2 * i], v[j][2 * i + 1]);
+                        else unpack_word_s(c[i], v[j][2 * i], v[j][2 * i + 1]);
                     }
-                    tc_st_32x32b_x16(t_buf + j * A_STAGE_COLS, v);
                 }
             }
+            // the buffer is free once the MMAs of its previous super-stage (ss - NB) completed
+            if (ss >= NB && !__all_sync(0xffffffffu, wait_done(ss - NB))) break;
+            tc_fence_after();
+#pragma unroll
+            for (uint32_t j = 0; j < (uint32_t)G_MAX; ++j)
+                if (j < n_k) tc_st_32x32b_x16(t_buf + j * A_STAGE_COLS, v[j]);
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
