@@ -345,7 +345,7 @@ def run_reference(args, case, world, rank):
     }
 
 
-def gemm_roofline(M, N, K, case, gemm_ms, pk, pk_kind, sm_mhz, traffic):
+def gemm_roofline(M, N, K, case, gemm_ms, pk, pk_kind, sm_mhz, traffic, kernel="w4a4_gemm_kernel"):
     """Roofline of the GEMM launch: tensor-bound when its operation intensity is above the
     ridge (INT8 peak / HBM bandwidth), HBM-bound below it (small M)."""
     ops = 2.0 * M * N * K
@@ -358,7 +358,7 @@ def gemm_roofline(M, N, K, case, gemm_ms, pk, pk_kind, sm_mhz, traffic):
         mma_rate = 148 * 8192 * 2 * sm_mhz * 1e6 / 1e12
     if ops / nbytes >= ridge:
         achieved = ops / (gemm_ms * 1e-3) / 1e12
-        r = {"bound": "tensor", "kernel": "w4a4_gemm_kernel", "achieved": achieved,
+        r = {"bound": "tensor", "kernel": kernel, "achieved": achieved,
              "peak": int8_peak, "unit": "TOPS", "frac": achieved / int8_peak, "traffic": traffic,
              "peak_source": f"{pk_kind} bf16 burst x {INT8_OVER_BF16} (INT8:BF16 nominal)"}
         if mma_rate:
@@ -366,7 +366,7 @@ def gemm_roofline(M, N, K, case, gemm_ms, pk, pk_kind, sm_mhz, traffic):
             r["kind_i8_rate_tops"] = mma_rate
         return r
     achieved = nbytes / (gemm_ms * 1e-3) / 1e9
-    return {"bound": "hbm", "kernel": "w4a4_gemm_kernel", "achieved": achieved,
+    return {"bound": "hbm", "kernel": kernel, "achieved": achieved,
             "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
             "traffic": traffic, "algorithmic_bytes": nbytes,
             "tops": ops / (gemm_ms * 1e-3) / 1e12, "peak_source": f"{pk_kind} HBM copy"}
@@ -503,11 +503,15 @@ def run_ck(args, case, world, rank, local):
     pk, pk_kind = peaks()
     s1_bytes = W.algorithmic_bytes_rotate_quant(M, K, g, case.dtype)
     s1_gbs = s1_bytes / (s1_ms * 1e-3) / 1e9
-    gemm_file = os.path.join(ROOT, "rotated_w4a4_quantized_group_b200", "csrc", "ck_w4a4_gemm.cu")
-    rq_file = os.path.join(ROOT, "rotated_w4a4_quantized_group_b200", "csrc", "ck_rotate_quant.cu")
+    csrc = os.path.join(ROOT, "rotated_w4a4_quantized_group_b200", "csrc")
+    # the source of the kernels this workload runs (few rows: the split-K GEMM; fp32: the fp32
+    # stage-1 kernels)
+    gemm_kernel = "w4a4_splitk_kernel" if M <= 64 else "w4a4_gemm_kernel"
+    gemm_file = os.path.join(csrc, "ck_w4a4_splitk.cu" if M <= 64 else "ck_w4a4_gemm.cu")
+    rq_file = os.path.join(csrc, "ck_rq_f32.cu" if case.dtype == "f32" else "ck_rotate_quant.cu")
     clocks = clk.summary()
     roof = gemm_roofline(M, N, K, case, gemm_ms, pk, pk_kind, clocks.get("sm_mhz"),
-                         recorded_traffic(gemm_file, case.name))
+                         recorded_traffic(gemm_file, case.name), gemm_kernel)
     x, out, ws, wp, wsc, bias = sets[0].x, sets[0].out, sets[0].ws, sets[0].wp, sets[0].wsc, sets[0].bias
     footprint = S * (x_bytes + wsz + out_bytes + w_bytes)
 
