@@ -235,11 +235,14 @@ __global__ void __launch_bounds__(rqf32::kThreads, 2)
             // (m GBb + j - b GBb) of the box
             const int o16 = (ngroups + 15) / 16;
             const int wpr = p.RB >= kWarps ? 1 : kWarps / p.RB;
+            // the box of group j: 0 when one box holds the slice's groups, else j / 256 (boxes
+            // of 256 groups)
+            const int bshift = p.nboxes == 1 ? 30 : 8;
             for (int mrow = warp / wpr; ok && mrow < p.RB; mrow += kWarps / wpr) {
                 float mx = 0.f;
                 for (int o = warp % wpr; ok && o < o16; o += wpr) {
                     const int jlast = (16 * o + 15) < ngroups ? (16 * o + 15) : (ngroups - 1);
-                    if (!wait_box(jlast / p.GBb)) {
+                    if (!wait_box(jlast >> bshift)) {
                         ok = false;
                         break;
                     }
@@ -251,7 +254,7 @@ __global__ void __launch_bounds__(rqf32::kThreads, 2)
                     for (int t2 = 0; t2 < 2; ++t2) {
                         const int j = 16 * o + 8 * t2 + fr;
                         jv[t2] = j < ngroups;
-                        const int b = jv[t2] ? j / p.GBb : 0;
+                        const int b = jv[t2] ? j >> bshift : 0;
                         bxs[t2] = tile + (size_t)b * box_floats;
                         rows_[t2] = jv[t2] ? (uint32_t)(mrow * p.GBb + (j - b * p.GBb)) : 0u;
                         const uint32_t ph = (rows_[t2] >> 1) & 3u;
@@ -340,13 +343,19 @@ __global__ void __launch_bounds__(rqf32::kThreads, 2)
                     }
                 }
             } else {
-                // thread -> (row m, group j) of the slice: 16 consecutive values
-                for (int u = tid; u < p.RB * ngroups; u += kThreads) {
-                    const int m = u / ngroups, j = u - m * ngroups;
-                    if (m >= rows) continue;
+                // thread -> (row m, group j) of the slice: 16 consecutive values; (m, j) advance
+                // by kThreads groups at a time without a division
+                int m = tid / ngroups, j = tid - m * ngroups;
+                const int dm = kThreads / ngroups, dj = kThreads - dm * ngroups;
+                for (; m < rows; m += dm, j += dj) {
+                    if (j >= ngroups) {
+                        j -= ngroups;
+                        ++m;
+                        if (m >= rows) break;
+                    }
                     RowDivisor dv(row_s[m], p.qmax);
                     dv.r = row_r[m];
-                    const int b = j / p.GBb;
+                    const int b = p.nboxes == 1 ? 0 : j >> 8;   // boxes of 256 groups
                     const float* bx = tile + (size_t)b * box_floats;
                     const uint32_t row = (uint32_t)(m * p.GBb + (j - b * p.GBb));
                     float y[16];
@@ -504,6 +513,8 @@ __global__ void __launch_bounds__(rqff::kThreads, 2)
                 // write y over x; fold |y| into the maximum of each group-row's row
                 float run = 0.f;
                 int run_row = -1;
+                // the row of group-row gr0 + r: one division per tile, then a count
+                int row_of = gr0 / gpr, left = gpr - (gr0 - row_of * gpr);
 #pragma unroll
                 for (int r = 0; r < kTileGR; ++r) {
                     if (r < nr) {
@@ -513,7 +524,12 @@ __global__ void __launch_bounds__(rqff::kThreads, 2)
 #pragma unroll
                         for (int o = 16; o > 0; o >>= 1)
                             mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                        const int row = (gr0 + r) / gpr;
+                        if (left == 0) {
+                            ++row_of;
+                            left = gpr;
+                        }
+                        --left;
+                        const int row = row_of;
                         if (row != run_row) {
                             if (run_row >= 0 && lane == 0) atomicMax(&amax_sh[run_row], __float_as_uint(run));
                             run_row = row;
@@ -541,8 +557,8 @@ __global__ void __launch_bounds__(rqff::kThreads, 2)
         if (ok) {
             const int rows = (int)((p.M - m0) < p.RB ? (p.M - m0) : p.RB);
             const int cpr = (int)(p.K / 16);   // 16-value chunks per row
-            for (int u = tid; u < rows * cpr; u += kThreads) {
-                const int m = u / cpr, j = u - m * cpr;
+            for (int m = 0; m < rows; ++m)
+            for (int j = tid; j < cpr; j += kThreads) {
                 RowDivisor dv(row_s[m], p.qmax);
                 dv.r = row_r[m];
                 const float* src = xt + (size_t)m * p.K + 16 * j;
@@ -601,6 +617,9 @@ ck_status launch_rq_f32_ffma64(const void* x, int64_t M, int64_t K, int64_t sm, 
     int64_t rb = (int64_t)((budget - r_bytes) / (2 * row_bytes));
     if (rb < 1) return CK_ERR_UNSUPPORTED;
     if (rb > kMaxRB) rb = kMaxRB;
+    // few rows: blocks small enough that every SM gets work
+    const int64_t spread = (M + 2LL * num_sms() - 1) / (2LL * num_sms());
+    if (rb > spread) rb = spread < 1 ? 1 : spread;
     if (rb > M) rb = M;
     RqFfmaParams p;
     p.M = M;

@@ -179,14 +179,14 @@ def test_rotate_quant_long_rows(dt, g, K):
                    x=x, R=R)
 
 
-@pytest.mark.parametrize("M,groups,pitch", [(77, 5, 0), (33, 1, 0), (5, 255, 0), (3, 256, 0),
-                                            (130, 60, 64), (9, 160, 0)])
+@pytest.mark.parametrize("M,groups,pitch", [(700, 5, 0), (33, 1, 0), (5, 255, 0), (3, 256, 0),
+                                            (1300, 60, 64), (9, 160, 0)])
 def test_rotate_quant_f32_g64_blocks(M, groups, pitch):
-    """fp32 rows at g = 64 (the FFMA kernel): blocks of whole rows, a ragged last block
-    (77 rows of 5 groups in blocks of 32), one-group rows, the longest rows one box holds (255
+    """fp32 rows at g = 64 (the FFMA kernel): blocks of whole rows with a ragged last block
+    (700 rows of 5 groups in blocks of 3), one-group rows, the longest rows one box holds (255
     and 256 groups), a row pitch past K, and rows of 60 and 160 groups whose warp tiles of 16
-    group-rows straddle rows.  R is a non-symmetric orthogonal matrix.  Every output is
-    compared."""
+    group-rows straddle rows (1300 rows of 60 groups in blocks of 3).  R is a non-symmetric
+    orthogonal matrix.  Every output is compared."""
     g, K = 64, 64 * groups
     case = W.RotateCase(f"f32_g64_{M}_{groups}", M=M, K=K, g=g, dtype="f32", seed=M + groups)
     x = W.make_rotate_inputs(case)["x"]
