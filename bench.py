@@ -380,6 +380,16 @@ def sets_for(per_set_bytes: int, cap: int) -> int:
     return int(max(3, min(cap, need)))
 
 
+def kernel_sources(case):
+    """(GEMM kernel name, GEMM source, stage-1 source) of the kernels a workload runs: few rows
+    take the split-K GEMM, fp32 activations the fp32 stage-1 kernels."""
+    csrc = os.path.join(ROOT, "rotated_w4a4_quantized_group_b200", "csrc")
+    few = case.M <= 64
+    return ("w4a4_splitk_kernel" if few else "w4a4_gemm_kernel",
+            os.path.join(csrc, "ck_w4a4_splitk.cu" if few else "ck_w4a4_gemm.cu"),
+            os.path.join(csrc, "ck_rq_f32.cu" if case.dtype == "f32" else "ck_rotate_quant.cu"))
+
+
 def capture(fn) -> "torch.cuda.CUDAGraph":
     """A CUDA graph of the kernels fn launches on the current stream (run once before)."""
     fn()
@@ -503,12 +513,7 @@ def run_ck(args, case, world, rank, local):
     pk, pk_kind = peaks()
     s1_bytes = W.algorithmic_bytes_rotate_quant(M, K, g, case.dtype)
     s1_gbs = s1_bytes / (s1_ms * 1e-3) / 1e9
-    csrc = os.path.join(ROOT, "rotated_w4a4_quantized_group_b200", "csrc")
-    # the source of the kernels this workload runs (few rows: the split-K GEMM; fp32: the fp32
-    # stage-1 kernels)
-    gemm_kernel = "w4a4_splitk_kernel" if M <= 64 else "w4a4_gemm_kernel"
-    gemm_file = os.path.join(csrc, "ck_w4a4_splitk.cu" if M <= 64 else "ck_w4a4_gemm.cu")
-    rq_file = os.path.join(csrc, "ck_rq_f32.cu" if case.dtype == "f32" else "ck_rotate_quant.cu")
+    gemm_kernel, gemm_file, rq_file = kernel_sources(case)
     clocks = clk.summary()
     roof = gemm_roofline(M, N, K, case, gemm_ms, pk, pk_kind, clocks.get("sm_mhz"),
                          recorded_traffic(gemm_file, case.name), gemm_kernel)

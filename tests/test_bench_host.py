@@ -113,3 +113,26 @@ def test_clock_sampler_runs_without_a_gpu():
     with bench.ClockSampler(0) as c:
         pass
     assert isinstance(c.summary(), dict)
+
+
+def test_sets_for_cover_three_l2s():
+    """Launch data is cycled through copies totalling at least three L2s (and at least 3)."""
+    import bench
+    l2x3 = bench.L2_COLD_FOOTPRINT
+    for per_set in (1, 8 << 20, 94 << 20, 165 << 20, 485 << 20, 2 << 30):
+        n = bench.sets_for(per_set, 4096)
+        assert n >= 3
+        assert n * per_set >= l2x3 or n == 4096
+        assert (n - 1) * per_set < l2x3 or n == 3
+    assert bench.sets_for(1, 64) == 64
+
+
+def test_kernel_sources_follow_the_workload():
+    import os
+    import bench
+    from rotated_w4a4_quantized_group_b200 import workloads as W
+    for name, case in W.LINEAR_CASES.items():
+        kern, gemm_file, rq_file = bench.kernel_sources(case)
+        assert os.path.exists(gemm_file) and os.path.exists(rq_file)
+        assert (kern == "w4a4_splitk_kernel") == (case.M <= 64)
+        assert os.path.basename(rq_file) == ("ck_rq_f32.cu" if case.dtype == "f32" else "ck_rotate_quant.cu")
