@@ -1401,6 +1401,11 @@ ck_status launch_rotate_quant(const void* x, ck_dtype dt, int64_t M, int64_t K, 
                                                   qmax, dev_status, stream);
         if (st != CK_ERR_UNSUPPORTED) return st;
     }
+    if (dt == CK_F32 && g == 256) {
+        const ck_status st = launch_rq_f32_ffma256(x, M, K, sm, sk, R, scale_in, codes, ldq, scales,
+                                                   qmax, dev_status, stream);
+        if (st != CK_ERR_UNSUPPORTED) return st;
+    }
     if (dt == CK_F32 && g == 16) {
         const ck_status st = launch_rq_f32_g16(x, M, K, sm, sk, R, scale_in, codes, ldq, scales,
                                                qmax, dev_status, stream);

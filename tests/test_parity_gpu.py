@@ -202,6 +202,29 @@ def test_rotate_quant_f32_g64_blocks(M, groups, pitch):
                    g, x=x, R=R)
 
 
+@pytest.mark.parametrize("M,groups,pitch", [(703, 3, 0), (100, 15, 0), (300, 15, 64), (5, 40, 0),
+                                            (3, 48, 0), (150, 1, 0)])
+def test_rotate_quant_f32_g256_blocks(M, groups, pitch):
+    """fp32 rows at g = 256 (the FFMA kernel with R passing through shared memory in four
+    blocks of 64 rows): blocks of 5 rows with a ragged last one (703 rows of 3 groups), one-row
+    blocks (15, 40 and 48 groups), a row pitch past K, and one-group rows.  The partial sums
+    continue across the four passes, so each value is the in-order fp32 FMA chain.  R is a
+    non-symmetric orthogonal matrix.  Every output is compared."""
+    g, K = 256, 256 * groups
+    case = W.RotateCase(f"f32_g256_{M}_{groups}", M=M, K=K, g=g, dtype="f32", seed=M + groups)
+    x = W.make_rotate_inputs(case)["x"]
+    if pitch:
+        buf = torch.zeros(M, K + pitch, dtype=x.dtype)
+        buf[:, :K] = x
+        x = buf[:, :K]
+    R = W.haar_orthogonal(g, torch.Generator().manual_seed(M * groups)).float().contiguous()
+    codes, scales = ck.ck_rotate_quant(to_device(x), R.cuda(), g)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.rotate_quant(x, R, g)
+    compare_stage1(codes.cpu().numpy(), scales.cpu().numpy(), oc, os_, torch.float32, case.name,
+                   g, x=x, R=R)
+
+
 @pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
 def test_rotate_quant_zero_rows_and_caller_zero_scale(dt):
     x = torch.randn(20, 128, generator=torch.Generator().manual_seed(5)).to(DT[dt])
