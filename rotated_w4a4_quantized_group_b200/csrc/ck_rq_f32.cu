@@ -488,25 +488,38 @@ __global__ void __launch_bounds__(rqff::kThreads, 2)
 #pragma unroll
                 for (int r = 0; r < kTileGR; ++r) acc0[r] = acc1[r] = 0.f;
                 const float* xg = xt + (size_t)gr0 * 64;
+                // one step of four values of i for group-row r of the tile
+                auto step = [&](int r, int i, const float2 (&rq)[4]) {
+                    const float4 xv = *reinterpret_cast<const float4*>(xg + r * 64 + i);
+                    acc0[r] = __fmaf_rn(xv.x, rq[0].x, acc0[r]);
+                    acc1[r] = __fmaf_rn(xv.x, rq[0].y, acc1[r]);
+                    acc0[r] = __fmaf_rn(xv.y, rq[1].x, acc0[r]);
+                    acc1[r] = __fmaf_rn(xv.y, rq[1].y, acc1[r]);
+                    acc0[r] = __fmaf_rn(xv.z, rq[2].x, acc0[r]);
+                    acc1[r] = __fmaf_rn(xv.z, rq[2].y, acc1[r]);
+                    acc0[r] = __fmaf_rn(xv.w, rq[3].x, acc0[r]);
+                    acc1[r] = __fmaf_rn(xv.w, rq[3].y, acc1[r]);
+                };
+                if (nr == kTileGR) {   // a full tile: no predicates in the loop
 #pragma unroll 1
-                for (int i = 0; i < 64; i += 4) {
-                    float2 rq[4];
+                    for (int i = 0; i < 64; i += 4) {
+                        float2 rq[4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        rq[q] = *reinterpret_cast<const float2*>(Rs + (i + q) * 64 + 2 * lane);
+                        for (int q = 0; q < 4; ++q)
+                            rq[q] = *reinterpret_cast<const float2*>(Rs + (i + q) * 64 + 2 * lane);
 #pragma unroll
-                    for (int r = 0; r < kTileGR; ++r) {
-                        if (r < nr) {
-                            const float4 xv = *reinterpret_cast<const float4*>(xg + r * 64 + i);
-                            acc0[r] = __fmaf_rn(xv.x, rq[0].x, acc0[r]);
-                            acc1[r] = __fmaf_rn(xv.x, rq[0].y, acc1[r]);
-                            acc0[r] = __fmaf_rn(xv.y, rq[1].x, acc0[r]);
-                            acc1[r] = __fmaf_rn(xv.y, rq[1].y, acc1[r]);
-                            acc0[r] = __fmaf_rn(xv.z, rq[2].x, acc0[r]);
-                            acc1[r] = __fmaf_rn(xv.z, rq[2].y, acc1[r]);
-                            acc0[r] = __fmaf_rn(xv.w, rq[3].x, acc0[r]);
-                            acc1[r] = __fmaf_rn(xv.w, rq[3].y, acc1[r]);
-                        }
+                        for (int r = 0; r < kTileGR; ++r) step(r, i, rq);
+                    }
+                } else {
+#pragma unroll 1
+                    for (int i = 0; i < 64; i += 4) {
+                        float2 rq[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            rq[q] = *reinterpret_cast<const float2*>(Rs + (i + q) * 64 + 2 * lane);
+#pragma unroll
+                        for (int r = 0; r < kTileGR; ++r)
+                            if (r < nr) step(r, i, rq);
                     }
                 }
                 __syncwarp();   // every lane has read the tile's x before any lane overwrites it
