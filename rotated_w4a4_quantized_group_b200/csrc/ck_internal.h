@@ -49,6 +49,9 @@ ck_status launch_rotate_quant(const void* x, ck_dtype dt, int64_t M, int64_t K, 
 
 // Stage 1 for fp32 input with g = 16, row-major or column-major, on the FP64 tensor-core
 // rotation (ck_rq_f32.cu).  Returns CK_ERR_UNSUPPORTED for shapes or layouts it does not take.
+ck_status launch_rq_tf32(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
+                         const void* R, const float* scale_in, int8_t* codes, int64_t ldq,
+                         float* scales, int qmax, int* dev_status, cudaStream_t stream);
 ck_status launch_rq_f32_ffma64(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
                                const void* R, const float* scale_in, int8_t* codes, int64_t ldq,
                                float* scales, int qmax, int* dev_status, cudaStream_t stream);

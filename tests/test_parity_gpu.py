@@ -261,6 +261,27 @@ def test_rotate_quant_non_finite_follows_the_oracle_convention(dt):
                    x=x, R=R, rows=[0, 3])
 
 
+@pytest.mark.parametrize("g", [64, 256])
+def test_rotate_quant_f32_non_finite_at_wide_groups(g):
+    """fp32 at g = 64 (split-TF32 tensor cores) and g = 256: a NaN makes its row's scale NaN
+    and codes 0, an inf makes its row's scale inf, as in the exact rotation.  R is a Hadamard
+    matrix, whose entries are exact in TF32 (its low parts are all zero), so an inf in the
+    high part of a split would meet zeros; other rows follow the parity rule."""
+    x = torch.randn(4, 2 * g, generator=torch.Generator().manual_seed(7))
+    x[1, 5] = float("nan")
+    x[2, g + 9] = float("inf")
+    R = W.hadamard(g).float()
+    codes, scales = ck.ck_rotate_quant(x.cuda(), R.cuda(), g)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.rotate_quant(x, R, g)
+    gs = scales.cpu().numpy()
+    assert math.isnan(gs[1]) and math.isnan(os_[1])
+    assert math.isinf(gs[2]) and math.isinf(os_[2])
+    np.testing.assert_array_equal(codes.cpu().numpy()[1:3], oc[1:3])
+    compare_stage1(codes.cpu().numpy()[[0, 3]], gs[[0, 3]], oc[[0, 3]], os_[[0, 3]], torch.float32,
+                   "", g, x=x, R=R, rows=[0, 3])
+
+
 def test_rotate_quant_unaligned_and_strided_views():
     base = torch.randn(50, 3 * 64 + 1, generator=torch.Generator().manual_seed(7)).to(torch.bfloat16)
     x = base[:, 1:1 + 128]                       # row pitch 193, base offset by one element
