@@ -52,9 +52,6 @@ ck_status launch_rotate_quant(const void* x, ck_dtype dt, int64_t M, int64_t K, 
 ck_status launch_rq_tf32(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
                          const void* R, const float* scale_in, int8_t* codes, int64_t ldq,
                          float* scales, int qmax, int* dev_status, cudaStream_t stream);
-ck_status launch_rq_f32_ffma64(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
-                               const void* R, const float* scale_in, int8_t* codes, int64_t ldq,
-                               float* scales, int qmax, int* dev_status, cudaStream_t stream);
 ck_status launch_rq_f32_ffma256(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
                                 const void* R, const float* scale_in, int8_t* codes, int64_t ldq,
                                 float* scales, int qmax, int* dev_status, cudaStream_t stream);

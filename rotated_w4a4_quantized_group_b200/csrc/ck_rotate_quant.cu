@@ -1397,11 +1397,8 @@ ck_status launch_rotate_quant(const void* x, ck_dtype dt, int64_t M, int64_t K, 
     }
 #undef CK_RQ_ARGS
     if (dt == CK_F32 && g == 64) {
-        ck_status st = launch_rq_tf32(x, M, K, sm, sk, R, scale_in, codes, ldq, scales, qmax,
-                                      dev_status, stream);
-        if (st != CK_ERR_UNSUPPORTED) return st;
-        st = launch_rq_f32_ffma64(x, M, K, sm, sk, R, scale_in, codes, ldq, scales, qmax,
-                                  dev_status, stream);
+        const ck_status st = launch_rq_tf32(x, M, K, sm, sk, R, scale_in, codes, ldq, scales,
+                                            qmax, dev_status, stream);
         if (st != CK_ERR_UNSUPPORTED) return st;
     }
     if (dt == CK_F32 && g == 256) {

@@ -394,279 +394,6 @@ __global__ void __launch_bounds__(rqf32::kThreads, 2)
     if (ncta > 1) cluster_sync_all();
 }
 
-// ===================================================================== fp32, g = 64, FFMA
-//
-// The same operation for g = 64 on row-major fp32 rows, with the rotation as an fp32 sum of
-// fused multiply-adds in i order (y = fma(x[63] R[63][c], ... fma(x[0] R[0][c], 0))), the
-// rotation "in fp32" of the pages computed as an fp32 matmul would be.  Blocks of RB whole
-// rows arrive by TMA in one 3-D box (64 channels, K / 64 groups, RB rows) into one of two
-// buffers, so the next block loads while this one is rotated.  R (16 KB) stays in shared
-// memory.  Each warp rotates tiles of 16 group-rows x 64 channels, lane l owning channels 2 l
-// and 2 l + 1: per four values of i it reads x[r][i .. i + 3] as one broadcast 16-byte load per
-// group-row and R[i .. i + 3][2 l, 2 l + 1] once, for 128 fused multiply-adds.  The rotated
-// values overwrite x in place (only the warp that reads a group-row writes it), the row maxima
-// meet in shared memory, and the codes are stored 16 at a time.
-namespace rqff {
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kTileGR = 16;                       // group-rows per warp tile
-constexpr int kMaxRB = 32;
-constexpr size_t kSmemPerCta = 110 * 1024;        // two CTAs per SM when the rows allow it
-constexpr size_t kSmemMax = 220 * 1024;
-}  // namespace rqff
-
-struct RqFfmaParams {
-    int64_t M, K, ldq, nblocks;
-    int RB;               // rows per block
-    int ngr;              // group-rows per block, RB K / 64
-    uint32_t box_bytes;   // RB K 4
-    int vec_codes, qmax;
-};
-
-__global__ void __launch_bounds__(rqff::kThreads, 2)
-    rq_f32_ffma64_kernel(const __grid_constant__ CUtensorMap xmap, const float* __restrict__ R,
-                         const float* __restrict__ scale_in, int8_t* __restrict__ codes,
-                         float* __restrict__ scales, RqFfmaParams p, int* dev_status) {
-    using namespace rqff;
-    extern __shared__ __align__(1024) unsigned char ff_smem[];
-    float* base = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(ff_smem) + 127) &
-                                           ~uintptr_t(127));
-    float* Rs = base;                                   // R[i][c], 64 x 64
-    float* const xbuf0 = base + 64 * 64;                // the two block buffers
-    float* const xbuf1 = xbuf0 + (size_t)p.RB * p.K;
-    __shared__ __align__(8) uint64_t full[2];
-    __shared__ unsigned int amax_sh[kMaxRB];
-    __shared__ float row_s[kMaxRB], row_r[kMaxRB];
-    __shared__ int abort_flag;
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int gpr = (int)(p.K / 64);                    // group-rows per row
-    // thread 0's count of the blocks it issued and of those it saw land (its drain after a
-    // timeout waits for the ones in between)
-    uint32_t issued = 0, landed = 0;
-    bool landing = true;
-    for (int i = tid; i < 64 * 64 / 4; i += kThreads)
-        reinterpret_cast<float4*>(Rs)[i] = __ldg(reinterpret_cast<const float4*>(R) + i);
-    if (tid < kMaxRB) amax_sh[tid] = 0u;
-    if (tid == 0) {
-        mbar_init(&full[0], 1);
-        mbar_init(&full[1], 1);
-        abort_flag = 0;
-        fence_mbar_init();
-        tma_prefetch_desc(&xmap);
-        // the first two blocks go out at once, one per buffer
-        for (int b = 0; b < 2; ++b) {
-            const int64_t blk = blockIdx.x + (int64_t)b * gridDim.x;
-            if (blk < p.nblocks) {
-                mbar_arrive_expect_tx(&full[b], p.box_bytes);
-                tma_load_3d(b ? xbuf1 : xbuf0, &xmap, &full[b], 0, 0, (int32_t)(blk * p.RB));
-                ++issued;
-            }
-        }
-    }
-    __syncthreads();
-
-    uint32_t it = 0;
-    for (int64_t blk = blockIdx.x; blk < p.nblocks; blk += gridDim.x, ++it) {
-        const int buf = (int)(it & 1u);
-        const uint32_t par = (it >> 1) & 1u;
-        float* xt = buf ? xbuf1 : xbuf0;
-        const int64_t m0 = blk * p.RB;
-        const bool skip = abort_flag != 0;   // read after the previous block's barriers
-        bool ok = !skip && __all_sync(0xffffffffu, mbar_wait(&full[buf], par, &abort_flag, dev_status));
-        if (tid == 0) {
-            landing = landing && ok;
-            if (landing) ++landed;
-        }
-        // ---------------------------------------------------------------- rotate in place
-        if (ok) {
-            const int ntiles = (p.ngr + kTileGR - 1) / kTileGR;
-            for (int t = warp; t < ntiles; t += kWarps) {
-                const int gr0 = t * kTileGR;
-                const int nr = (p.ngr - gr0) < kTileGR ? (p.ngr - gr0) : kTileGR;
-                float acc0[kTileGR], acc1[kTileGR];
-#pragma unroll
-                for (int r = 0; r < kTileGR; ++r) acc0[r] = acc1[r] = 0.f;
-                const float* xg = xt + (size_t)gr0 * 64;
-                // one step of four values of i for group-row r of the tile
-                auto step = [&](int r, int i, const float2 (&rq)[4]) {
-                    const float4 xv = *reinterpret_cast<const float4*>(xg + r * 64 + i);
-                    acc0[r] = __fmaf_rn(xv.x, rq[0].x, acc0[r]);
-                    acc1[r] = __fmaf_rn(xv.x, rq[0].y, acc1[r]);
-                    acc0[r] = __fmaf_rn(xv.y, rq[1].x, acc0[r]);
-                    acc1[r] = __fmaf_rn(xv.y, rq[1].y, acc1[r]);
-                    acc0[r] = __fmaf_rn(xv.z, rq[2].x, acc0[r]);
-                    acc1[r] = __fmaf_rn(xv.z, rq[2].y, acc1[r]);
-                    acc0[r] = __fmaf_rn(xv.w, rq[3].x, acc0[r]);
-                    acc1[r] = __fmaf_rn(xv.w, rq[3].y, acc1[r]);
-                };
-                if (nr == kTileGR) {   // a full tile: no predicates in the loop
-#pragma unroll 1
-                    for (int i = 0; i < 64; i += 4) {
-                        float2 rq[4];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            rq[q] = *reinterpret_cast<const float2*>(Rs + (i + q) * 64 + 2 * lane);
-#pragma unroll
-                        for (int r = 0; r < kTileGR; ++r) step(r, i, rq);
-                    }
-                } else {
-#pragma unroll 1
-                    for (int i = 0; i < 64; i += 4) {
-                        float2 rq[4];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            rq[q] = *reinterpret_cast<const float2*>(Rs + (i + q) * 64 + 2 * lane);
-#pragma unroll
-                        for (int r = 0; r < kTileGR; ++r)
-                            if (r < nr) step(r, i, rq);
-                    }
-                }
-                __syncwarp();   // every lane has read the tile's x before any lane overwrites it
-                // write y over x; fold |y| into the maximum of each group-row's row
-                float run = 0.f;
-                int run_row = -1;
-                // the row of group-row gr0 + r: one division per tile, then a count
-                int row_of = gr0 / gpr, left = gpr - (gr0 - row_of * gpr);
-#pragma unroll
-                for (int r = 0; r < kTileGR; ++r) {
-                    if (r < nr) {
-                        *reinterpret_cast<float2*>(xt + (size_t)(gr0 + r) * 64 + 2 * lane) =
-                            make_float2(acc0[r], acc1[r]);
-                        float mx = fmax_nan(fabsf(acc0[r]), fabsf(acc1[r]));
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1)
-                            mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                        if (left == 0) {
-                            ++row_of;
-                            left = gpr;
-                        }
-                        --left;
-                        const int row = row_of;
-                        if (row != run_row) {
-                            if (run_row >= 0 && lane == 0) atomicMax(&amax_sh[run_row], __float_as_uint(run));
-                            run_row = row;
-                            run = mx;
-                        } else {
-                            run = fmax_nan(run, mx);
-                        }
-                    }
-                }
-                if (run_row >= 0 && lane == 0) atomicMax(&amax_sh[run_row], __float_as_uint(run));
-            }
-        }
-        __syncthreads();
-        // ---------------------------------------------------------------- row scales
-        if (tid < p.RB) {
-            const float s = f32_row_scale(__uint_as_float(amax_sh[tid]), scale_in, p.qmax);
-            const RowDivisor dv(s, p.qmax);
-            row_s[tid] = s;
-            row_r[tid] = dv.r;
-            if (m0 + tid < p.M && ok) scales[m0 + tid] = s;
-            amax_sh[tid] = 0u;
-        }
-        __syncthreads();
-        // ---------------------------------------------------------------- quantize + store
-        if (ok) {
-            const int rows = (int)((p.M - m0) < p.RB ? (p.M - m0) : p.RB);
-            const int cpr = (int)(p.K / 16);   // 16-value chunks per row
-            for (int m = 0; m < rows; ++m)
-            for (int j = tid; j < cpr; j += kThreads) {
-                RowDivisor dv(row_s[m], p.qmax);
-                dv.r = row_r[m];
-                const float* src = xt + (size_t)m * p.K + 16 * j;
-                float y[16];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 v = *reinterpret_cast<const float4*>(src + 4 * q);
-                    y[4 * q] = v.x;
-                    y[4 * q + 1] = v.y;
-                    y[4 * q + 2] = v.z;
-                    y[4 * q + 3] = v.w;
-                }
-                uint32_t out[4];
-                quant16_any(y, dv, scale_in == nullptr, out);
-                int8_t* dst = codes + (m0 + m) * p.ldq + 16 * j;
-                if (p.vec_codes) {
-                    *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) dst[q] = (int8_t)((out[q / 4] >> (8 * (q % 4))) & 0xFF);
-                }
-            }
-        }
-        __syncthreads();   // the buffer is free: the block after next loads into it
-        if (tid == 0) {
-            const int64_t nxt = blk + 2 * (int64_t)gridDim.x;
-            if (abort_flag == 0 && nxt < p.nblocks) {
-                fence_proxy_async_smem();   // the threads' writes to the buffer precede the copy's
-                mbar_arrive_expect_tx(&full[buf], p.box_bytes);
-                tma_load_3d(xt, &xmap, &full[buf], 0, 0, (int32_t)(nxt * p.RB));
-                ++issued;
-            }
-        }
-    }
-    // after a timeout, copies still in flight land before the CTA leaves: the CTA's k-th block
-    // loads into buffer k % 2 on phase (k / 2) % 2
-    if (tid == 0)
-        for (uint32_t k = landed; k < issued; ++k) mbar_wait(&full[k & 1u], (k >> 1) & 1u, nullptr, nullptr);
-    __syncthreads();
-}
-
-// fp32, g = 64, unit K stride, 16-byte-aligned x and row pitch, K / 64 <= 256.  Returns
-// CK_ERR_UNSUPPORTED when the shape does not fit.
-ck_status launch_rq_f32_ffma64(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
-                               const void* R, const float* scale_in, int8_t* codes, int64_t ldq,
-                               float* scales, int qmax, int* dev_status, cudaStream_t stream) {
-    using namespace rqff;
-    if (sk != 1 || !aligned(x, 16) || !aligned(R, 16) || K % 64 != 0 || K / 64 > 256 ||
-        (M > 1 && (sm % 4 != 0 || sm < K)) || M >= (1LL << 31))
-        return CK_ERR_UNSUPPORTED;
-    const size_t r_bytes = 64 * 64 * 4 + 128;
-    const size_t row_bytes = (size_t)K * 4;
-    // rows per block: two CTAs per SM if a block of one row fits, the two buffers filled
-    size_t budget = kSmemPerCta;
-    if (r_bytes + 2 * row_bytes > budget) budget = kSmemMax;
-    int64_t rb = (int64_t)((budget - r_bytes) / (2 * row_bytes));
-    if (rb < 1) return CK_ERR_UNSUPPORTED;
-    if (rb > kMaxRB) rb = kMaxRB;
-    // few rows: blocks small enough that every SM gets work
-    const int64_t spread = (M + 2LL * num_sms() - 1) / (2LL * num_sms());
-    if (rb > spread) rb = spread < 1 ? 1 : spread;
-    if (rb > M) rb = M;
-    RqFfmaParams p;
-    p.M = M;
-    p.K = K;
-    p.ldq = ldq;
-    p.RB = (int)rb;
-    p.ngr = (int)(rb * (K / 64));
-    p.nblocks = (M + rb - 1) / rb;
-    p.box_bytes = (uint32_t)(rb * row_bytes);
-    p.vec_codes = (aligned(codes, 16) && ldq % 16 == 0) ? 1 : 0;
-    p.qmax = qmax;
-
-    CUtensorMap map;
-    const uint64_t dims[3] = {64, (uint64_t)(K / 64), (uint64_t)M};
-    const uint64_t strides[2] = {256, (uint64_t)(M > 1 ? sm : K) * 4};
-    const uint32_t box[3] = {64, (uint32_t)(K / 64), (uint32_t)rb};
-    const ck_status st = encode_tma(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, x, dims, strides,
-                                    box, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (st != CK_OK) return st;
-    const size_t smem = r_bytes + 2 * (size_t)p.box_bytes;
-    if (cudaFuncSetAttribute(rq_f32_ffma64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-        return CK_ERR_CUDA;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rq_f32_ffma64_kernel, kThreads,
-                                                      smem) != cudaSuccess || per_sm < 1)
-        return CK_ERR_UNSUPPORTED;
-    const int64_t cap = (int64_t)per_sm * num_sms();
-    const int grid = (int)(p.nblocks < cap ? p.nblocks : cap);
-    rq_f32_ffma64_kernel<<<grid, kThreads, smem, stream>>>(map, static_cast<const float*>(R),
-                                                           scale_in, codes, scales, p, dev_status);
-    return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
-}
-
 // ===================================================================== fp32, g = 256, FFMA
 //
 // g = 256 on row-major fp32 rows: R (256 KB) does not fit in shared memory, so it passes
@@ -676,6 +403,14 @@ ck_status launch_rq_f32_ffma64(const void* x, int64_t M, int64_t K, int64_t sm, 
 // Blocks of whole rows arrive by TMA (one 3-D box of 256 channels x K / 256 groups x RB rows)
 // into one of two buffers.  A work unit is 8 group-rows x 64 channels (lane l: channels
 // 64 cb + 2 l, + 1); the last pass folds |y| into the row maxima; then the codes.
+struct RqFfmaParams {
+    int64_t M, K, ldq, nblocks;
+    int RB;               // rows per block
+    int ngr;              // group-rows per block, RB K / 256
+    uint32_t box_bytes;   // RB K 4
+    int vec_codes, qmax;
+};
+
 namespace rqff256 {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;

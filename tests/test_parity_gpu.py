@@ -179,13 +179,13 @@ def test_rotate_quant_long_rows(dt, g, K):
                    x=x, R=R)
 
 
-@pytest.mark.parametrize("M,groups,pitch", [(700, 5, 0), (33, 1, 0), (5, 255, 0), (3, 256, 0),
+@pytest.mark.parametrize("M,groups,pitch", [(710, 5, 0), (33, 1, 0), (5, 255, 0), (3, 256, 0),
                                             (1300, 60, 64), (9, 160, 0)])
 def test_rotate_quant_f32_g64_blocks(M, groups, pitch):
-    """fp32 rows at g = 64 (the FFMA kernel): blocks of whole rows with a ragged last block
-    (700 rows of 5 groups in blocks of 3), one-group rows, the longest rows one box holds (255
-    and 256 groups), a row pitch past K, and rows of 60 and 160 groups whose warp tiles of 16
-    group-rows straddle rows (1300 rows of 60 groups in blocks of 3).  R is a non-symmetric
+    """fp32 rows at g = 64 (split TF32 on tensor cores): tiles of whole rows with a ragged last
+    tile (710 rows of 5 groups in tiles of 25; 33 one-group rows in one tile of 128), rows of
+    60 groups two to a tile with a row pitch past K, and rows split in two parts (160 groups;
+    255 and 256, the longest, one part with a group past the row).  R is a non-symmetric
     orthogonal matrix.  Every output is compared."""
     g, K = 64, 64 * groups
     case = W.RotateCase(f"f32_g64_{M}_{groups}", M=M, K=K, g=g, dtype="f32", seed=M + groups)

@@ -56,10 +56,14 @@ def _healthy():
 
 @pytest.mark.parametrize("what,dt,g,M,K,layout", [
     ("tensor-core stage 1", torch.bfloat16, 64, 512, 3840, "row"),
-    ("warp-per-row stage 1", torch.bfloat16, 16, 512, 3840, "row"),
+    ("tensor-core stage 1, split rows", torch.bfloat16, 64, 64, 10240, "row"),
+    ("warp-per-row stage 1", torch.bfloat16, 16, 512, 3856, "row"),
     ("block-ring stage 1", torch.float16, 16, 64, 32768, "row"),
     ("fp32 stage 1, row-major", torch.float32, 16, 512, 3840, "row"),
-    ("fp32 stage 1, column-major cluster", torch.float32, 16, 512, 3840, "col")])
+    ("fp32 stage 1, column-major cluster", torch.float32, 16, 512, 3840, "col"),
+    ("fp32 split-TF32 stage 1", torch.float32, 64, 512, 3840, "row"),
+    ("fp32 split-TF32 stage 1, split rows", torch.float32, 64, 64, 10240, "row"),
+    ("fp32 g = 256 FFMA stage 1", torch.float32, 256, 64, 3840, "row")])
 def test_stage1_wait_expiry_returns_a_status(L, what, dt, g, M, K, layout):
     x = torch.randn(M, K).to(dt)
     if layout == "col":
