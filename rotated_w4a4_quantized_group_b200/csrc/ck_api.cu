@@ -255,11 +255,13 @@ static ck_status linear_impl(const void* x, ck_dtype x_dtype, int64_t M, int64_t
         wp = dst;
         wld = wp_pitch;
     }
+    // the GEMM overlaps stage 1's tail when stage 1 is the kernel right before it
+    const bool after_stage1 = !codes_in && w_aligned;
     if (w8)
         return launch_w8a8_gemm(codes, ldq, row_scale, M, K, wp, wld, N, w_scale, scale_dtype,
-                                bias, segs, out_dtype, dev_status, stream);
+                                bias, segs, out_dtype, after_stage1, dev_status, stream);
     return launch_w4a4_gemm(codes, ldq, row_scale, M, K, wp, wld, N, w_scale, scale_dtype, bias,
-                            segs, out_dtype, dev_status, stream);
+                            segs, out_dtype, after_stage1, dev_status, stream);
 }
 
 }  // namespace ck

@@ -119,6 +119,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// ------------------------------------------------------------------ dependent launches
+
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization may
+// start while the kernel before it in the stream still runs (once every CTA of that kernel has
+// called grid_dependents_launch() or exited); its grid_dependency_wait() returns when that
+// kernel has completed and its memory writes are visible.  Without the launch attribute the
+// wait returns at once and the trigger does nothing.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependents_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ warps
 
 // True in exactly one lane of the (fully converged) warp, false in the others.

@@ -60,28 +60,32 @@ ck_status launch_rq_f32_g16(const void* x, int64_t M, int64_t K, int64_t sm, int
                             float* scales, int qmax, int* dev_status, cudaStream_t stream);
 
 // Stage 2 launch: codes (M, K) int8 with 16-byte-aligned rows (ldq % 16 == 0), packed
-// weights with 16-byte-aligned rows (w_ld % 16 == 0).
+// weights with 16-byte-aligned rows (w_ld % 16 == 0).  after_stage1: the kernel just before
+// this one on the stream is the stage-1 launch that writes the codes and row scales (and
+// nothing this GEMM reads besides them); the GEMM is then launched as its programmatic
+// dependent, so it may start (set up, load and expand its weights) while stage 1 finishes,
+// and reads the codes and scales only after stage 1 has completed.
 ck_status launch_w4a4_gemm(const int8_t* codes, int64_t ldq, const float* a_scale, int64_t M,
                            int64_t K, const int8_t* w_packed, int64_t w_ld, int64_t N,
                            const void* w_scale, ck_dtype scale_dt, const void* bias,
-                           const OutSegs& segs, ck_dtype out_dt, int* dev_status,
-                           cudaStream_t stream);
+                           const OutSegs& segs, ck_dtype out_dt, bool after_stage1,
+                           int* dev_status, cudaStream_t stream);
 
 // The W8A8 variant's stage 2: INT8 weights (N, K) with 16-byte-aligned rows (w_ld % 16 == 0),
 // the same codes, epilogue and outputs as launch_w4a4_gemm.
 ck_status launch_w8a8_gemm(const int8_t* codes, int64_t ldq, const float* a_scale, int64_t M,
                            int64_t K, const int8_t* w, int64_t w_ld, int64_t N,
                            const void* w_scale, ck_dtype scale_dt, const void* bias,
-                           const OutSegs& segs, ck_dtype out_dt, int* dev_status,
-                           cudaStream_t stream);
+                           const OutSegs& segs, ck_dtype out_dt, bool after_stage1,
+                           int* dev_status, cudaStream_t stream);
 
 // Stage 2 for M <= 64 with K split over a thread-block cluster (ck_w4a4_splitk.cu); same
 // arguments as launch_w4a4_gemm.  Returns CK_ERR_UNSUPPORTED for shapes it does not take.
 ck_status launch_w4a4_splitk(const int8_t* codes, int64_t ldq, const float* a_scale, int64_t M,
                              int64_t K, const int8_t* w_packed, int64_t w_ld, int64_t N,
                              const void* w_scale, ck_dtype scale_dt, const void* bias,
-                             const OutSegs& segs, ck_dtype out_dt, int* dev_status,
-                             cudaStream_t stream);
+                             const OutSegs& segs, ck_dtype out_dt, bool after_stage1,
+                             int* dev_status, cudaStream_t stream);
 
 ck_status launch_unpack_w4(const int8_t* packed, int64_t N, int64_t K, int64_t ld_packed,
                            int8_t* out, int64_t ld_out, cudaStream_t stream);

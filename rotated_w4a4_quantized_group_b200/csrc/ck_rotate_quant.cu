@@ -115,6 +115,8 @@ __global__ void __launch_bounds__(kGenThreads)
                       const T* __restrict__ R, int g, int r_in_smem,
                       const float* __restrict__ scale_in, int8_t* __restrict__ codes, int64_t ldq,
                       float* __restrict__ scales, int vec_codes, int qmax) {
+    // the linear's GEMM, launched as this kernel's dependent, may start its prologue now
+    grid_dependents_launch();
     extern __shared__ __align__(16) unsigned char gen_smem[];
     float* xs = reinterpret_cast<float*>(gen_smem);
     T* Rs = reinterpret_cast<T*>(xs + K);
@@ -303,6 +305,8 @@ __global__ void __launch_bounds__(kRqThreads, 1)
     rq_mma_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ R,
                   const float* __restrict__ scale_in, int8_t* __restrict__ codes,
                   float* __restrict__ scales, RqMmaParams p, int* dev_status) {
+    // the linear's GEMM, launched as this kernel's dependent, may start its prologue now
+    grid_dependents_launch();
     constexpr int KT = G / 16;   // k-tiles of the m16n8k16 MMA
     constexpr int NT = G / 8;    // n-tiles
     extern __shared__ __align__(1024) unsigned char mma_smem[];
@@ -531,6 +535,8 @@ __global__ void __launch_bounds__(kRowMaxWarps * 32, 1)
     rq_row_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ R,
                   const float* __restrict__ scale_in, int8_t* __restrict__ codes,
                   float* __restrict__ scales, RqRowParams p, int* dev_status) {
+    // the linear's GEMM, launched as this kernel's dependent, may start its prologue now
+    grid_dependents_launch();
     constexpr int KT = G / 16;   // k-tiles of the m16n8k16 MMA (input channels)
     constexpr int MT = G / 16;   // m-tiles (output channels)
     extern __shared__ __align__(1024) unsigned char row_smem[];
@@ -961,6 +967,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_sh;
+    // the linear's GEMM, launched as this kernel's dependent, may start its prologue now:
+    // after every CTA holds its tensor memory, so a GEMM CTA that lands on the same SM
+    // and waits for its columns never stands in the way of a CTA of this kernel
+    grid_dependents_launch();
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer

@@ -103,6 +103,8 @@ __global__ void __launch_bounds__(rqf32::kThreads, 2)
     rq_f32_g16_kernel(const __grid_constant__ CUtensorMap xmap, const float* __restrict__ R,
                       const float* __restrict__ scale_in, int8_t* __restrict__ codes,
                       float* __restrict__ scales, RqF32Params p, int* dev_status) {
+    // the linear's GEMM, launched as this kernel's dependent, may start its prologue now
+    grid_dependents_launch();
     using namespace rqf32;
     extern __shared__ __align__(1024) unsigned char f32_smem[];
     float* tile = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(f32_smem) + 1023) &
@@ -424,6 +426,8 @@ __global__ void __launch_bounds__(rqff256::kThreads, 1)
     rq_f32_ffma256_kernel(const __grid_constant__ CUtensorMap xmap, const float* __restrict__ R,
                           const float* __restrict__ scale_in, int8_t* __restrict__ codes,
                           float* __restrict__ scales, RqFfmaParams p, int* dev_status) {
+    // the linear's GEMM, launched as this kernel's dependent, may start its prologue now
+    grid_dependents_launch();
     using namespace rqff256;
     extern __shared__ __align__(1024) unsigned char f256_smem[];
     float* base = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(f256_smem) + 127) &

@@ -169,6 +169,10 @@ __global__ void __launch_bounds__(rqtf::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_sh;
+    // the linear's GEMM, launched as this kernel's dependent, may start its prologue now:
+    // after every CTA holds its tensor memory, so a GEMM CTA that lands on the same SM
+    // and waits for its columns never stands in the way of a CTA of this kernel
+    grid_dependents_launch();
 
     if (warp == kWarpTma) {
         // ---------------------------------------------------------------- TMA producer

@@ -181,6 +181,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         // warp WARP_TMA_X brings the even k-blocks of each super-stage, warp WARP_TMA_X2 the
         // odd ones: one box per issuing thread and k-block, so two boxes load at once
         if (lane == 0) {
+            grid_dependency_wait();   // the codes may be the output of the kernel before this one
             const uint32_t par = warp == WARP_TMA_X2 ? 1u : 0u;
             uint32_t issued = 0, slot = 0;
             bool ok = true;
@@ -250,6 +251,10 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
             bool ok = true;
             for (uint32_t ss = 0; ok && ss < my_ss; ++ss) {
                 const uint32_t set = ss & 1u;
+                // this wait needs the unpack warps' pass over super-stage ss - 2, which follows
+                // their pass over ss - 4, which waited for the MMAs of ss - 4 - NB: MMAs that
+                // need the codes, from the kernel before this one
+                if (ss == NB + 2 * UNP_SETS) grid_dependency_wait();
                 if (ss >= UNP_SETS &&
                     !mbar_wait(&w_empty[set], ((ss >> 1) - 1) & 1u, &abort_flag, p.dev_status)) {
                     ok = false;
@@ -280,6 +285,9 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         // The whole warp walks the ring and takes every wait (a vote makes each decision
         // uniform), so every value an MMA takes is computed uniformly across the warp; one lane,
         // elected once, issues all MMAs and commits (a commit tracks its own thread's MMAs).
+        // Its waits start once the kernel before this one (stage 1) has completed, so none of
+        // their time limits covers the rest of that kernel.
+        grid_dependency_wait();
         const bool leader = elect_one();
         // descriptor of code k-block 0 of slot 0; k-block j of slot s starts
         // (s G + j) x_bytes later (start-address field counts 16-byte units)
@@ -395,6 +403,8 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                 }
             }
             // the buffer is free once the MMAs of its previous super-stage (ss - NB) completed
+            // (MMAs that need the codes: the wait starts after the kernel before this one)
+            if (ss >= NB && ss < NB + UNP_SETS) grid_dependency_wait();   // once
             if (ss >= NB && !__all_sync(0xffffffffu, wait_done(ss - NB))) break;
             tc_fence_after();
 #pragma unroll
@@ -412,6 +422,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         // ---------------------------------------------------------------- epilogue
         const int q = warp & 3;                        // TMEM lanes 32q .. 32q + 31
         const int eh = warp >= EPI_WARP1 ? 1 : 0;      // rows 32k + 16 eh .. + 15 of each 32
+        grid_dependency_wait();   // so may the row scales
         uint32_t lt = 0;
         for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++lt) {
             const uint32_t acc = lt & 1u;
@@ -500,26 +511,39 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
 template <typename OutT, typename ScaleT>
 static ck_status launch_typed(const CUtensorMap& xmap, const CUtensorMap& wmap,
                               const GemmParams& p, size_t smem, int grid, bool x16, bool w8,
-                              cudaStream_t stream) {
+                              bool dependent, cudaStream_t stream) {
     auto kern = w8 ? w4a4_gemm_kernel<OutT, ScaleT, false, true>
                    : x16 ? w4a4_gemm_kernel<OutT, ScaleT, true, false>
                          : w4a4_gemm_kernel<OutT, ScaleT, false, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return CK_ERR_CUDA;
-    kern<<<grid, gemm::THREADS, smem, stream>>>(xmap, wmap, p);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(gemm::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = dependent ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kern, xmap, wmap, p) != cudaSuccess) return CK_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 
 template <typename OutT>
 static ck_status launch_out(const CUtensorMap& xmap, const CUtensorMap& wmap, const GemmParams& p,
-                            size_t smem, int grid, bool x16, bool w8, ck_dtype scale_dt,
+                            size_t smem, int grid, bool x16, bool w8, bool dep, ck_dtype scale_dt,
                             cudaStream_t stream) {
     switch (scale_dt) {
-        case CK_F32: return launch_typed<OutT, float>(xmap, wmap, p, smem, grid, x16, w8, stream);
-        case CK_F16: return launch_typed<OutT, __half>(xmap, wmap, p, smem, grid, x16, w8, stream);
+        case CK_F32:
+            return launch_typed<OutT, float>(xmap, wmap, p, smem, grid, x16, w8, dep, stream);
+        case CK_F16:
+            return launch_typed<OutT, __half>(xmap, wmap, p, smem, grid, x16, w8, dep, stream);
         case CK_BF16:
-            return launch_typed<OutT, __nv_bfloat16>(xmap, wmap, p, smem, grid, x16, w8, stream);
+            return launch_typed<OutT, __nv_bfloat16>(xmap, wmap, p, smem, grid, x16, w8, dep,
+                                                     stream);
         default: return CK_ERR_INVALID_ARG;
     }
 }
@@ -548,8 +572,8 @@ static int choose_bna(int64_t M, int64_t N, int sms) {
 static ck_status launch_persistent(const int8_t* codes, int64_t ldq, const float* a_scale,
                                    int64_t M, int64_t K, const int8_t* w, int64_t w_ld, int64_t N,
                                    const void* w_scale, ck_dtype scale_dt, const void* bias,
-                                   const OutSegs& segs, ck_dtype out_dt, bool w8, int* dev_status,
-                                   cudaStream_t stream) {
+                                   const OutSegs& segs, ck_dtype out_dt, bool w8, bool dep,
+                                   int* dev_status, cudaStream_t stream) {
     using namespace gemm;
     const int sms = num_sms();
     GemmParams p;
@@ -627,10 +651,13 @@ static ck_status launch_persistent(const int8_t* codes, int64_t ldq, const float
     const int grid = (int)(p.tiles < sms ? p.tiles : sms);
     const bool x16 = !w8 && K <= SCALED16_MAX_K;
     switch (out_dt) {
-        case CK_F32: return launch_out<float>(xmap, wmap, p, smem, grid, x16, w8, scale_dt, stream);
-        case CK_F16: return launch_out<__half>(xmap, wmap, p, smem, grid, x16, w8, scale_dt, stream);
+        case CK_F32:
+            return launch_out<float>(xmap, wmap, p, smem, grid, x16, w8, dep, scale_dt, stream);
+        case CK_F16:
+            return launch_out<__half>(xmap, wmap, p, smem, grid, x16, w8, dep, scale_dt, stream);
         case CK_BF16:
-            return launch_out<__nv_bfloat16>(xmap, wmap, p, smem, grid, x16, w8, scale_dt, stream);
+            return launch_out<__nv_bfloat16>(xmap, wmap, p, smem, grid, x16, w8, dep, scale_dt,
+                                             stream);
         default: return CK_ERR_INVALID_ARG;
     }
 }
@@ -638,27 +665,27 @@ static ck_status launch_persistent(const int8_t* codes, int64_t ldq, const float
 ck_status launch_w4a4_gemm(const int8_t* codes, int64_t ldq, const float* a_scale, int64_t M,
                            int64_t K, const int8_t* w_packed, int64_t w_ld, int64_t N,
                            const void* w_scale, ck_dtype scale_dt, const void* bias,
-                           const OutSegs& segs, ck_dtype out_dt, int* dev_status,
-                           cudaStream_t stream) {
+                           const OutSegs& segs, ck_dtype out_dt, bool after_stage1,
+                           int* dev_status, cudaStream_t stream) {
     if (M == 0 || N == 0) return CK_OK;
     if (M <= 64) {   // few rows: split K over clusters so the weights stream on every SM
         const ck_status st = launch_w4a4_splitk(codes, ldq, a_scale, M, K, w_packed, w_ld, N,
                                                 w_scale, scale_dt, bias, segs, out_dt,
-                                                dev_status, stream);
+                                                after_stage1, dev_status, stream);
         if (st != CK_ERR_UNSUPPORTED) return st;
     }
     return launch_persistent(codes, ldq, a_scale, M, K, w_packed, w_ld, N, w_scale, scale_dt,
-                             bias, segs, out_dt, false, dev_status, stream);
+                             bias, segs, out_dt, false, after_stage1, dev_status, stream);
 }
 
 ck_status launch_w8a8_gemm(const int8_t* codes, int64_t ldq, const float* a_scale, int64_t M,
                            int64_t K, const int8_t* w, int64_t w_ld, int64_t N,
                            const void* w_scale, ck_dtype scale_dt, const void* bias,
-                           const OutSegs& segs, ck_dtype out_dt, int* dev_status,
-                           cudaStream_t stream) {
+                           const OutSegs& segs, ck_dtype out_dt, bool after_stage1,
+                           int* dev_status, cudaStream_t stream) {
     if (M == 0 || N == 0) return CK_OK;
     return launch_persistent(codes, ldq, a_scale, M, K, w, w_ld, N, w_scale, scale_dt, bias, segs,
-                             out_dt, true, dev_status, stream);
+                             out_dt, true, after_stage1, dev_status, stream);
 }
 
 }  // namespace ck

@@ -14,7 +14,9 @@
 //   warps 0, 2  issue TMA copies of the CTA's whole K range at once, one box per lane: packed
 //               weights (warp 0; 128 rows x 64 bytes per k-block, 64-byte swizzle) and codes
 //               (warp 2; BNA rows x 128 bytes, 128-byte swizzle), two k-blocks per box, one
-//               mbarrier per box pair;
+//               mbarrier per box; the codes only once the kernel before this one (stage 1,
+//               of which this kernel is the programmatic dependent) has completed, so the
+//               weights stream in and are expanded while stage 1 still runs;
 //   warps 4-7   expand the weight nibbles (one weight row per thread) into tensor memory in
 //               chunks of up to six k-blocks, the MMA's A operand, then read the accumulator;
 //   warp 1      allocates tensor memory and issues tcgen05.mma kind::i8 (128 x BNA x 32, A from
@@ -79,7 +81,9 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
     unsigned char* xbuf = wbuf + (size_t)kb_slots * W_BYTES;
     int32_t* partial = reinterpret_cast<int32_t*>(xbuf + (size_t)kb_slots * p.x_bytes);  // [BNA][128]
 
-    __shared__ __align__(8) uint64_t ld_full[KB_MAX / 2], a_full, chunk_done, acc_full, drain_bar;
+    // w_full[i] / x_full[i]: the weights / codes of k-block pair i have landed
+    __shared__ __align__(8) uint64_t w_full[KB_MAX / 2], x_full[KB_MAX / 2], a_full, chunk_done,
+        acc_full, drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
 
@@ -92,7 +96,10 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
     const int n0 = (int)blockIdx.y * BW;
 
     if (tid == 0) {
-        for (int i = 0; i < KB_MAX / 2; ++i) mbar_init(&ld_full[i], 1);
+        for (int i = 0; i < KB_MAX / 2; ++i) {
+            mbar_init(&w_full[i], 1);
+            mbar_init(&x_full[i], 1);
+        }
         mbar_init(&a_full, 4);
         mbar_init(&chunk_done, 1);
         mbar_init(&acc_full, 1);
@@ -113,31 +120,29 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
 
     if (warp == WARP_TMA || warp == WARP_TMA2) {
         // ---------------------------------------------------------------- TMA: the whole range
-        // lane i of warp WARP_TMA brings pair i's weights, lane i of warp WARP_TMA2 its codes:
-        // one box per issuing thread, so the copies do not queue behind one another.  The pair's
-        // byte count is registered on its barrier before either warp issues (named barrier).
-        if (warp == WARP_TMA) {
-            for (int i = lane; i < npairs; i += 32) {
-                const uint32_t nk = p.box3d ? 2u : (uint32_t)((n_kb - 2 * i) < 2 ? (n_kb - 2 * i) : 2);
-                mbar_arrive_expect_tx(&ld_full[i], nk * (W_BYTES + p.x_bytes));
-            }
-        }
-        asm volatile("bar.sync 1, 64;" ::: "memory");
+        // lane i of warp WARP_TMA brings pair i's weights, lane i of warp WARP_TMA2 its codes,
+        // each on its own barrier: one box per issuing thread, so the copies do not queue
+        // behind one another.  The codes may be the output of the kernel before this one (its
+        // programmatic dependent launch lets the weights stream and expand meanwhile).
+        uint64_t* bar = warp == WARP_TMA ? w_full : x_full;
+        const uint32_t bytes = warp == WARP_TMA ? W_BYTES : p.x_bytes;
+        if (warp == WARP_TMA2) grid_dependency_wait();
         for (int i = lane; i < npairs; i += 32) {
             const int kb = kb_lo + 2 * i;
             const uint32_t nk = p.box3d ? 2u : (uint32_t)((n_kb - 2 * i) < 2 ? (n_kb - 2 * i) : 2);
+            mbar_arrive_expect_tx(&bar[i], nk * bytes);
             if (p.box3d) {
                 if (warp == WARP_TMA)
-                    tma_load_3d(wbuf + (size_t)(2 * i) * W_BYTES, &wmap, &ld_full[i], 0, n0, kb);
+                    tma_load_3d(wbuf + (size_t)(2 * i) * W_BYTES, &wmap, &bar[i], 0, n0, kb);
                 else
-                    tma_load_3d(xbuf + (size_t)(2 * i) * p.x_bytes, &xmap, &ld_full[i], 0, 0, kb);
+                    tma_load_3d(xbuf + (size_t)(2 * i) * p.x_bytes, &xmap, &bar[i], 0, 0, kb);
             } else {
                 for (uint32_t j = 0; j < nk; ++j) {
                     if (warp == WARP_TMA)
-                        tma_load_2d(wbuf + (size_t)(2 * i + j) * W_BYTES, &wmap, &ld_full[i],
+                        tma_load_2d(wbuf + (size_t)(2 * i + j) * W_BYTES, &wmap, &bar[i],
                                     (kb + (int)j) * (BK / 2), n0);
                     else
-                        tma_load_2d(xbuf + (size_t)(2 * i + j) * p.x_bytes, &xmap, &ld_full[i],
+                        tma_load_2d(xbuf + (size_t)(2 * i + j) * p.x_bytes, &xmap, &bar[i],
                                     (kb + (int)j) * BK, 0);
                 }
             }
@@ -145,7 +150,9 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
     } else if (warp == WARP_MMA) {
         // ---------------------------------------------------------------- MMA issuer
         // the warp walks the chunks together (votes make each wait's outcome uniform, so the
-        // MMA operands are computed uniformly); one elected lane issues every MMA and commit
+        // MMA operands are computed uniformly); one elected lane issues every MMA and commit.
+        // Its waits start once the kernel before this one has completed.
+        grid_dependency_wait();
         const bool leader = elect_one();
         const uint64_t bdesc0 = smem_desc_k_sw128(smem_u32(xbuf));
         const uint32_t kstep = p.x_bytes >> 4;
@@ -157,9 +164,9 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
             }
             const int kb0 = c * CHUNK_KB;
             const int nc = (n_kb - kb0) < CHUNK_KB ? (n_kb - kb0) : CHUNK_KB;
-            // the codes of the chunk landed (the expansion waited for the same barriers)
+            // the codes of the chunk landed
             for (int i = kb0 / 2; i <= (kb0 + nc - 1) / 2; ++i)
-                if (!__all_sync(0xffffffffu, mbar_wait(&ld_full[i], 0, &abort_flag, p.dev_status))) ok = false;
+                if (!__all_sync(0xffffffffu, mbar_wait(&x_full[i], 0, &abort_flag, p.dev_status))) ok = false;
             if (!ok) break;
             tc_fence_after();
             if (leader) {
@@ -193,6 +200,7 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
         bool ok = true;
         for (int c = 0; ok && c < nchunks; ++c) {
             if (c > 0) {   // the chunk's tensor memory is free once the previous chunk's MMAs ended
+                grid_dependency_wait();   // MMAs that need the codes
                 if (!__all_sync(0xffffffffu, mbar_wait(&chunk_done, (uint32_t)(c - 1) & 1u,
                                                        &abort_flag, p.dev_status))) {
                     ok = false;
@@ -204,7 +212,7 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
             const int nc = (n_kb - kb0) < CHUNK_KB ? (n_kb - kb0) : CHUNK_KB;
             for (int j = 0; j < nc; ++j) {
                 const int kb = kb0 + j;
-                if (!__all_sync(0xffffffffu, mbar_wait(&ld_full[kb >> 1], 0, &abort_flag,
+                if (!__all_sync(0xffffffffu, mbar_wait(&w_full[kb >> 1], 0, &abort_flag,
                                                        p.dev_status))) {
                     ok = false;
                     break;
@@ -248,6 +256,7 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
     // ---------------------------------------------------------------- cluster reduction
     __syncthreads();
     if (ncta > 1) cluster_sync_all();
+    grid_dependency_wait();   // the row scales, as the codes
     if (!abort_flag) {
         // this CTA's share of the tile's 4-channel vectors: [lo, hi) of BNA * 32
         const int nvec = p.BNA * (BW / 4);
@@ -284,7 +293,10 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
     // own still landing (after a timeout the copies were never waited for)
     if (ncta > 1) cluster_sync_all();
     if (warp == WARP_TMA && lane == 0 && abort_flag)
-        for (int i = 0; i < npairs; ++i) mbar_wait(&ld_full[i], 0, nullptr, nullptr);
+        for (int i = 0; i < npairs; ++i) {
+            mbar_wait(&w_full[i], 0, nullptr, nullptr);
+            mbar_wait(&x_full[i], 0, nullptr, nullptr);
+        }
     __syncthreads();
     if (warp == WARP_MMA) {
         tc_fence_after();
@@ -295,17 +307,19 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
 template <typename OutT, typename ScaleT>
 static ck_status splitk_launch_typed(const CUtensorMap& xmap, const CUtensorMap& wmap,
                                      const SplitKParams& p, int S, int tiles_n, size_t smem,
-                                     bool x16, cudaStream_t stream) {
+                                     bool x16, bool dep, cudaStream_t stream) {
     auto kern = x16 ? w4a4_splitk_kernel<OutT, ScaleT, true> : w4a4_splitk_kernel<OutT, ScaleT, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return CK_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)S;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3((unsigned)S, (unsigned)tiles_n, 1);
     cfg.blockDim = dim3(splitk::THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
@@ -315,6 +329,7 @@ static ck_status splitk_launch_typed(const CUtensorMap& xmap, const CUtensorMap&
     int max_clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess || max_clusters < 1)
         return CK_ERR_UNSUPPORTED;
+    cfg.numAttrs = dep ? 2 : 1;
     if (cudaLaunchKernelEx(&cfg, kern, xmap, wmap, p) != cudaSuccess) return CK_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
@@ -322,15 +337,17 @@ static ck_status splitk_launch_typed(const CUtensorMap& xmap, const CUtensorMap&
 template <typename OutT>
 static ck_status splitk_launch_out(const CUtensorMap& xmap, const CUtensorMap& wmap,
                                    const SplitKParams& p, int S, int tiles_n, size_t smem,
-                                   bool x16, ck_dtype scale_dt, cudaStream_t stream) {
+                                   bool x16, bool dep, ck_dtype scale_dt, cudaStream_t stream) {
     switch (scale_dt) {
         case CK_F32:
-            return splitk_launch_typed<OutT, float>(xmap, wmap, p, S, tiles_n, smem, x16, stream);
+            return splitk_launch_typed<OutT, float>(xmap, wmap, p, S, tiles_n, smem, x16, dep,
+                                                    stream);
         case CK_F16:
-            return splitk_launch_typed<OutT, __half>(xmap, wmap, p, S, tiles_n, smem, x16, stream);
+            return splitk_launch_typed<OutT, __half>(xmap, wmap, p, S, tiles_n, smem, x16, dep,
+                                                     stream);
         case CK_BF16:
             return splitk_launch_typed<OutT, __nv_bfloat16>(xmap, wmap, p, S, tiles_n, smem, x16,
-                                                            stream);
+                                                            dep, stream);
         default: return CK_ERR_INVALID_ARG;
     }
 }
@@ -338,8 +355,8 @@ static ck_status splitk_launch_out(const CUtensorMap& xmap, const CUtensorMap& w
 ck_status launch_w4a4_splitk(const int8_t* codes, int64_t ldq, const float* a_scale, int64_t M,
                              int64_t K, const int8_t* w_packed, int64_t w_ld, int64_t N,
                              const void* w_scale, ck_dtype scale_dt, const void* bias,
-                             const OutSegs& segs, ck_dtype out_dt, int* dev_status,
-                             cudaStream_t stream) {
+                             const OutSegs& segs, ck_dtype out_dt, bool after_stage1,
+                             int* dev_status, cudaStream_t stream) {
     using namespace splitk;
     if (M < 1 || M > MAX_M || N < 1) return CK_ERR_UNSUPPORTED;
     const int sms = num_sms();
@@ -408,12 +425,14 @@ ck_status launch_w4a4_splitk(const int8_t* codes, int64_t ldq, const float* a_sc
     const bool x16 = K <= (1LL << 21) - 1;
     switch (out_dt) {
         case CK_F32:
-            return splitk_launch_out<float>(xmap, wmap, p, S, (int)tiles_n, smem, x16, scale_dt, stream);
+            return splitk_launch_out<float>(xmap, wmap, p, S, (int)tiles_n, smem, x16,
+                                            after_stage1, scale_dt, stream);
         case CK_F16:
-            return splitk_launch_out<__half>(xmap, wmap, p, S, (int)tiles_n, smem, x16, scale_dt, stream);
+            return splitk_launch_out<__half>(xmap, wmap, p, S, (int)tiles_n, smem, x16,
+                                             after_stage1, scale_dt, stream);
         case CK_BF16:
             return splitk_launch_out<__nv_bfloat16>(xmap, wmap, p, S, (int)tiles_n, smem, x16,
-                                                    scale_dt, stream);
+                                                    after_stage1, scale_dt, stream);
         default: return CK_ERR_INVALID_ARG;
     }
 }

@@ -127,6 +127,26 @@ def test_sets_for_cover_three_l2s():
     assert bench.sets_for(1, 64) == 64
 
 
+def test_step_schedule_runs_exactly_the_asked_steps():
+    """The timed replays run exactly K steps: full graphs of S steps, then one graph of the
+    first K mod S steps."""
+    import bench
+    built = []
+
+    def partial(r):
+        built.append(r)
+        return ("first", r)
+
+    for S in (1, 3, 7, 51):
+        for n in (1, 2, 3, 5, 10, 50, 200):
+            built.clear()
+            sched = bench.step_schedule(("full", S), S, partial, n)
+            steps = sum(S if g[0] == "full" else g[1] for g in sched)
+            assert steps == n
+            assert built == ([n % S] if n % S else [])
+            assert all(g == ("full", S) for g in sched[: n // S])
+
+
 def test_kernel_sources_follow_the_workload():
     import os
     import bench

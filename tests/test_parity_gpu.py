@@ -580,6 +580,27 @@ def test_rotate_quant_f32_g16_equals_the_oracle_bit_for_bit(layout, M, K, pad):
     np.testing.assert_array_equal(codes[idx].cpu().numpy(), oc)
 
 
+@pytest.mark.parametrize("layout,M,K", [("row", 9472, 512), ("row", 2000, 3840),
+                                         ("col", 2368, 3840), ("col", 1100, 16384)])
+def test_rotate_quant_f32_g16_many_blocks_per_cta(layout, M, K):
+    """Several row blocks per CTA: the blocks cycle through the CTA's tile buffers, later
+    blocks' copies landing while earlier ones are rotated and quantized, and the rotation of
+    one block overlaps the cluster's exchange of the previous block's maxima.  Every row's
+    codes and scale equal the oracle's bit for bit."""
+    g = torch.Generator().manual_seed(M + K)
+    x = torch.randn(M, K, generator=g)
+    x[:, torch.randperm(K, generator=g)[: K // 64]] *= 30.0
+    x[torch.randperm(M, generator=g)[:7]] *= 1e-3
+    if layout == "col":
+        x = _colmajor(x)
+    R = W.haar_orthogonal(16, torch.Generator().manual_seed(M)).float().contiguous()
+    codes, scales = ck.ck_rotate_quant(to_device(x), R.cuda(), 16)
+    torch.cuda.synchronize()
+    oc, os_ = oracle.rotate_quant(x, R, 16)
+    np.testing.assert_array_equal(scales.cpu().numpy(), os_)
+    np.testing.assert_array_equal(codes.cpu().numpy(), oc)
+
+
 @pytest.mark.parametrize("layout", ["col", "row"])
 def test_rotate_quant_f32_g16_caller_scale_and_non_finite(layout):
     M, K = 48, 256
