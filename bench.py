@@ -535,26 +535,68 @@ def run_ck(args, case, world, rank, local):
     x, out, ws, wp, wsc, bias = sets[0].x, sets[0].out, sets[0].ws, sets[0].wp, sets[0].wsc, sets[0].bias
     footprint = S * (x_bytes + wsz + out_bytes + w_bytes)
 
-    # ---- end to end through the public call with host buffers (pinned), copies timed
+    # ---- end to end through the public call with host buffers (pinned), copies timed: every
+    # step's input and output copies are inside the timed region.  Two schedules, the faster
+    # reported: one stream (copy in, linear, copy out, step after step), and three streams
+    # (host -> device, the linear, device -> host) with two device buffers of each kind, so the
+    # copies of neighbouring steps overlap the linear and each other (PCIe is full duplex) at
+    # the price of cross-stream waits, which dominate for small steps.
     xh = inp["x"].contiguous().pin_memory() if case.layout != "colmajor" else \
         inp["x"].t().contiguous().pin_memory().t()
-    xd = x.clone() if case.layout != "colmajor" else x.t().clone().t()
-    oh = torch.empty(M, N, dtype=out.dtype).pin_memory()
-    e2e_steps = max(3, min(args.steps, 20))
-    for i in range(2 + e2e_steps):
-        if i == 2:
-            barrier(world)
-            ea = torch.cuda.Event(enable_timing=True)
-            ea.record(stream)
-        xd.copy_(xh, non_blocking=True)
-        ck.ck_w4a4_linear(xd, R, g, wp, wsc, bias, out=out, workspace=ws, dev_status=status,
-                          stream=stream)
-        oh.copy_(out, non_blocking=True)
-    eb = torch.cuda.Event(enable_timing=True)
-    eb.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(ea.elapsed_time(eb) / e2e_steps, world)
+    nbuf = 2
+    xds = [x.clone() if case.layout != "colmajor" else x.t().clone().t() for _ in range(nbuf)]
+    outs = [torch.empty_like(out) for _ in range(nbuf)]
+    ohs = [torch.empty(M, N, dtype=out.dtype).pin_memory() for _ in range(nbuf)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_done = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_out = [torch.cuda.Event() for _ in range(nbuf)]
+
+    def e2e_run(n):
+        for i in range(n):
+            b = i % nbuf
+            if i >= nbuf:
+                s_in.wait_event(ev_done[b])     # the linear of step i - nbuf has read xds[b]
+            with torch.cuda.stream(s_in):
+                xds[b].copy_(xh, non_blocking=True)
+            ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if i >= nbuf:
+                stream.wait_event(ev_out[b])    # step i - nbuf's output has left outs[b]
+            ck.ck_w4a4_linear(xds[b], R, g, wp, wsc, bias, out=outs[b], workspace=ws,
+                              dev_status=status, stream=stream)
+            ev_done[b].record(stream)
+            s_out.wait_event(ev_done[b])
+            with torch.cuda.stream(s_out):
+                ohs[b].copy_(outs[b], non_blocking=True)
+            ev_out[b].record(s_out)
+
+    def e2e_serial(n):
+        for i in range(n):
+            xds[0].copy_(xh, non_blocking=True)
+            ck.ck_w4a4_linear(xds[0], R, g, wp, wsc, bias, out=outs[0], workspace=ws,
+                              dev_status=status, stream=stream)
+            ohs[0].copy_(outs[0], non_blocking=True)
+
+    def e2e_time(run, first, last, n):
+        run(2)
+        torch.cuda.synchronize()
+        barrier(world)
+        ea = torch.cuda.Event(enable_timing=True)
+        eb = torch.cuda.Event(enable_timing=True)
+        ea.record(first)
+        run(n)
+        eb.record(last)
+        torch.cuda.synchronize()
+        return max_over_ranks(ea.elapsed_time(eb) / n, world)
+
+    e2e_steps = max(3, min(args.steps, 40))
+    e2e_all = {"one stream": e2e_time(e2e_serial, stream, stream, e2e_steps),
+               "three streams": e2e_time(e2e_run, s_in, s_out, e2e_steps)}
+    e2e_sched = min(e2e_all, key=e2e_all.get)
+    e2e_ms = e2e_all[e2e_sched]
     e2e_val = flops * world / (e2e_ms * 1e-3) / 1e12
+    oh = ohs[0]
 
     if rank != 0:
         return None
@@ -568,9 +610,16 @@ def run_ck(args, case, world, rank, local):
                    "gbs": s1_gbs, "hbm_peak_gbs": pk["hbm_gbs"], "frac": s1_gbs / pk["hbm_gbs"],
                    "traffic": recorded_traffic(rq_file, case.name)},
         "gemm_ms": gemm_ms,
-        "e2e": {"value": e2e_val, "unit": UNIT, "ms_per_step": e2e_ms,
+        "e2e": {"value": e2e_val, "unit": UNIT, "ms_per_step": e2e_ms, "steps": e2e_steps,
                 "h2d_bytes_per_step": xh.numel() * xh.element_size(),
-                "d2h_bytes_per_step": oh.numel() * oh.element_size()},
+                "d2h_bytes_per_step": oh.numel() * oh.element_size(),
+                "schedule": e2e_sched,
+                "ms_per_step_by_schedule": e2e_all,
+                "method": "public linear call on a device copy of pinned host activations, the "
+                          "output copied back to pinned host memory, every step; one stream, "
+                          "or three (copies in, the linear, copies out; two buffers each, so "
+                          "neighbouring steps' copies overlap), the faster reported; events "
+                          "from before the first input copy to after the last output copy"},
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "wall_s_timed_region": t_wall,

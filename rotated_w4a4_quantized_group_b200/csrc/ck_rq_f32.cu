@@ -20,7 +20,7 @@
 // Row-major input (unit K stride) and column-major input (unit M stride, the transposed view
 // of a (K, M) buffer) are both read by TMA straight from HBM, each byte once:
 //   - a block of RB rows is split along K over a thread-block cluster of C CTAs, each holding
-//     its K slice of the block in shared memory (at most 64 KB, two CTAs per SM);
+//     its K slice of the block in shared memory (at most 64 KB; two or three CTAs per SM);
 //   - column-major input: 16 rows per block, boxes of 16 rows x 256 channels (64-byte rows);
 //     row-major input: boxes of up to 256 groups x RB rows, as (channel, group, row);
 //   - eight warps rotate the slice in place: 8 group-rows x 16 channels per task, x converted
@@ -98,8 +98,9 @@ __device__ __forceinline__ float f32_row_scale(float amax, const float* scale_in
     return (s < FLT_MIN) ? FLT_MIN : s;   // lower clamp; NaN stays NaN
 }
 
-template <bool COL>
-__global__ void __launch_bounds__(rqf32::kThreads, 2)
+// MINB: CTAs per SM the registers are budgeted for (2: up to 128 a thread; 3: up to 85)
+template <bool COL, int MINB>
+__global__ void __launch_bounds__(rqf32::kThreads, MINB)
     rq_f32_g16_kernel(const __grid_constant__ CUtensorMap xmap, const float* __restrict__ R,
                       const float* __restrict__ scale_in, int8_t* __restrict__ codes,
                       float* __restrict__ scales, RqF32Params p, int* dev_status) {
@@ -734,14 +735,6 @@ ck_status launch_rq_f32_g16(const void* x, int64_t M, int64_t K, int64_t sm, int
     if (st != CK_OK) return st;
 
     const size_t smem = (size_t)p.nboxes * p.box_stride + 1024;
-    auto kern = col ? rq_f32_g16_kernel<true> : rq_f32_g16_kernel<false>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return CK_ERR_CUDA;
-    if (C > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-                     cudaSuccess)
-        return CK_ERR_UNSUPPORTED;
-
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -753,16 +746,45 @@ ck_status launch_rq_f32_g16(const void* x, int64_t M, int64_t K, int64_t sm, int
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // persistent clusters: as many as can be resident (two CTAs per SM), at most one per block
     cfg.gridDim = dim3((unsigned)C, 1, 1);
-    int max_clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess || max_clusters < 1)
-        return CK_ERR_UNSUPPORTED;
-    const int64_t gy = p.nblocks < max_clusters ? p.nblocks : max_clusters;
-    cfg.gridDim = dim3((unsigned)C, (unsigned)gy, 1);
-    if (cudaLaunchKernelEx(&cfg, kern, map, static_cast<const float*>(R), scale_in, codes, scales,
-                           p, dev_status) != cudaSuccess)
-        return CK_ERR_CUDA;
+    // persistent clusters: as many as can be resident, at most one per block.  Three CTAs per
+    // SM (registers capped at 85) when the blocks outnumber what two CTAs per SM hold: more
+    // CTAs overlap one another's load, rotation, cluster exchange and quantize phases; with
+    // fewer blocks the wider register budget makes each CTA faster.
+    auto prepare = [&](auto kern, int& max_clusters) -> ck_status {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return CK_ERR_CUDA;
+        if (C > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                          1) != cudaSuccess)
+            return CK_ERR_UNSUPPORTED;
+        max_clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess ||
+            max_clusters < 1)
+            return CK_ERR_UNSUPPORTED;
+        return CK_OK;
+    };
+    auto run = [&](auto kern, int max_clusters) -> ck_status {
+        const int64_t gy = p.nblocks < max_clusters ? p.nblocks : max_clusters;
+        cfg.gridDim = dim3((unsigned)C, (unsigned)gy, 1);
+        if (cudaLaunchKernelEx(&cfg, kern, map, static_cast<const float*>(R), scale_in, codes,
+                               scales, p, dev_status) != cudaSuccess)
+            return CK_ERR_CUDA;
+        return CK_OK;
+    };
+    auto k2 = col ? rq_f32_g16_kernel<true, 2> : rq_f32_g16_kernel<false, 2>;
+    auto k3 = col ? rq_f32_g16_kernel<true, 3> : rq_f32_g16_kernel<false, 3>;
+    int mc2 = 0, mc3 = 0;
+    st = prepare(k2, mc2);
+    if (st != CK_OK) return st;
+    if (p.nblocks > mc2) {
+        st = prepare(k3, mc3);
+        if (st != CK_OK) return st;
+        st = mc3 > mc2 ? run(k3, mc3) : run(k2, mc2);
+    } else {
+        st = run(k2, mc2);
+    }
+    if (st != CK_OK) return st;
     return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
 }
 
