@@ -55,6 +55,12 @@ ck_status launch_rq_tf32(const void* x, int64_t M, int64_t K, int64_t sm, int64_
 ck_status launch_rq_f32_ffma256(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
                                 const void* R, const float* scale_in, int8_t* codes, int64_t ldq,
                                 float* scales, int qmax, int* dev_status, cudaStream_t stream);
+// fp32 stage 1 at g = 64 or 256 on row-major rows (ck_rq_tf32.cu picks the kernel);
+// CK_ERR_UNSUPPORTED for shapes no kernel there takes.
+ck_status launch_rq_f32_wide(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
+                             const void* R, int g, const float* scale_in, int8_t* codes,
+                             int64_t ldq, float* scales, int qmax, int* dev_status,
+                             cudaStream_t stream);
 ck_status launch_rq_f32_g16(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
                             const void* R, const float* scale_in, int8_t* codes, int64_t ldq,
                             float* scales, int qmax, int* dev_status, cudaStream_t stream);

@@ -22,6 +22,8 @@
 //                      quantize from shared memory.
 //   rq_f32_g16_kernel  (ck_rq_f32.cu) fp32, g = 16, row-major or column-major: K split over
 //                      a cluster, FP64 tensor-core rotation, absmax over distributed shared memory.
+//   fp32, g in {64, 256}, row-major: launch_rq_f32_wide (ck_rq_tf32.cu) picks the split-TF32
+//                      tensor-core kernel (g = 64) or the FFMA kernel (g = 256).
 //   rq_generic_kernel  every dtype, g and stride: one row per CTA step, fp32 FFMA with R
 //                      in shared memory (or read through L1 when it does not fit).
 // The TMA-fed kernels store 16 codes at a time where the code rows are 16-byte aligned; the
@@ -1406,14 +1408,9 @@ ck_status launch_rotate_quant(const void* x, ck_dtype dt, int64_t M, int64_t K, 
         return g == 64 ? launch_mma<__half, 64>(CK_RQ_ARGS) : launch_mma<__half, 16>(CK_RQ_ARGS);
     }
 #undef CK_RQ_ARGS
-    if (dt == CK_F32 && g == 64) {
-        const ck_status st = launch_rq_tf32(x, M, K, sm, sk, R, scale_in, codes, ldq, scales,
-                                            qmax, dev_status, stream);
-        if (st != CK_ERR_UNSUPPORTED) return st;
-    }
-    if (dt == CK_F32 && g == 256) {
-        const ck_status st = launch_rq_f32_ffma256(x, M, K, sm, sk, R, scale_in, codes, ldq, scales,
-                                                   qmax, dev_status, stream);
+    if (dt == CK_F32 && (g == 64 || g == 256)) {
+        const ck_status st = launch_rq_f32_wide(x, M, K, sm, sk, R, g, scale_in, codes, ldq,
+                                                scales, qmax, dev_status, stream);
         if (st != CK_ERR_UNSUPPORTED) return st;
     }
     if (dt == CK_F32 && g == 16) {

@@ -435,4 +435,17 @@ ck_status launch_rq_tf32(const void* x, int64_t M, int64_t K, int64_t sm, int64_
     return scale_in ? run(rq_tf32_kernel<false, 1>) : run(rq_tf32_kernel<true, 1>);
 }
 
+ck_status launch_rq_f32_wide(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
+                             const void* R, int g, const float* scale_in, int8_t* codes,
+                             int64_t ldq, float* scales, int qmax, int* dev_status,
+                             cudaStream_t stream) {
+    if (g == 64)
+        return launch_rq_tf32(x, M, K, sm, sk, R, scale_in, codes, ldq, scales, qmax, dev_status,
+                              stream);
+    if (g == 256)
+        return launch_rq_f32_ffma256(x, M, K, sm, sk, R, scale_in, codes, ldq, scales, qmax,
+                                     dev_status, stream);
+    return CK_ERR_UNSUPPORTED;
+}
+
 }  // namespace ck
