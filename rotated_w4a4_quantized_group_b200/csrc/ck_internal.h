@@ -47,8 +47,11 @@ ck_status launch_rotate_quant(const void* x, ck_dtype dt, int64_t M, int64_t K, 
                               int8_t* codes, int64_t ldq, float* scales, int qmax,
                               int* dev_status, cudaStream_t stream);
 
-// Stage 1 for fp32 input with g = 16, row-major or column-major, on the FP64 tensor-core
-// rotation (ck_rq_f32.cu).  Returns CK_ERR_UNSUPPORTED for shapes or layouts it does not take.
+// fp32 stage-1 kernels; each returns CK_ERR_UNSUPPORTED for shapes or layouts it does not take:
+//   launch_rq_tf32         g = 64, row-major, split TF32 on the tensor cores (ck_rq_tf32.cu)
+//   launch_rq_f32_ffma256  g = 256, row-major, K <= 16384, FFMA (ck_rq_f32_256.cu)
+//   launch_rq_f32_g16      g = 16, row-major or column-major, FP64 tensor-core rotation
+//                          (ck_rq_f32.cu)
 ck_status launch_rq_tf32(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
                          const void* R, const float* scale_in, int8_t* codes, int64_t ldq,
                          float* scales, int qmax, int* dev_status, cudaStream_t stream);

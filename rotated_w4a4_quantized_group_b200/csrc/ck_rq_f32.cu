@@ -397,266 +397,6 @@ __global__ void __launch_bounds__(rqf32::kThreads, MINB)
     if (ncta > 1) cluster_sync_all();
 }
 
-// ===================================================================== fp32, g = 256, FFMA
-//
-// g = 256 on row-major fp32 rows: R (256 KB) does not fit in shared memory, so it passes
-// through it in four blocks of 64 rows (i = 64 b .. 64 b + 63, all 256 channels, 64 KB).  Pass
-// b adds x[r][i] R[i][c] for its 64 values of i to the partial sums left in the y buffer by pass
-// b - 1: each y is the fp32 FMA chain over i = 0 .. 255 in order, as one pass would form it.
-// Blocks of whole rows arrive by TMA (one 3-D box of 256 channels x K / 256 groups x RB rows)
-// into one of two buffers.  A work unit is 8 group-rows x 64 channels (lane l: channels
-// 64 cb + 2 l, + 1); the last pass folds |y| into the row maxima; then the codes.
-struct RqFfmaParams {
-    int64_t M, K, ldq, nblocks;
-    int RB;               // rows per block
-    int ngr;              // group-rows per block, RB K / 256
-    uint32_t box_bytes;   // RB K 4
-    int vec_codes, qmax;
-};
-
-namespace rqff256 {
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kUnitGR = 8;                  // group-rows per work unit
-constexpr int kMaxRB = 8;
-constexpr size_t kRBlockBytes = 64 * 256 * 4;
-constexpr size_t kSmemMax = 220 * 1024;
-}  // namespace rqff256
-
-__global__ void __launch_bounds__(rqff256::kThreads, 1)
-    rq_f32_ffma256_kernel(const __grid_constant__ CUtensorMap xmap, const float* __restrict__ R,
-                          const float* __restrict__ scale_in, int8_t* __restrict__ codes,
-                          float* __restrict__ scales, RqFfmaParams p, int* dev_status) {
-    // the linear's GEMM, launched as this kernel's dependent, may start its prologue now
-    grid_dependents_launch();
-    using namespace rqff256;
-    extern __shared__ __align__(1024) unsigned char f256_smem[];
-    float* base = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(f256_smem) + 127) &
-                                           ~uintptr_t(127));
-    float* const Rb = base;                                   // R[64 b + i][c], 64 x 256
-    float* const ybuf = Rb + 64 * 256;                        // RB x K partial sums
-    float* const xbuf0 = ybuf + (size_t)p.RB * p.K;           // the two block buffers
-    float* const xbuf1 = xbuf0 + (size_t)p.RB * p.K;
-    __shared__ __align__(8) uint64_t full[2];
-    __shared__ unsigned int amax_sh[kMaxRB];
-    __shared__ float row_s[kMaxRB], row_r[kMaxRB];
-    __shared__ int abort_flag;
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int gpr = (int)(p.K / 256);                  // group-rows per row
-    uint32_t issued = 0, landed = 0;
-    bool landing = true;
-    if (tid < kMaxRB) amax_sh[tid] = 0u;
-    if (tid == 0) {
-        mbar_init(&full[0], 1);
-        mbar_init(&full[1], 1);
-        abort_flag = 0;
-        fence_mbar_init();
-        tma_prefetch_desc(&xmap);
-        for (int b = 0; b < 2; ++b) {
-            const int64_t blk = blockIdx.x + (int64_t)b * gridDim.x;
-            if (blk < p.nblocks) {
-                mbar_arrive_expect_tx(&full[b], p.box_bytes);
-                tma_load_3d(b ? xbuf1 : xbuf0, &xmap, &full[b], 0, 0, (int32_t)(blk * p.RB));
-                ++issued;
-            }
-        }
-    }
-    __syncthreads();
-
-    const int noct = (p.ngr + kUnitGR - 1) / kUnitGR;   // octets of group-rows per block
-    const int nunits = noct * 4;                         // x 4 channel blocks
-    uint32_t it = 0;
-    for (int64_t blk = blockIdx.x; blk < p.nblocks; blk += gridDim.x, ++it) {
-        const int buf = (int)(it & 1u);
-        const uint32_t par = (it >> 1) & 1u;
-        const float* xt = buf ? xbuf1 : xbuf0;
-        const int64_t m0 = blk * p.RB;
-        const bool skip = abort_flag != 0;
-        const bool ok = !skip && __all_sync(0xffffffffu, mbar_wait(&full[buf], par, &abort_flag, dev_status));
-        if (tid == 0) {
-            landing = landing && ok;
-            if (landing) ++landed;
-        }
-        for (int b = 0; b < 4; ++b) {
-            __syncthreads();   // every warp is done with the previous R block
-            if (ok) {
-                const float4* src = reinterpret_cast<const float4*>(R + (size_t)b * 64 * 256);
-                float4* dst = reinterpret_cast<float4*>(Rb);
-                for (int i = tid; i < 64 * 256 / 4; i += kThreads) dst[i] = __ldg(src + i);
-            }
-            __syncthreads();
-            if (!ok) continue;
-            for (int u = warp; u < nunits; u += kWarps) {
-                const int gr0 = (u >> 2) * kUnitGR, cb = u & 3;
-                const int nr = (p.ngr - gr0) < kUnitGR ? (p.ngr - gr0) : kUnitGR;
-                const int ch = 64 * cb + 2 * lane;
-                float a0[kUnitGR], a1[kUnitGR];
-#pragma unroll
-                for (int r = 0; r < kUnitGR; ++r) {
-                    if (b > 0 && r < nr) {
-                        const float2 v = *reinterpret_cast<const float2*>(ybuf + (size_t)(gr0 + r) * 256 + ch);
-                        a0[r] = v.x;
-                        a1[r] = v.y;
-                    } else {
-                        a0[r] = a1[r] = 0.f;
-                    }
-                }
-                const float* xg = xt + (size_t)gr0 * 256 + 64 * b;
-#pragma unroll 2
-                for (int i = 0; i < 64; i += 4) {
-                    float2 rq[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        rq[q] = *reinterpret_cast<const float2*>(Rb + (i + q) * 256 + ch);
-#pragma unroll
-                    for (int r = 0; r < kUnitGR; ++r) {
-                        if (r < nr) {
-                            const float4 xv = *reinterpret_cast<const float4*>(xg + r * 256 + i);
-                            a0[r] = __fmaf_rn(xv.x, rq[0].x, a0[r]);
-                            a1[r] = __fmaf_rn(xv.x, rq[0].y, a1[r]);
-                            a0[r] = __fmaf_rn(xv.y, rq[1].x, a0[r]);
-                            a1[r] = __fmaf_rn(xv.y, rq[1].y, a1[r]);
-                            a0[r] = __fmaf_rn(xv.z, rq[2].x, a0[r]);
-                            a1[r] = __fmaf_rn(xv.z, rq[2].y, a1[r]);
-                            a0[r] = __fmaf_rn(xv.w, rq[3].x, a0[r]);
-                            a1[r] = __fmaf_rn(xv.w, rq[3].y, a1[r]);
-                        }
-                    }
-                }
-                int row_of = gr0 / gpr, left = gpr - (gr0 - row_of * gpr);
-                float run = 0.f;
-                int run_row = -1;
-#pragma unroll
-                for (int r = 0; r < kUnitGR; ++r) {
-                    if (r < nr) {
-                        *reinterpret_cast<float2*>(ybuf + (size_t)(gr0 + r) * 256 + ch) = make_float2(a0[r], a1[r]);
-                        if (b == 3) {   // final values: fold |y| into the row maximum
-                            float mx = fmax_nan(fabsf(a0[r]), fabsf(a1[r]));
-#pragma unroll
-                            for (int o = 16; o > 0; o >>= 1)
-                                mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                            if (left == 0) {
-                                ++row_of;
-                                left = gpr;
-                            }
-                            --left;
-                            if (row_of != run_row) {
-                                if (run_row >= 0 && lane == 0) atomicMax(&amax_sh[run_row], __float_as_uint(run));
-                                run_row = row_of;
-                                run = mx;
-                            } else {
-                                run = fmax_nan(run, mx);
-                            }
-                        }
-                    }
-                }
-                if (b == 3 && run_row >= 0 && lane == 0) atomicMax(&amax_sh[run_row], __float_as_uint(run));
-            }
-        }
-        __syncthreads();
-        // the x buffer is free: the block after next loads into it
-        if (tid == 0) {
-            const int64_t nxt = blk + 2 * (int64_t)gridDim.x;
-            if (abort_flag == 0 && nxt < p.nblocks) {
-                mbar_arrive_expect_tx(&full[buf], p.box_bytes);
-                tma_load_3d(buf ? xbuf1 : xbuf0, &xmap, &full[buf], 0, 0, (int32_t)(nxt * p.RB));
-                ++issued;
-            }
-        }
-        // ---------------------------------------------------------------- row scales
-        if (tid < p.RB) {
-            const float s = f32_row_scale(__uint_as_float(amax_sh[tid]), scale_in, p.qmax);
-            const RowDivisor dv(s, p.qmax);
-            row_s[tid] = s;
-            row_r[tid] = dv.r;
-            if (m0 + tid < p.M && ok) scales[m0 + tid] = s;
-            amax_sh[tid] = 0u;
-        }
-        __syncthreads();
-        // ---------------------------------------------------------------- quantize + store
-        if (ok) {
-            const int rows = (int)((p.M - m0) < p.RB ? (p.M - m0) : p.RB);
-            const int cpr = (int)(p.K / 16);
-            for (int m = 0; m < rows; ++m)
-            for (int j = tid; j < cpr; j += kThreads) {
-                RowDivisor dv(row_s[m], p.qmax);
-                dv.r = row_r[m];
-                const float* src = ybuf + (size_t)m * p.K + 16 * j;
-                float y[16];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 v = *reinterpret_cast<const float4*>(src + 4 * q);
-                    y[4 * q] = v.x;
-                    y[4 * q + 1] = v.y;
-                    y[4 * q + 2] = v.z;
-                    y[4 * q + 3] = v.w;
-                }
-                uint32_t out[4];
-                quant16_any(y, dv, scale_in == nullptr, out);
-                int8_t* dst = codes + (m0 + m) * p.ldq + 16 * j;
-                if (p.vec_codes) {
-                    *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) dst[q] = (int8_t)((out[q / 4] >> (8 * (q % 4))) & 0xFF);
-                }
-            }
-        }
-    }
-    // after a timeout, copies still in flight land before the CTA leaves
-    if (tid == 0)
-        for (uint32_t k = landed; k < issued; ++k) mbar_wait(&full[k & 1u], (k >> 1) & 1u, nullptr, nullptr);
-    __syncthreads();
-}
-
-// fp32, g = 256, unit K stride, 16-byte-aligned x, R and row pitch, K / 256 <= 256.  Returns
-// CK_ERR_UNSUPPORTED when the shape does not fit.
-ck_status launch_rq_f32_ffma256(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
-                                const void* R, const float* scale_in, int8_t* codes, int64_t ldq,
-                                float* scales, int qmax, int* dev_status, cudaStream_t stream) {
-    using namespace rqff256;
-    if (sk != 1 || !aligned(x, 16) || !aligned(R, 16) || K % 256 != 0 || K / 256 > 256 ||
-        (M > 1 && (sm % 4 != 0 || sm < K)) || M >= (1LL << 31))
-        return CK_ERR_UNSUPPORTED;
-    const size_t row_bytes = (size_t)K * 4;
-    // R block + y + two x buffers of RB rows
-    int64_t rb = (int64_t)((kSmemMax - kRBlockBytes - 128) / (3 * row_bytes));
-    if (rb < 1) return CK_ERR_UNSUPPORTED;
-    if (rb > kMaxRB) rb = kMaxRB;
-    const int64_t spread = (M + num_sms() - 1) / num_sms();
-    if (rb > spread) rb = spread < 1 ? 1 : spread;
-    if (rb > M) rb = M;
-    RqFfmaParams p;
-    p.M = M;
-    p.K = K;
-    p.ldq = ldq;
-    p.RB = (int)rb;
-    p.ngr = (int)(rb * (K / 256));
-    p.nblocks = (M + rb - 1) / rb;
-    p.box_bytes = (uint32_t)(rb * row_bytes);
-    p.vec_codes = (aligned(codes, 16) && ldq % 16 == 0) ? 1 : 0;
-    p.qmax = qmax;
-
-    CUtensorMap map;
-    const uint64_t dims[3] = {256, (uint64_t)(K / 256), (uint64_t)M};
-    const uint64_t strides[2] = {1024, (uint64_t)(M > 1 ? sm : K) * 4};
-    const uint32_t box[3] = {256, (uint32_t)(K / 256), (uint32_t)rb};
-    const ck_status st = encode_tma(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, x, dims, strides,
-                                    box, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (st != CK_OK) return st;
-    const size_t smem = 128 + kRBlockBytes + 3 * (size_t)p.box_bytes;
-    if (cudaFuncSetAttribute(rq_f32_ffma256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-        return CK_ERR_CUDA;
-    const int grid = (int)(p.nblocks < num_sms() ? p.nblocks : num_sms());
-    rq_f32_ffma256_kernel<<<grid, kThreads, smem, stream>>>(map, static_cast<const float*>(R),
-                                                            scale_in, codes, scales, p, dev_status);
-    return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
-}
-
-// fp32, g = 16, unit K stride (row-major) or unit M stride (column-major) with 16-byte-aligned
-// x and row or column pitch.  Returns CK_ERR_UNSUPPORTED when the shape does not fit.
 ck_status launch_rq_f32_g16(const void* x, int64_t M, int64_t K, int64_t sm, int64_t sk,
                             const void* R, const float* scale_in, int8_t* codes, int64_t ldq,
                             float* scales, int qmax, int* dev_status, cudaStream_t stream) {

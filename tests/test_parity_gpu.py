@@ -203,13 +203,16 @@ def test_rotate_quant_f32_g64_blocks(M, groups, pitch):
 
 
 @pytest.mark.parametrize("M,groups,pitch", [(703, 3, 0), (100, 15, 0), (300, 15, 64), (5, 40, 0),
-                                            (3, 48, 0), (150, 1, 0)])
+                                            (3, 48, 0), (150, 1, 0), (1200, 15, 0), (10000, 1, 0),
+                                            (300, 64, 0), (4, 80, 0)])
 def test_rotate_quant_f32_g256_blocks(M, groups, pitch):
-    """fp32 rows at g = 256 (the FFMA kernel with R passing through shared memory in four
-    blocks of 64 rows): blocks of 5 rows with a ragged last one (703 rows of 3 groups), one-row
-    blocks (15, 40 and 48 groups), a row pitch past K, and one-group rows.  The partial sums
-    continue across the four passes, so each value is the in-order fp32 FMA chain.  R is a
-    non-symmetric orthogonal matrix.  Every output is compared."""
+    """fp32 rows at g = 256 (the FFMA kernel: R streams through shared memory in slices of 32
+    rows, the partial sums stay in registers): blocks of 5 rows with a ragged last one (703
+    rows of 3 groups), one-row blocks (15, 40 and 48 groups), a row pitch past K, one-group
+    rows, several four-row blocks per CTA (1200 x 15 groups), 64-row blocks (10000 x 1 group),
+    the widest row a block takes (64 groups), and a wider one (80 groups) that the generic
+    kernel takes.  Each value is the in-order fp32 FMA chain.  R is a non-symmetric orthogonal
+    matrix.  Every output is compared."""
     g, K = 256, 256 * groups
     case = W.RotateCase(f"f32_g256_{M}_{groups}", M=M, K=K, g=g, dtype="f32", seed=M + groups)
     x = W.make_rotate_inputs(case)["x"]
