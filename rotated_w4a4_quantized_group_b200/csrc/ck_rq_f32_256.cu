@@ -53,6 +53,10 @@ struct RqF256Params {
     int vec_codes, qmax;
 };
 
+// NJ: group-rows a warp computes, ceil(RB K / 256 / 8).  Every warp computes NJ of them (the
+// x buffers hold 8 NJ group-rows), so the FMA step has no per-row branch; group-rows past the
+// block's (never written by the copy) are neither folded into a maximum nor stored.
+template <int NJ>
 __global__ void __launch_bounds__(rqf256::kThreads, 1)
     rq_f32_ffma256_kernel(const __grid_constant__ CUtensorMap xmap,
                           const __grid_constant__ CUtensorMap rmap,
@@ -67,7 +71,7 @@ __global__ void __launch_bounds__(rqf256::kThreads, 1)
     float* const rslot0 = base;                                 // R rows 32 s .. 32 s + 31
     float* const rslot1 = base + kSlice * 256;
     float* const xbuf0 = base + 2 * kSlice * 256;               // the two row-block buffers
-    float* const xbuf1 = xbuf0 + (size_t)p.RB * p.K;
+    float* const xbuf1 = xbuf0 + (size_t)NJ * kWarps * 256;
     __shared__ __align__(8) uint64_t xfull[2], rfull[2];
     __shared__ unsigned int amax_sh[kMaxRB];
     __shared__ float row_s[kMaxRB], row_r[kMaxRB];
@@ -75,7 +79,6 @@ __global__ void __launch_bounds__(rqf256::kThreads, 1)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int ngr = p.RB * p.gpr;                                 // group-rows a block
-    const int nj = ngr > warp ? (ngr - warp + kWarps - 1) / kWarps : 0;   // this warp's
     const int nmine = (int)((p.nblocks - 1 - blockIdx.x) / gridDim.x + 1);
     const int nslices = nmine * kSlices;                          // R slices this CTA reads
     int xissued = 0, rissued = 0;                                 // thread 0's copies
@@ -110,9 +113,9 @@ __global__ void __launch_bounds__(rqf256::kThreads, 1)
         const float* xt = (it & 1) ? xbuf1 : xbuf0;
         bool ok = abort_flag == 0 &&
                   mbar_wait(&xfull[it & 1], (uint32_t)(it >> 1) & 1u, &abort_flag, dev_status);
-        float acc[kRows][8];
+        float acc[NJ][8];
 #pragma unroll
-        for (int j = 0; j < kRows; ++j)
+        for (int j = 0; j < NJ; ++j)
 #pragma unroll
             for (int c = 0; c < 8; ++c) acc[j][c] = 0.f;
         for (int s = 0; s < kSlices; ++s) {
@@ -125,19 +128,18 @@ __global__ void __launch_bounds__(rqf256::kThreads, 1)
                 for (int i = 0; i < kSlice; i += 4) {
                     // every operand of the step is loaded before the first FMA, so that the
                     // loads' latency is paid once per step, not once per group-row
-                    float4 ra[4], rb[4], xv[kRows];
+                    float4 ra[4], rb[4], xv[NJ];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         ra[u] = *reinterpret_cast<const float4*>(rs + (i + u) * 256 + c0);
                         rb[u] = *reinterpret_cast<const float4*>(rs + (i + u) * 256 + 128 + c0);
                     }
 #pragma unroll
-                    for (int j = 0; j < kRows; ++j)
-                        xv[j] = j < nj ? *reinterpret_cast<const float4*>(xs + (size_t)j * kWarps * 256 + i)
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int j = 0; j < NJ; ++j)
+                        xv[j] = *reinterpret_cast<const float4*>(xs + (size_t)j * kWarps * 256 + i);
 #pragma unroll
-                    for (int j = 0; j < kRows; ++j) {
-                        if (j < nj) {
+                    for (int j = 0; j < NJ; ++j) {
+                        {
                             const float xq[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
 #pragma unroll
                             for (int u = 0; u < 4; ++u) {
@@ -164,8 +166,8 @@ __global__ void __launch_bounds__(rqf256::kThreads, 1)
         // ---------------------------------------------------------------- row maxima
         if (ok) {
 #pragma unroll
-            for (int j = 0; j < kRows; ++j) {
-                if (j < nj) {
+            for (int j = 0; j < NJ; ++j) {
+                if (warp + kWarps * j < ngr) {
                     float mx = 0.f;
 #pragma unroll
                     for (int c = 0; c < 8; ++c) mx = fmax_nan(mx, fabsf(acc[j][c]));
@@ -190,8 +192,8 @@ __global__ void __launch_bounds__(rqf256::kThreads, 1)
         // ---------------------------------------------------------------- codes
         if (ok) {
 #pragma unroll
-            for (int j = 0; j < kRows; ++j) {
-                if (j < nj) {
+            for (int j = 0; j < NJ; ++j) {
+                if (warp + kWarps * j < ngr) {
                     const int gr = warp + kWarps * j;
                     const int m = gr / p.gpr, gi = gr - m * p.gpr;
                     if (m0 + m < p.M) {
@@ -270,14 +272,26 @@ ck_status launch_rq_f32_ffma256(const void* x, int64_t M, int64_t K, int64_t sm,
                                         box, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (st != CK_OK) return st;
     }
-    const size_t smem = 128 + 2 * (size_t)kSliceBytes + 2 * (size_t)p.box_bytes;
-    if (cudaFuncSetAttribute(rq_f32_ffma256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-        return CK_ERR_CUDA;
+    const int nj = (int)((rb * gpr + kWarps - 1) / kWarps);   // group-rows a warp, 1 .. 8
+    const size_t smem = 128 + 2 * (size_t)kSliceBytes + 2 * (size_t)nj * kWarps * 1024;
     const int grid = (int)(p.nblocks < num_sms() ? p.nblocks : num_sms());
-    rq_f32_ffma256_kernel<<<grid, kThreads, smem, stream>>>(xm, rm, scale_in, codes, scales, p,
-                                                            dev_status);
-    return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+    auto run = [&](auto kern) -> ck_status {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return CK_ERR_CUDA;
+        kern<<<grid, kThreads, smem, stream>>>(xm, rm, scale_in, codes, scales, p, dev_status);
+        return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
+    };
+    switch (nj) {
+        case 1: return run(rq_f32_ffma256_kernel<1>);
+        case 2: return run(rq_f32_ffma256_kernel<2>);
+        case 3: return run(rq_f32_ffma256_kernel<3>);
+        case 4: return run(rq_f32_ffma256_kernel<4>);
+        case 5: return run(rq_f32_ffma256_kernel<5>);
+        case 6: return run(rq_f32_ffma256_kernel<6>);
+        case 7: return run(rq_f32_ffma256_kernel<7>);
+        default: return run(rq_f32_ffma256_kernel<8>);
+    }
 }
 
 }  // namespace ck
