@@ -25,13 +25,13 @@
 // 256), each part its own 64-column block of the accumulator:
 //   warp 0      TMA of x: per tile and part, two boxes of 32 channels (128 bytes, 128-byte
 //               swizzle) of every group, into a ring of 16 KB stages
-//   warps 2, 3  the split: mid and lo of each stage into two twin stages (and +-inf moved out
-//               of hi)
+//   warps 2-5   the split: mid and lo of each stage into two twin stages (and +-inf moved out
+//               of hi); four warps, so that the split keeps pace with the copies and the MMAs
 //   warp 1      TMEM and the MMAs: per 8 values of i, tcgen05.mma kind::tf32 of hi Rhi, hi Rlo,
 //               mid Rhi and lo Rhi (M = 128 group-rows, N = 64 channels), R^T (hi and lo)
 //               resident in shared memory; the whole warp walks the ring, one elected lane
 //               issues
-//   warps 4-19  four groups of four epilogue warps (four tiles in flight): read the fp32
+//   warps 6-21  four groups of four epilogue warps (four tiles in flight): read the fp32
 //               accumulator twice from TMEM, the row absmax through shared atomics and a group
 //               barrier, the scale, the codes in 16-byte stores
 // Every wait is bounded; a timeout records CK_ERR_TIMEOUT and the kernel drains and returns.
@@ -45,8 +45,8 @@
 namespace ck {
 
 namespace rqtf {
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpSplit0 = 2, kSplitWarps = 2;
-constexpr int kEpiWarp0 = 4, kEpiWarps = 16, kGrpWarps = 4;
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpSplit0 = 2, kSplitWarps = 4;
+constexpr int kEpiWarp0 = 6, kEpiWarps = 16, kGrpWarps = 4;
 constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
 constexpr int kAcc = kEpiWarps / kGrpWarps;       // tiles in flight
 constexpr int kStages = 3;                        // 16 KB x stages (and as many mid and lo)
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(rqtf::kThreads, 1)
         // ---------------------------------------------------------------- split
         // mid and lo stages s from x element by element (the stages share one layout); a +-inf
         // x goes whole into mid and leaves 0 in hi
-        const int st = (warp - kWarpSplit0) * 32 + lane;   // 0 .. 63
+        const int st = (warp - kWarpSplit0) * 32 + lane;   // 0 .. 32 kSplitWarps - 1
         for (int n = 0; n < my_boxes; ++n) {
             const int s = n % kStages;
             if (!__all_sync(0xffffffffu, mbar_wait(&x_full[s], (uint32_t)(n / kStages) & 1u,
