@@ -46,7 +46,7 @@ extern "C" {
 typedef enum {
     CK_OK = 0,
     CK_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad dtype, bad group size        */
-    CK_ERR_UNSUPPORTED = 2,   /* a valid call this build does not implement               */
+    CK_ERR_UNSUPPORTED = 2,   /* a valid call this library does not implement             */
     CK_ERR_OVERFLOW = 3,      /* 64 * K > INT32_MAX: the INT32 accumulator could overflow */
     CK_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required               */
     CK_ERR_CUDA = 5,          /* a CUDA runtime/driver call or a launch failed            */
@@ -80,7 +80,7 @@ typedef enum { CK_F32 = 0, CK_F16 = 1, CK_BF16 = 2, CK_I8 = 3 } ck_dtype;
  * from an exact-arithmetic evaluation where y / s lies within rounding of a half-integer.
  * Errors: CK_ERR_INVALID_ARG (null x/R/codes/scales, M < 0, K <= 0, K % g != 0,
  * bad g or dtype, ldq < K, R not 16-byte aligned), CK_ERR_UNSUPPORTED (a shape no kernel of
- * this build takes: an fp32 row of more than about 56,000 channels, unless g = 16 and x is
+ * this library takes: an fp32 row of more than about 56,000 channels, unless g = 16 and x is
  * row-major or column-major with a 16-byte-aligned pitch), CK_ERR_CUDA (launch failure).
  */
 ck_status ck_rotate_quant(const void* x, ck_dtype x_dtype, int64_t M, int64_t K,
