@@ -8,12 +8,14 @@
 //   s[m] = max(fp32(max_k |y[m, k]|) / 7, FLT_MIN)   or the caller's tensor-wise scale
 //   q[m, k] = clamp(round_half_even(y[m, k] / s[m]), -8, 7)
 //
-// Four kernels, tried in this order:
-//   rq_tc_kernel       bf16/fp16, g in {64, 256}, rows of at most 128 groups, unit K stride,
-//                      16-byte aligned x and R.  Whole rows fill the 128 lanes of a
-//                      tcgen05.mma.kind::f16 chain against R^T resident in shared memory; the
-//                      fp32 result in tensor memory is rounded, reduced and quantized by
-//                      sixteen epilogue warps, several tiles in flight.
+// The kernels, tried in this order:
+//   rq_tc_kernel       bf16/fp16, g in {16, 64, 256}, unit K stride, 16-byte aligned x and
+//                      R; rows of at most 128 groups (g = 256) or 128 64-channel group-rows
+//                      (g = 16 and 64; up to 256 in two parts).  Whole rows fill the 128 lanes
+//                      of a tcgen05.mma.kind::f16 chain against R^T resident in shared memory
+//                      (block-diagonal for g = 16: one MMA per 16-channel group); the fp32
+//                      result in tensor memory is rounded, reduced and quantized by sixteen
+//                      epilogue warps, several tiles in flight.
 //   rq_row_kernel      bf16/fp16, g in {16, 64}, rows that fit two buffers per warp.  Each warp
 //                      owns whole rows, filled by its own TMA copies, and rotates them with
 //                      mma.sync (y^T = R^T x^T) in place.

@@ -20,18 +20,26 @@
 //               owns one weight row (a TMEM lane) and one half of each k-block's K; it expands
 //               64 four-bit codes per k-block to bytes and writes them into the set's TMEM
 //               weight buffer with tcgen05.st
-//   warp 1      TMEM allocation and the single MMA-issuing thread: tcgen05.mma kind::i8 with
-//               A from TMEM, 128 x BNA x 32 per instruction.  Its waits, fences and commits
-//               cost far more than an MMA issue, so the ring is organised in super-stages of
-//               G k-blocks (G = 2-4): one wait for the codes, one for the weights and one
-//               commit per 4G MMAs
+//   warp 1      TMEM allocation and the MMAs: tcgen05.mma kind::i8 with A from TMEM, 128 x BNA
+//               x 32 per instruction.  The whole warp walks the ring and takes every wait (a
+//               vote makes each outcome uniform) and one elected lane issues; waits, fences
+//               and commits cost far more than an MMA issue, so the ring is organised in
+//               super-stages of G = 2 k-blocks: one wait for the codes, one for the weights and
+//               one commit per 8 MMAs
 //   warps 4-7, 24-27  epilogue, two warps per TMEM lane quarter taking alternate 16-row
-//               chunks: tcgen05.ld of the finished accumulator, fp32 scale/bias, and per output
-//               row one store of 32 consecutive channels per warp, overlapped with the MMAs of
-//               the next tile (two accumulators); the tile's row scales are loaded before its
-//               accumulator is ready
+//               chunks: tcgen05.ld of the finished accumulator, fp32 scale/bias, and 16-byte
+//               stores of 16 rows x 32 channels staged in shared memory, overlapped with the
+//               MMAs of the next tile (two accumulators); the tile's row scales are loaded
+//               before its accumulator is ready
 // TMEM columns: accumulators [0, BNA) and [BNA, 2 BNA), then nb (2-4) weight buffers of G
 // k-blocks (32 columns each).  Every role walks its ring indices incrementally.
+//
+// Launched after stage 1 inside the linear, the kernel is stage 1's programmatic dependent:
+// the weight producer and the unpack start at once, and the roles that read stage 1's output
+// (the code producers, the epilogue's row scales) or whose bounded waits would otherwise run
+// while stage 1 still does (the MMA warp, the unpack from its first wait on an MMA, the weight
+// producer from the super-stage whose slot needs such an unpack) first wait for stage 1 to
+// complete (griddepcontrol.wait; at once when the kernel was launched normally).
 //
 // Weight bytes.  For K < 2^21 each code w is written as the byte 16 w (its nibble moved to
 // the byte's high half: two logic operations per four codes instead of a sign extension);
