@@ -19,6 +19,8 @@ the workload (the path has no exchange step): weak scaling, max device time over
 rows spread over the host's cores by threads) on a bounded sample of the same workload.
 `--sweep` times stage 1 alone on the 72 rotate+quantize cases (M x K x g x dtype x layout)
 and prints one JSON object with a line per case (microseconds, GB/s, fraction of HBM).
+`--next` times the grouped linear, the W8A8 linear and the packed quantizer at the headline
+shape and prints one JSON object with a line per item.
 """
 from __future__ import annotations
 
@@ -687,6 +689,108 @@ def run_sweep(args, local):
             "cases": out}
 
 
+def run_next(args, local):
+    """The rows beyond the single linear, at the headline shape (M = 8192, K = 3840, g = 64,
+    bf16 activations), each timed like the sweep: launches cycle through copies of their data
+    totalling at least three times the L2, captured in one CUDA graph, events around the timed
+    replays only.
+      grouped linear    one stage 1 feeding three concatenated 3840-channel weights (Q, K, V),
+                        against three separate linears on the same activations;
+      W8A8 linear       INT8 codes and INT8 (N, K) weights: the whole linear, and the GEMM alone
+                        from codes against the INT8 peak;
+      packed quantizer  nibble-packed codes, round half to even and stochastic rounding, GB/s."""
+    from types import SimpleNamespace
+
+    from rotated_w4a4_quantized_group_b200 import ck
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pk, pk_kind = peaks()
+    int8_peak = pk["bf16_tflops"] * INT8_OVER_BF16
+    stream = torch.cuda.current_stream(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    case = W.LINEAR_CASES[W.HEADLINE]
+    M, K, g, Nq = case.M, case.K, case.g, case.N
+    inp = W.make_linear_inputs(case)
+    x_host, R = inp["x"].contiguous(), inp["R"].to(dev)
+    gen = torch.Generator().manual_seed(11)
+    bf = torch.bfloat16
+
+    def per_launch_ms(fn, sets):
+        graph = capture(lambda: [fn(st) for st in sets])
+        for _ in range(2):
+            graph.replay()
+        reps = max(1, -(-args.steps // len(sets)))
+        return timed_replays([graph], reps, stream) / (reps * len(sets))
+
+    items = []
+    # ---- grouped linear: Q, K and V of one activation tensor
+    N3 = 3 * Nq
+    wq = torch.randint(-128, 128, (N3, K // 2), dtype=torch.int8, generator=gen)
+    wsc = (torch.rand(N3, generator=gen) * 0.01).to(bf)
+    wsz = ck.workspace_bytes(M, N3, K, K // 2)
+    S = sets_for(M * K * 2 + N3 * K // 2 + M * N3 * 2 + wsz, 64)
+    sets = [SimpleNamespace(x=x_host.to(dev), w=wq.to(dev), ws=wsc.to(dev),
+                            outs=[torch.empty(M, Nq, dtype=bf, device=dev) for _ in range(3)],
+                            wsp=torch.empty(wsz, dtype=torch.uint8, device=dev)) for _ in range(S)]
+    t_grp = per_launch_ms(lambda st: ck.ck_w4a4_grouped_linear(
+        st.x, R, g, st.w, st.ws, None, [Nq] * 3, outs=st.outs, workspace=st.wsp,
+        dev_status=status), sets)
+    t_three = per_launch_ms(lambda st: [ck.ck_w4a4_linear(
+        st.x, R, g, st.w[i * Nq:(i + 1) * Nq], st.ws[i * Nq:(i + 1) * Nq], None, out=st.outs[i],
+        workspace=st.wsp, dev_status=status) for i in range(3)], sets)
+    ops = 2.0 * M * N3 * K
+    items.append({"item": "grouped_linear_qkv", "M": M, "K": K, "N": [Nq] * 3, "g": g,
+                  "us": t_grp * 1e3, "tops": ops / (t_grp * 1e-3) / 1e12,
+                  "three_linears_us": t_three * 1e3, "speedup_vs_three_linears": t_three / t_grp,
+                  "sets": S})
+    del sets
+    # ---- W8A8 linear
+    w8 = torch.randint(-128, 128, (Nq, K), dtype=torch.int8, generator=gen)
+    ws8 = (torch.rand(Nq, generator=gen) * 0.01).to(bf)
+    wsz8 = int(ck.lib().ck_w8a8_linear_workspace_bytes(M, Nq, K, K))
+    S = sets_for(M * K * 3 + Nq * K + M * Nq * 2 + wsz8, 64)
+    sets = [SimpleNamespace(x=x_host.to(dev), w=w8.to(dev), ws=ws8.to(dev),
+                            out=torch.empty(M, Nq, dtype=bf, device=dev),
+                            wsp=torch.empty(wsz8, dtype=torch.uint8, device=dev),
+                            q=torch.empty(M, K, dtype=torch.int8, device=dev),
+                            s=torch.empty(M, dtype=torch.float32, device=dev)) for _ in range(S)]
+    for st in sets:
+        ck.ck_rotate_quant_int8(st.x, R, g, codes=st.q, scales=st.s)
+    t_lin8 = per_launch_ms(lambda st: ck.ck_w8a8_linear(
+        st.x, R, g, st.w, st.ws, None, out=st.out, workspace=st.wsp, dev_status=status), sets)
+    t_gemm8 = per_launch_ms(lambda st: ck.ck_w8a8_linear(
+        st.q, None, 0, st.w, st.ws, None, a_scale=st.s, out=st.out, workspace=st.wsp,
+        dev_status=status), sets)
+    ops = 2.0 * M * Nq * K
+    items.append({"item": "w8a8_linear", "M": M, "K": K, "N": Nq, "g": g,
+                  "us": t_lin8 * 1e3, "tops": ops / (t_lin8 * 1e-3) / 1e12,
+                  "gemm_us": t_gemm8 * 1e3, "gemm_tops": ops / (t_gemm8 * 1e-3) / 1e12,
+                  "gemm_frac_of_int8_peak": ops / (t_gemm8 * 1e-3) / 1e12 / int8_peak, "sets": S})
+    del sets
+    # ---- packed quantizer
+    nbytes = M * K * 2 + M * K // 2 + 4 * M + g * g * 2
+    S = sets_for(nbytes, 4096)
+    sets = [SimpleNamespace(x=x_host.to(dev), p=torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
+                            s=torch.empty(M, dtype=torch.float32, device=dev)) for _ in range(S)]
+    for stoch in (False, True):
+        t = per_launch_ms(lambda st: ck.ck_rotate_quant_packed(
+            st.x, R, g, stochastic=stoch, seed=1234, packed=st.p, scales=st.s), sets)
+        gbs = nbytes / (t * 1e-3) / 1e9
+        items.append({"item": "packed_quantizer_" + ("stochastic" if stoch else "nearest"),
+                      "M": M, "K": K, "g": g, "us": t * 1e3, "algorithmic_bytes": nbytes,
+                      "gbs": gbs, "frac_hbm": gbs / pk["hbm_gbs"], "sets": S})
+    del sets
+    torch.cuda.synchronize()
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()}")
+    return {"next": "grouped linear, W8A8 linear and packed quantizer at the headline shape",
+            "int8_peak_tops": int8_peak, "hbm_peak_gbs": pk["hbm_gbs"], "peak_source": pk_kind,
+            "l2": "launches cycle through copies of their data totalling >= 3 x the 126 MB L2, "
+                  "replayed from a CUDA graph; events around the timed replays only",
+            "items": items}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -699,6 +803,7 @@ def main():
     ap.add_argument("--clock-soak-s", type=float, default=1.0)
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--sweep-filter", default="")
+    ap.add_argument("--next", action="store_true")
     args = ap.parse_args()
     case = W.LINEAR_CASES[args.workload]
 
@@ -714,6 +819,10 @@ def main():
         if args.sweep:
             if rank == 0:
                 print(json.dumps(run_sweep(args, local)), flush=True)
+            return
+        if args.next:
+            if rank == 0:
+                print(json.dumps(run_next(args, local)), flush=True)
             return
         res = run_ck(args, case, world, rank, local)
         if res is not None:

@@ -119,6 +119,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// ------------------------------------------------------------------ Philox4x32-10
+
+// Philox4x32-10 is the counter-based generator of Salmon, Moraes, Dror and Shaw ("Parallel
+// random numbers: as easy as 1, 2, 3", SC 2011): ten rounds of two 32 x 32 -> 64-bit products
+// mixed with the key, the key bumped by two Weyl constants between rounds.
+// Word 0 of Philox4x32-10 of a 128-bit counter under a 64-bit key.
+__device__ __forceinline__ uint32_t philox_word0(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                                 uint32_t k0, uint32_t k1) {
+#pragma unroll
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
+        const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
+        const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+        c0 = n0;
+        c1 = lo1;
+        c2 = n2;
+        c3 = lo0;
+    }
+    return c0;
+}
+
 // ------------------------------------------------------------------ dependent launches
 
 // Programmatic dependent launch.  A kernel launched with programmatic stream serialization may

@@ -834,6 +834,7 @@ struct RqTcParams {
     uint32_t idesc;
     int vec_codes;
     int qmax;          // code grid [-qmax - 1, qmax]
+    uint64_t seed, offset;   // packed stochastic output: the Philox key and counter offset
 };
 
 template <typename T, bool DYN>
@@ -863,6 +864,73 @@ __device__ __forceinline__ void tc_quant_store(const uint32_t (&yp)[8], const Ro
     }
 }
 
+// Sixteen codes of one row packed two to a byte (even channel in the low nibble), 8 bytes at
+// dst.  PK = 1: rounded half to even, the codes tc_quant_store writes.  PK = 2: stochastic,
+// q = clamp(floor(fl(t + u)), -8, 7) with t = fl(y / s) and u = (r >> 8) 2^-24, r word 0 of
+// Philox4x32-10 at counter (e, offset) under key seed, e = row K + channel (e0 the first
+// channel's); a NaN t gives 0.
+template <typename T, bool DYN, int PK>
+__device__ __forceinline__ void tc_packed_store(const uint32_t (&yp)[8], const RowDivisor& dv,
+                                                uint8_t* dst, bool vec, uint64_t e0,
+                                                uint64_t seed, uint64_t offset) {
+    uint32_t out[4];   // sixteen codes, four a word, first code lowest
+    if constexpr (PK == 1) {
+        if (DYN) {
+            unsigned long long y2[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) y2[k] = MmaOp<T>::unpack2(yp[k]);
+            quant16_dyn2(y2, dv, out);
+        } else {
+            float y[16];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float2 a = MmaOp<T>::unpack(yp[k]);
+                y[2 * k] = a.x;
+                y[2 * k + 1] = a.y;
+            }
+            quant16(y, dv, out);
+        }
+    } else {
+        const uint32_t k0s = (uint32_t)seed, k1s = (uint32_t)(seed >> 32);
+        const uint32_t o0 = (uint32_t)offset, o1 = (uint32_t)(offset >> 32);
+        int q[16];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float2 a = MmaOp<T>::unpack(yp[k]);
+            const float y[2] = {a.x, a.y};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float t = dv.fast ? quotient_fast(y[e], dv.s, dv.r) : __fdiv_rn(y[e], dv.s);
+                const uint64_t el = e0 + (uint64_t)(2 * k + e);
+                const uint32_t rnd = philox_word0((uint32_t)el, (uint32_t)(el >> 32), o0, o1, k0s, k1s);
+                const float u = __uint2float_rn(rnd >> 8) * 0x1p-24f;   // exact
+                float v = floorf(__fadd_rn(t, u));
+                v = fminf(fmaxf(v, -8.0f), 7.0f);
+                q[2 * k + e] = t != t ? 0 : (int)v;
+            }
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w) out[w] = pack4_codes(q[4 * w], q[4 * w + 1], q[4 * w + 2], q[4 * w + 3]);
+    }
+    // four byte codes c0 .. c3 of a word -> the two bytes (c0 & 15) | c1 << 4, (c2 & 15) | c3 << 4
+    uint32_t h[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const uint32_t n = out[w] & 0x0F0F0F0Fu;
+        h[w] = __byte_perm(n | (n >> 4), 0u, 0x4420);   // bytes 0 and 2, upper half zero
+    }
+    const uint32_t lo = h[0] | (h[1] << 16), hi = h[2] | (h[3] << 16);
+    if (vec) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            dst[k] = (uint8_t)(lo >> (8 * k));
+            dst[4 + k] = (uint8_t)(hi >> (8 * k));
+        }
+    }
+}
+
 // RG = G: R is the g x g rotation.  RG = 16 < G = 64: rows of g = 16 groups viewed as 64-channel
 // group-rows; each of the four 16-channel groups is its own MMA (M = 128, N = 16, K = 16) of
 // the group's 16 channels against R^T, into its own 16 accumulator columns, so no group sees
@@ -873,12 +941,15 @@ __device__ __forceinline__ void tc_quant_store(const uint32_t (&yp)[8], const Ro
 // 64-column block a of the tile's accumulator (D[l, 64 a + c] for group-row a L + l), so a
 // group's accumulator has 128 columns; the epilogue reads both blocks twice (row absmax, then
 // the codes).
-template <typename T, int G, bool DYN, int RG = G, int P = 1>
+// PK = 0: INT8 codes; PK = 1, 2: codes packed two to a byte at `codes` (row pitch ldq bytes),
+// rounded half to even (1) or stochastically (2) (tc_packed_store).
+template <typename T, int G, bool DYN, int RG = G, int P = 1, int PK = 0>
 __global__ void __launch_bounds__(kTcThreads, 1)
     rq_tc_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ R,
                  const float* __restrict__ scale_in, int8_t* __restrict__ codes,
                  float* __restrict__ scales, RqTcParams p, int* dev_status) {
     static_assert(P == 1 || G == 64, "split rows only at G = 64");
+    static_assert(PK == 0 || (P == 1 && G == 64), "packed codes from the 64-column epilogue only");
     constexpr int kAcc = kTcAcc<G>, kStages = kTcXStages<G>, kAtoms = P > 1 ? P : G / 64;
     constexpr int kAccCols = G * P;                 // TMEM columns of one accumulator
     constexpr int kGrpWarps = kTcEpiWarps / kAcc;   // 4 or 8
@@ -1190,7 +1261,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const RowDivisor dv(sc, p.qmax);
             if (row_ok && rho == 0 && h == 0) scales[row] = sc;
             int8_t* dst = codes + row * p.ldq + rho * G + h * kCols;
-            if constexpr (kCols == 64) {
+            if constexpr (kCols == 64 && PK != 0) {
+                if (row_ok) {
+                    // channels rho G .. rho G + 63 of the row: 32 bytes of packed codes
+                    uint8_t* pdst = reinterpret_cast<uint8_t*>(codes) + row * p.ldq + rho * (G / 2);
+                    const uint64_t e0 = (uint64_t)row * (uint64_t)p.K + (uint64_t)(rho * G);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        tc_packed_store<T, DYN, PK>(*reinterpret_cast<const uint32_t(*)[8]>(&yp[8 * u]),
+                                                    dv, pdst + 8 * u, p.vec_codes != 0,
+                                                    e0 + (uint64_t)(16 * u), p.seed, p.offset);
+                }
+            } else if constexpr (kCols == 64) {
                 if (row_ok) {
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
@@ -1233,12 +1315,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 // Tensor-core kernel for bf16/fp16, g in {64, 256}, K / g <= 128 (P = 1), or g = 64 rows of
 // 129 .. 128 P groups split in P parts.  Returns CK_ERR_UNSUPPORTED otherwise.
-template <typename T, int G, int RG = G, int P = 1>
+template <typename T, int G, int RG = G, int P = 1, int PK = 0>
 static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, const void* R,
                            const float* scale_in, int8_t* codes, int64_t ldq, float* scales,
                            int qmax, int* dev_status, cudaStream_t stream,
-                           CUtensorMapDataType tdt) {
+                           CUtensorMapDataType tdt, uint64_t seed = 0, uint64_t offset = 0) {
     RqTcParams p;
+    p.seed = seed;
+    p.offset = offset;
     p.M = M;
     p.K = K;
     p.ldq = ldq;
@@ -1252,7 +1336,9 @@ static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, cons
     p.tiles = (int)tiles;
     p.box_bytes = (uint32_t)(p.RB * p.L * 128);
     p.idesc = idesc_f16(128, G, std::is_same<T, __nv_bfloat16>::value);
-    p.vec_codes = (aligned(codes, 16) && ldq % 16 == 0) ? 1 : 0;
+    // 16-byte code stores, or 8-byte packed stores
+    p.vec_codes = PK == 0 ? ((aligned(codes, 16) && ldq % 16 == 0) ? 1 : 0)
+                          : ((aligned(codes, 8) && ldq % 8 == 0) ? 1 : 0);
     p.qmax = qmax;
 
     // x as (channel within group, group, row); each box is 64 channels (128 bytes) of every
@@ -1274,7 +1360,38 @@ static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, cons
                                                  scales, p, dev_status);
         return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
     };
-    return scale_in ? run(rq_tc_kernel<T, G, false, RG, P>) : run(rq_tc_kernel<T, G, true, RG, P>);
+    return scale_in ? run(rq_tc_kernel<T, G, false, RG, P, PK>)
+                    : run(rq_tc_kernel<T, G, true, RG, P, PK>);
+}
+
+// The packed quantizer on the tensor-core kernel: bf16/fp16 rows of unit stride with g = 16 or
+// 64 and at most 128 64-channel group-rows; CK_ERR_UNSUPPORTED otherwise.
+ck_status launch_rotate_quant_packed_tc(const void* x, ck_dtype dt, int64_t M, int64_t K,
+                                        int64_t sm, int64_t sk, const void* R, int g,
+                                        const float* scale_in, bool stochastic, uint64_t seed,
+                                        uint64_t offset, uint8_t* packed, int64_t ldp,
+                                        float* scales, cudaStream_t stream) {
+    const bool half16 = dt == CK_BF16 || dt == CK_F16;
+    if (!half16 || (g != 16 && g != 64) || sk != 1 || !aligned(x, 16) || !aligned(R, 16) ||
+        sm % 8 != 0 || sm <= 0 || K % 64 != 0 || K / 64 > 128 || M >= (1LL << 31))
+        return CK_ERR_UNSUPPORTED;
+    const bool bf = dt == CK_BF16;
+    const CUtensorMapDataType tdt = bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    int8_t* out = reinterpret_cast<int8_t*>(packed);
+#define CK_RQP_ARGS x, M, K, sm, R, scale_in, out, ldp, scales, 7, nullptr, stream, tdt, seed, offset
+    if (g == 64) {
+        if (bf)
+            return stochastic ? launch_tc<__nv_bfloat16, 64, 64, 1, 2>(CK_RQP_ARGS)
+                              : launch_tc<__nv_bfloat16, 64, 64, 1, 1>(CK_RQP_ARGS);
+        return stochastic ? launch_tc<__half, 64, 64, 1, 2>(CK_RQP_ARGS)
+                          : launch_tc<__half, 64, 64, 1, 1>(CK_RQP_ARGS);
+    }
+    if (bf)
+        return stochastic ? launch_tc<__nv_bfloat16, 64, 16, 1, 2>(CK_RQP_ARGS)
+                          : launch_tc<__nv_bfloat16, 64, 16, 1, 1>(CK_RQP_ARGS);
+    return stochastic ? launch_tc<__half, 64, 16, 1, 2>(CK_RQP_ARGS)
+                      : launch_tc<__half, 64, 16, 1, 1>(CK_RQP_ARGS);
+#undef CK_RQP_ARGS
 }
 
 // ===================================================================== host launch

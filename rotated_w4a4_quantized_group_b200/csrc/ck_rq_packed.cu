@@ -16,7 +16,9 @@
 // random numbers: as easy as 1, 2, 3", SC 2011): ten rounds of two 32 x 32 -> 64-bit products
 // mixed with the key, the key bumped by two Weyl constants between rounds.
 //
-// One row per CTA step (grid-stride over rows): the row is read once into shared memory
+// 16-bit rows of g = 16 or 64 and at most 128 64-channel group-rows go to the tensor-core
+// stage-1 kernel with a packed epilogue (ck_rotate_quant.cu).  Every other row here: one row
+// per CTA step (grid-stride over rows): the row is read once into shared memory
 // (any strides), each thread rotates 4-channel chunks with fp32 FMAs against R in shared
 // memory and rounds them to the dtype, the row absmax is reduced through shared memory, and a
 // second pass rotates again, quantizes and stores 2 bytes per chunk.
@@ -32,26 +34,6 @@ namespace ck {
 
 namespace rqp {
 constexpr int kThreads = 256;
-}
-
-// Word 0 of Philox4x32-10 of a 128-bit counter under a 64-bit key.
-__device__ __forceinline__ uint32_t philox_word0(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
-                                                 uint32_t k0, uint32_t k1) {
-#pragma unroll
-    for (int round = 0; round < 10; ++round) {
-        if (round > 0) {
-            k0 += 0x9E3779B9u;
-            k1 += 0xBB67AE85u;
-        }
-        const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
-        const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
-        const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
-        c0 = n0;
-        c1 = lo1;
-        c2 = n2;
-        c3 = lo0;
-    }
-    return c0;
 }
 
 template <typename T>
@@ -192,6 +174,11 @@ ck_status launch_rotate_quant_packed(const void* x, ck_dtype dt, int64_t M, int6
                                      uint8_t* packed, int64_t ldp, float* scales,
                                      cudaStream_t stream) {
     if (M == 0) return CK_OK;
+    // 16-bit rows of g = 16 or 64 and at most 128 64-channel group-rows: the tensor-core kernel
+    const ck_status st = launch_rotate_quant_packed_tc(x, dt, M, K, sm, sk, R, g, scale_in,
+                                                       stochastic, seed, offset, packed, ldp,
+                                                       scales, stream);
+    if (st != CK_ERR_UNSUPPORTED) return st;
     switch (dt) {
         case CK_F32:
             return launch_packed_typed<float>(x, M, K, sm, sk, R, g, scale_in, stochastic, seed,

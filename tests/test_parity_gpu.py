@@ -904,6 +904,25 @@ def test_packed_quantizer_nearest_matches_stage1_codes():
     np.testing.assert_array_equal(_unpack_codes(packed.cpu().numpy()), codes.cpu().numpy())
 
 
+@pytest.mark.parametrize("dt,g,M,K,pitch", [("bf16", 64, 1000, 3840, 0), ("f16", 16, 333, 1024, 0),
+                                             ("bf16", 16, 8192, 3840, 0), ("f16", 64, 129, 8192, 3)])
+def test_packed_quantizer_nearest_equals_stage1_codes_on_tensor_cores(dt, g, M, K, pitch):
+    """16-bit rows of g = 16 or 64 and at most 128 64-channel groups take the tensor-core
+    stage-1 kernel with a packed epilogue: with round half to even its codes are stage 1's
+    codes for any R, bit for bit, and the scales are equal.  A Haar R, several rows per tile
+    and split tiles, an output pitch that is not a multiple of 8 bytes (byte stores)."""
+    x = torch.randn(M, K, generator=torch.Generator().manual_seed(M + K)).to(DT[dt]).cuda()
+    R = W.haar_orthogonal(g, torch.Generator().manual_seed(g)).to(DT[dt]).contiguous().cuda()
+    buf = torch.zeros(M, K // 2 + pitch, dtype=torch.uint8, device="cuda")
+    packed, s1 = ck.ck_rotate_quant_packed(x, R, g, packed=buf[:, : K // 2])
+    codes, s2 = ck.ck_rotate_quant(x, R, g)
+    torch.cuda.synchronize()
+    assert torch.equal(s1, s2)
+    np.testing.assert_array_equal(_unpack_codes(packed.cpu().numpy()), codes.cpu().numpy())
+    if pitch:
+        assert int(buf[:, K // 2:].abs().sum()) == 0   # nothing written past each row
+
+
 @pytest.mark.parametrize("dt,g", [("bf16", 64), ("f16", 256), ("f32", 16)])
 def test_packed_quantizer_stochastic_general_rotation(dt, g):
     """A general R: y may differ from the oracle's by its accumulation's rounding, so a code may
