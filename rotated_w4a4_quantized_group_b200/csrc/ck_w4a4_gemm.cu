@@ -25,7 +25,7 @@
 //               vote makes each outcome uniform) and one elected lane issues; waits, fences
 //               and commits cost far more than an MMA issue, so the ring is organised in
 //               super-stages of G = 2 k-blocks: one wait for the codes, one for the weights and
-//               one commit per 8 MMAs
+//               one commit per 8 MMAs (INT8 weights, W8: G = 1, for a deeper shared-memory ring)
 //   warps 4-7, 24-27  epilogue, two warps per TMEM lane quarter taking alternate 16-row
 //               chunks: tcgen05.ld of the finished accumulator, fp32 scale/bias, and 16-byte
 //               stores of 16 rows x 32 channels staged in shared memory, overlapped with the
@@ -586,14 +586,16 @@ static ck_status launch_persistent(const int8_t* codes, int64_t ldq, const float
     const int sms = num_sms();
     GemmParams p;
     p.BNA = choose_bna(M, N, sms);
-    const bool box3d = K % BK == 0;
+    const bool box3d = !w8 && K % BK == 0;
     const int num_kb = (int)((K + BK - 1) / BK);
     // weight bytes per row of one k-block: 64 packed (two codes a byte) or 128
     const uint32_t wkb = w8 ? BK : BK / 2;
     const CUtensorMapSwizzle wsw = w8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap xmap, wmap;
-    // with whole 128-byte k-blocks, one 3-D box fetches the G k-blocks of a super-stage:
-    // (byte of the k-block, row, k-block); otherwise one 2-D box per k-block, zero past K
+    // packed weights with whole 128-byte k-blocks: one 3-D box fetches the G = 2 k-blocks of a
+    // super-stage, (byte of the k-block, row, k-block); otherwise one 2-D box per k-block, zero
+    // past K.  INT8 weights (W8) take super-stages of one k-block: a ring slot then holds 40 KB
+    // (codes and weights) instead of 80, five slots instead of two.
     const uint32_t G_box = 2;
     {
         // codes: one 2-D box (128 bytes x BNA rows) per k-block, zero past K and M
@@ -630,7 +632,7 @@ static ck_status launch_persistent(const int8_t* codes, int64_t ldq, const float
     // TMEM: two accumulators of BNA columns; for packed weights the rest holds the weight
     // buffers of G k-blocks (32 columns each), as many as fit (2..4): the unpack of a
     // super-stage may start once the MMAs of the super-stage nb before it completed
-    p.G = (int)G_box;   // the 3-D boxes above hold exactly one super-stage
+    p.G = w8 ? 1 : (int)G_box;   // the 3-D boxes above hold exactly one super-stage
     p.nb = w8 ? 2 : (int)((TMEM_COLS - 2u * (uint32_t)p.BNA) / ((uint32_t)p.G * A_STAGE_COLS));
     if (p.nb > NB_MAX) p.nb = NB_MAX;
     if (p.nb < 2) return CK_ERR_UNSUPPORTED;
