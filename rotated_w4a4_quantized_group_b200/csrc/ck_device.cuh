@@ -144,6 +144,43 @@ __device__ __forceinline__ uint32_t philox_word0(uint32_t c0, uint32_t c1, uint3
     return c0;
 }
 
+// philox_word0 for a run of counters (e, e >> 32, o0, o1) that differ only in e: the ten round
+// keys and the first round's product of the fixed third word o0 are computed once per run.
+struct PhiloxRun {
+    uint32_t k0[10], k1[10];
+    uint32_t lo_o0, hi_o0;   // 0xCD9E8D57 o0: its low and high words
+    uint32_t o1;
+    __device__ __forceinline__ PhiloxRun(uint64_t seed, uint64_t offset) {
+        uint32_t a = (uint32_t)seed, b = (uint32_t)(seed >> 32);
+#pragma unroll
+        for (int r = 0; r < 10; ++r) {
+            k0[r] = a;
+            k1[r] = b;
+            a += 0x9E3779B9u;
+            b += 0xBB67AE85u;
+        }
+        lo_o0 = 0xCD9E8D57u * (uint32_t)offset;
+        hi_o0 = __umulhi(0xCD9E8D57u, (uint32_t)offset);
+        o1 = (uint32_t)(offset >> 32);
+    }
+    __device__ __forceinline__ uint32_t word0(uint64_t e) const {
+        uint32_t c0 = (uint32_t)e;
+        const uint32_t lo = 0xD2511F53u * c0, hi = __umulhi(0xD2511F53u, c0);
+        c0 = hi_o0 ^ (uint32_t)(e >> 32) ^ k0[0];
+        uint32_t c1 = lo_o0, c2 = hi ^ o1 ^ k1[0], c3 = lo;
+#pragma unroll
+        for (int r = 1; r < 10; ++r) {
+            const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
+            const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
+            c0 = hi1 ^ c1 ^ k0[r];
+            c2 = hi0 ^ c3 ^ k1[r];
+            c1 = lo1;
+            c3 = lo0;
+        }
+        return c0;
+    }
+};
+
 // ------------------------------------------------------------------ dependent launches
 
 // Programmatic dependent launch.  A kernel launched with programmatic stream serialization may

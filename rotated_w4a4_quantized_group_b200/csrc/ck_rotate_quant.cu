@@ -891,8 +891,7 @@ __device__ __forceinline__ void tc_packed_store(const uint32_t (&yp)[8], const R
             quant16(y, dv, out);
         }
     } else {
-        const uint32_t k0s = (uint32_t)seed, k1s = (uint32_t)(seed >> 32);
-        const uint32_t o0 = (uint32_t)offset, o1 = (uint32_t)(offset >> 32);
+        const PhiloxRun ph(seed, offset);
         int q[16];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -902,7 +901,7 @@ __device__ __forceinline__ void tc_packed_store(const uint32_t (&yp)[8], const R
             for (int e = 0; e < 2; ++e) {
                 const float t = dv.fast ? quotient_fast(y[e], dv.s, dv.r) : __fdiv_rn(y[e], dv.s);
                 const uint64_t el = e0 + (uint64_t)(2 * k + e);
-                const uint32_t rnd = philox_word0((uint32_t)el, (uint32_t)(el >> 32), o0, o1, k0s, k1s);
+                const uint32_t rnd = ph.word0(el);
                 const float u = __uint2float_rn(rnd >> 8) * 0x1p-24f;   // exact
                 float v = floorf(__fadd_rn(t, u));
                 v = fminf(fmaxf(v, -8.0f), 7.0f);
@@ -1266,11 +1265,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     // channels rho G .. rho G + 63 of the row: 32 bytes of packed codes
                     uint8_t* pdst = reinterpret_cast<uint8_t*>(codes) + row * p.ldq + rho * (G / 2);
                     const uint64_t e0 = (uint64_t)row * (uint64_t)p.K + (uint64_t)(rho * G);
+                    if constexpr (PK == 1) {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        tc_packed_store<T, DYN, PK>(*reinterpret_cast<const uint32_t(*)[8]>(&yp[8 * u]),
-                                                    dv, pdst + 8 * u, p.vec_codes != 0,
-                                                    e0 + (uint64_t)(16 * u), p.seed, p.offset);
+                        for (int u = 0; u < 4; ++u)
+                            tc_packed_store<T, DYN, PK>(*reinterpret_cast<const uint32_t(*)[8]>(&yp[8 * u]),
+                                                        dv, pdst + 8 * u, p.vec_codes != 0,
+                                                        e0 + (uint64_t)(16 * u), p.seed, p.offset);
+                    } else {
+                        // one run of 16 draws at a time: unrolled, the four runs' Philox chains
+                        // spill (216 us against 147 at the headline shape)
+#pragma unroll 1
+                        for (int u = 0; u < 4; ++u)
+                            tc_packed_store<T, DYN, PK>(*reinterpret_cast<const uint32_t(*)[8]>(&yp[8 * u]),
+                                                        dv, pdst + 8 * u, p.vec_codes != 0,
+                                                        e0 + (uint64_t)(16 * u), p.seed, p.offset);
+                    }
                 }
             } else if constexpr (kCols == 64) {
                 if (row_ok) {
