@@ -108,8 +108,9 @@ size_t linear_scratch_need(const void* x, ck_dtype x_dtype, int64_t M, int64_t K
                            bool w8 = false);
 
 // The public packed quantizer (ck_rq_packed.cu), arguments already validated.
-// The packed quantizer on the tensor-core stage-1 kernel (ck_rotate_quant.cu): bf16/fp16, g = 16
-// or 64, unit K stride, at most 128 64-channel group-rows; CK_ERR_UNSUPPORTED otherwise.
+// The packed quantizer on the tensor-core stage-1 kernel (ck_rotate_quant.cu): bf16/fp16, unit K
+// stride, g = 16 or 64 with at most 128 64-channel group-rows, or g = 256 with at most 128
+// groups; CK_ERR_UNSUPPORTED otherwise.
 ck_status launch_rotate_quant_packed_tc(const void* x, ck_dtype dt, int64_t M, int64_t K,
                                         int64_t sm, int64_t sk, const void* R, int g,
                                         const float* scale_in, bool stochastic, uint64_t seed,

@@ -948,7 +948,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                  const float* __restrict__ scale_in, int8_t* __restrict__ codes,
                  float* __restrict__ scales, RqTcParams p, int* dev_status) {
     static_assert(P == 1 || G == 64, "split rows only at G = 64");
-    static_assert(PK == 0 || (P == 1 && G == 64), "packed codes from the 64-column epilogue only");
+    static_assert(PK == 0 || (P == 1 && (G == 64 || G == 256)), "packed codes: one-part tiles");
     constexpr int kAcc = kTcAcc<G>, kStages = kTcXStages<G>, kAtoms = P > 1 ? P : G / 64;
     constexpr int kAccCols = G * P;                 // TMEM columns of one accumulator
     constexpr int kGrpWarps = kTcEpiWarps / kAcc;   // 4 or 8
@@ -1295,6 +1295,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tc_ld_32x32b_x32(tacc + (uint32_t)c, v);
                     tc_wait_ld();
                     if (row_ok) {
+                        // packed codes: channel k0 of this chunk is byte k0 / 2 of the row
+                        const int k0 = rho * G + h * kCols + c;
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
                             uint32_t y8[8];
@@ -1302,8 +1304,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             for (int k = 0; k < 8; ++k)
                                 y8[k] = MmaOp<T>::pack(__uint_as_float(v[16 * u + 2 * k]),
                                                        __uint_as_float(v[16 * u + 2 * k + 1]));
-                            tc_quant_store<T, DYN>(y8, dv, scale_in, dst + c + 16 * u,
-                                                   p.vec_codes != 0);
+                            if constexpr (PK != 0)
+                                tc_packed_store<T, DYN, PK>(
+                                    y8, dv, reinterpret_cast<uint8_t*>(codes) + row * p.ldq + k0 / 2 + 8 * u,
+                                    p.vec_codes != 0, (uint64_t)row * (uint64_t)p.K + (uint64_t)(k0 + 16 * u),
+                                    p.seed, p.offset);
+                            else
+                                tc_quant_store<T, DYN>(y8, dv, scale_in, dst + c + 16 * u,
+                                                       p.vec_codes != 0);
                         }
                     }
                 }
@@ -1374,20 +1382,29 @@ static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, cons
 }
 
 // The packed quantizer on the tensor-core kernel: bf16/fp16 rows of unit stride with g = 16 or
-// 64 and at most 128 64-channel group-rows; CK_ERR_UNSUPPORTED otherwise.
+// 64 and at most 128 64-channel group-rows, or g = 256 and at most 128 groups;
+// CK_ERR_UNSUPPORTED otherwise.
 ck_status launch_rotate_quant_packed_tc(const void* x, ck_dtype dt, int64_t M, int64_t K,
                                         int64_t sm, int64_t sk, const void* R, int g,
                                         const float* scale_in, bool stochastic, uint64_t seed,
                                         uint64_t offset, uint8_t* packed, int64_t ldp,
                                         float* scales, cudaStream_t stream) {
     const bool half16 = dt == CK_BF16 || dt == CK_F16;
-    if (!half16 || (g != 16 && g != 64) || sk != 1 || !aligned(x, 16) || !aligned(R, 16) ||
-        sm % 8 != 0 || sm <= 0 || K % 64 != 0 || K / 64 > 128 || M >= (1LL << 31))
+    if (!half16 || (g != 16 && g != 64 && g != 256) || sk != 1 || !aligned(x, 16) ||
+        !aligned(R, 16) || sm % 8 != 0 || sm <= 0 || K % 64 != 0 || K / 64 > 128 ||
+        (g == 256 && (K % 256 != 0 || K / 256 > 128)) || M >= (1LL << 31))
         return CK_ERR_UNSUPPORTED;
     const bool bf = dt == CK_BF16;
     const CUtensorMapDataType tdt = bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     int8_t* out = reinterpret_cast<int8_t*>(packed);
 #define CK_RQP_ARGS x, M, K, sm, R, scale_in, out, ldp, scales, 7, nullptr, stream, tdt, seed, offset
+    if (g == 256) {
+        if (bf)
+            return stochastic ? launch_tc<__nv_bfloat16, 256, 256, 1, 2>(CK_RQP_ARGS)
+                              : launch_tc<__nv_bfloat16, 256, 256, 1, 1>(CK_RQP_ARGS);
+        return stochastic ? launch_tc<__half, 256, 256, 1, 2>(CK_RQP_ARGS)
+                          : launch_tc<__half, 256, 256, 1, 1>(CK_RQP_ARGS);
+    }
     if (g == 64) {
         if (bf)
             return stochastic ? launch_tc<__nv_bfloat16, 64, 64, 1, 2>(CK_RQP_ARGS)

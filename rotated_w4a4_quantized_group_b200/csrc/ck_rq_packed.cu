@@ -16,9 +16,10 @@
 // random numbers: as easy as 1, 2, 3", SC 2011): ten rounds of two 32 x 32 -> 64-bit products
 // mixed with the key, the key bumped by two Weyl constants between rounds.
 //
-// 16-bit rows of g = 16 or 64 and at most 128 64-channel group-rows go to the tensor-core
-// stage-1 kernel with a packed epilogue (ck_rotate_quant.cu).  Every other row here: one row
-// per CTA step (grid-stride over rows): the row is read once into shared memory
+// 16-bit rows of g = 16 or 64 and at most 128 64-channel group-rows, or of g = 256 and at most
+// 128 groups, go to the tensor-core stage-1 kernel with a packed epilogue (ck_rotate_quant.cu).
+// Every other row here: one row per CTA step (grid-stride over rows): the row is read once into
+// shared memory
 // (any strides), each thread rotates 4-channel chunks with fp32 FMAs against R in shared
 // memory and rounds them to the dtype, the row absmax is reduced through shared memory, and a
 // second pass rotates again, quantizes and stores 2 bytes per chunk.
@@ -174,7 +175,8 @@ ck_status launch_rotate_quant_packed(const void* x, ck_dtype dt, int64_t M, int6
                                      uint8_t* packed, int64_t ldp, float* scales,
                                      cudaStream_t stream) {
     if (M == 0) return CK_OK;
-    // 16-bit rows of g = 16 or 64 and at most 128 64-channel group-rows: the tensor-core kernel
+    // 16-bit rows of g = 16, 64 (at most 128 64-channel group-rows) or 256 (at most 128 groups):
+    // the tensor-core kernel
     const ck_status st = launch_rotate_quant_packed_tc(x, dt, M, K, sm, sk, R, g, scale_in,
                                                        stochastic, seed, offset, packed, ldp,
                                                        scales, stream);

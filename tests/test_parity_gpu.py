@@ -905,10 +905,11 @@ def test_packed_quantizer_nearest_matches_stage1_codes():
 
 
 @pytest.mark.parametrize("dt,g,M,K,pitch", [("bf16", 64, 1000, 3840, 0), ("f16", 16, 333, 1024, 0),
-                                             ("bf16", 16, 8192, 3840, 0), ("f16", 64, 129, 8192, 3)])
+                                             ("bf16", 16, 8192, 3840, 0), ("f16", 64, 129, 8192, 3),
+                                             ("bf16", 256, 700, 3840, 0), ("f16", 256, 65, 10240, 5)])
 def test_packed_quantizer_nearest_equals_stage1_codes_on_tensor_cores(dt, g, M, K, pitch):
-    """16-bit rows of g = 16 or 64 and at most 128 64-channel groups take the tensor-core
-    stage-1 kernel with a packed epilogue: with round half to even its codes are stage 1's
+    """16-bit rows of g = 16 or 64 and at most 128 64-channel groups, or g = 256 and at most 128
+    groups, take the tensor-core stage-1 kernel with a packed epilogue: with round half to even its codes are stage 1's
     codes for any R, bit for bit, and the scales are equal.  A Haar R, several rows per tile
     and split tiles, an output pitch that is not a multiple of 8 bytes (byte stores)."""
     x = torch.randn(M, K, generator=torch.Generator().manual_seed(M + K)).to(DT[dt]).cuda()
