@@ -835,6 +835,7 @@ struct RqTcParams {
     int vec_codes;
     int qmax;          // code grid [-qmax - 1, qmax]
     uint64_t seed, offset;   // packed stochastic output: the Philox key and counter offset
+    int dependent;           // launched as the programmatic dependent of the kernel before it
 };
 
 template <typename T, bool DYN>
@@ -994,10 +995,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&xmap);
-        // the first ring's worth of boxes goes out while the CTA stages R^T
-        for (int n = 0; n < kStages && n < my_boxes; ++n) issue(n);
+        // the first ring's worth of boxes goes out at once (while the CTA stages R^T) unless
+        // the kernel must first wait for the one before it
+        if (!p.dependent)
+            for (int n = 0; n < kStages && n < my_boxes; ++n) issue(n);
     }
     for (int i = tid; i < kAcc * kTcSlots * 128; i += kTcThreads) (&amax_sh[0][0][0])[i] = 0u;
+    if (p.dependent) {
+        // launched as the programmatic dependent of the kernel before it on the stream: what
+        // is above is on-chip set-up; x and R may be that kernel's output, and the codes and
+        // scales its input, so no global memory is touched before it has completed
+        grid_dependency_wait();
+        if (tid == 0)
+            for (int n = 0; n < kStages && n < my_boxes; ++n) issue(n);
+    }
     // R^T[n][k] = R[k][n] is the MMA's B operand (N = c), staged in 8 x 8 blocks: a thread
     // loads rows k0 .. k0 + 7 of R at columns n0 .. n0 + 7 (16 bytes each), transposes them in
     // registers and stores the 16-byte chunks of rows n0 .. n0 + 7 of R^T.  Consecutive
@@ -1340,6 +1351,7 @@ static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, cons
     RqTcParams p;
     p.seed = seed;
     p.offset = offset;
+    p.dependent = M <= 64 ? 1 : 0;   // see the launch below
     p.M = M;
     p.K = K;
     p.ldq = ldq;
@@ -1373,8 +1385,23 @@ static ck_status launch_tc(const void* x, int64_t M, int64_t K, int64_t sm, cons
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
             return CK_ERR_CUDA;
-        kern<<<grid, kTcThreads, smem, stream>>>(map, static_cast<const T*>(R), scale_in, codes,
-                                                 scales, p, dev_status);
+        // few rows (M <= 64): the programmatic dependent of the kernel before it (the kernel
+        // waits for it before touching global memory), so that its CTAs set up on the SMs that
+        // kernel has already left; with many rows that launch measured slower (126.5 -> 129.5
+        // us a headline step) and the launch is an ordinary one
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.gridDim = dim3((unsigned)grid, 1, 1);
+        cfg.blockDim = dim3(kTcThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = p.dependent ? 1 : 0;
+        if (cudaLaunchKernelEx(&cfg, kern, map, static_cast<const T*>(R), scale_in, codes, scales,
+                               p, dev_status) != cudaSuccess)
+            return CK_ERR_CUDA;
         return cudaGetLastError() == cudaSuccess ? CK_OK : CK_ERR_CUDA;
     };
     return scale_in ? run(rq_tc_kernel<T, G, false, RG, P, PK>)

@@ -117,6 +117,9 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_sh;
+    // a kernel launched as this one's programmatic dependent (the next linear's stage 1) may
+    // set up on the SMs this kernel leaves: after every CTA holds its tensor memory
+    grid_dependents_launch();
 
     if (warp == WARP_TMA || warp == WARP_TMA2) {
         // ---------------------------------------------------------------- TMA: the whole range
