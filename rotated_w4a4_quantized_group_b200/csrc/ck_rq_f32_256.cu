@@ -14,8 +14,10 @@
 // block of rows; the partial sums stay in registers across the slices:
 //   - a block is RB whole rows (RB K / 256 <= 64 group-rows; a 3-D TMA box of 256 channels x
 //     K / 256 groups x RB rows) in one of two buffers, the next block's copy in flight;
-//   - warp w owns group-rows w, w + 8, .. of the block (at most eight), lane l the channels
-//     4 l .. 4 l + 3 and 128 + 4 l .. 128 + 4 l + 3 of each: 64 fp32 accumulators a thread.
+//   - warp w computes group-rows w, w + 8, .. of the block, NJ = ceil(group-rows / 8) <= 8 of
+//     them (a template parameter: the FMA step has no per-row branch; the buffers hold 8 NJ
+//     group-rows and the padding ones are never folded into a maximum or stored), lane l the
+//     channels 4 l .. 4 l + 3 and 128 + 4 l .. 128 + 4 l + 3 of each: 8 NJ fp32 accumulators.
 //     Per value of i a lane reads two 16-byte pieces of R's row (the warp's 32 lanes read two
 //     contiguous 512-byte runs: no bank conflict) and each x value once, broadcast to the
 //     warp, so shared memory serves about one 128-byte wavefront per six FMA instructions and
